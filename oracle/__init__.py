@@ -1,0 +1,153 @@
+"""fp64 CPU oracle for Ulysses sequence-parallel self-attention.
+
+TEST INFRASTRUCTURE: only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+product path (``video_dit_sequence_b200``) never imports it and shares no code
+with it.
+
+What it computes, and the passages it follows:
+
+* ``pack`` / ``unpack`` -- the token<->head all-to-all of the fal.ai page
+  "Generate video with WAN 2.2 across four GPUs", section "Splitting one
+  generation across four GPUs" (each GPU sees the full sequence for its share
+  of the heads, then the shards return).  Index formulas in ``sp_oracle.c``.
+* ``attention_rows`` -- the unsharded softmax(q K^T scale) V of one head,
+  two-pass exact softmax in fp64; the sequence-parallel result must equal it
+  for every degree (LTX-2 "Multi-GPU Inference" README, Capabilities table:
+  SP is numerically equivalent to single-GPU).
+
+Every function is pinned by ``tests/test_oracle_pins.py`` against closed
+forms, invariants, a worked example, brute force and numpy's fp64 routines.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sp_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libsp_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compiles sp_oracle.c into libsp_oracle.so next to it."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    i64 = ctypes.c_int64
+    vp = ctypes.c_void_p
+    for name in ("sp_oracle_pack", "sp_oracle_unpack"):
+        f = getattr(lib, name)
+        f.argtypes = [vp, vp, i64, i64, i64, i64, i64]
+        f.restype = ctypes.c_int
+    lib.sp_oracle_attention_rows.argtypes = [
+        vp, vp, vp, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp,
+        ctypes.c_int]
+    lib.sp_oracle_attention_rows.restype = ctypes.c_int
+    return lib
+
+
+def build_variant(src_text: str, out_path: str):
+    """Compiles a modified copy of the oracle source (used by the tests that
+    plant mistakes in the oracle to show the pins catch them) and binds it."""
+    c_path = out_path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-pthread",
+                           "-o", out_path, c_path, "-lm"])
+    return _bind(out_path)
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(build())
+    return _lib
+
+
+def _dims(N: int, P: int) -> Tuple[int, int]:
+    Nl = -(-N // P)
+    return Nl, Nl * P
+
+
+def pack(xs: np.ndarray, N: int, lib=None) -> np.ndarray:
+    """Seq-sharded [P][B][Nl][H][D] -> head-sharded [P][B][Np][Hl][D]."""
+    assert xs.dtype == np.uint16 and xs.ndim == 5
+    P, B, Nl, H, D = xs.shape
+    assert Nl == _dims(N, P)[0]
+    if H % P:
+        raise ValueError("the Ulysses degree must divide the head count")
+    xs = np.ascontiguousarray(xs)
+    out = np.empty((P, B, P * Nl, H // P, D), dtype=np.uint16)
+    rc = (lib or _load()).sp_oracle_pack(xs.ctypes.data, out.ctypes.data, B, N, H, D, P)
+    assert rc == 0
+    return out
+
+
+def unpack(oh: np.ndarray, N: int, H: int, lib=None) -> np.ndarray:
+    """Head-sharded [P][B][Np][Hl][D] -> seq-sharded [P][B][Nl][H][D]."""
+    assert oh.dtype == np.uint16 and oh.ndim == 5
+    P, B, Np, Hl, D = oh.shape
+    Nl, Np2 = _dims(N, P)
+    assert Np == Np2 and Hl * P == H
+    oh = np.ascontiguousarray(oh)
+    out = np.empty((P, B, Nl, H, D), dtype=np.uint16)
+    rc = (lib or _load()).sp_oracle_unpack(oh.ctypes.data, out.ctypes.data, B, N, H, D, P)
+    assert rc == 0
+    return out
+
+
+def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                   rows: np.ndarray, scale: float = 0.0,
+                   threads: Optional[int] = None, lib=None):
+    """fp64 attention output and LSE for query rows (b, h, i).
+
+    q, k, v: logical [B][N][H][D] bf16 bit patterns (uint16).
+    rows: int64 array [R][3] of (b, h, i).
+    Returns (O [R][D] float64, LSE [R] float64 natural log).
+    """
+    assert q.dtype == k.dtype == v.dtype == np.uint16
+    assert q.shape == k.shape == v.shape and q.ndim == 4
+    B, N, H, D = q.shape
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    R = rows.shape[0]
+    o = np.empty((R, D), dtype=np.float64)
+    lse = np.empty(R, dtype=np.float64)
+    if threads is None:
+        threads = max(1, len(os.sched_getaffinity(0)))
+    rc = (lib or _load()).sp_oracle_attention_rows(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, B, N, H, D, float(scale),
+        R, rows.ctypes.data, o.ctypes.data, lse.ctypes.data, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle attention failed ({rc})")
+    return o, lse
+
+
+def attention_full(q, k, v, scale: float = 0.0, threads: Optional[int] = None,
+                   lib=None):
+    """Every row of every (b, h); returns O [B][N][H][D] and LSE [B][H][N]."""
+    B, N, H, D = q.shape
+    b, h, i = np.meshgrid(np.arange(B), np.arange(H), np.arange(N), indexing="ij")
+    rows = np.stack([b.ravel(), h.ravel(), i.ravel()], axis=1)
+    o, lse = attention_rows(q, k, v, rows, scale, threads, lib)
+    O = o.reshape(B, H, N, D).transpose(0, 2, 1, 3)
+    return np.ascontiguousarray(O), lse.reshape(B, H, N)

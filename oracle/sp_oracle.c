@@ -1,0 +1,205 @@
+/*
+ * fp64 CPU oracle for Ulysses sequence-parallel self-attention.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark use this file.  It shares no code, header, table or
+ * helper with the CUDA path, and it is deliberately plain and slow: loops in
+ * the order of the definitions, fp64 arithmetic, no blocking or fusion.
+ *
+ * Sources of the definitions (web pages on the method):
+ *  - fal.ai, "Generate video with WAN 2.2 across four GPUs", section
+ *    "Splitting one generation across four GPUs": at every attention layer an
+ *    all-to-all trades tokens for heads, each GPU then sees the full sequence
+ *    for its share of the heads (10 of 40 at four GPUs), and the shards
+ *    return to their own GPUs afterwards.
+ *  - same page, section "Tuning cost and GPU count": the Ulysses degree must
+ *    divide the attention head count.
+ *  - LTX-2 "Multi-GPU Inference" README, Capabilities table: sequence
+ *    parallelism is numerically equivalent to single-GPU inference.  The
+ *    oracle therefore computes the unsharded (single-GPU) attention for every
+ *    degree P.
+ *
+ * Readings where the pages are silent (stated, not taken from the pages):
+ *  - layout: rank r holds tokens r*Nl .. r*Nl+Nl-1 of the sequence as
+ *    [B][Nl][H][D]; the P shards are stored one after another, [P][B][Nl][H][D];
+ *    Nl = ceil(N/P); token slots >= N are padding.
+ *  - head group j holds heads j*Hl .. j*Hl+Hl-1 (Hl = H/P); after the exchange
+ *    group j's buffer is [B][Np][Hl][D] with Np = P*Nl, chunks in rank order,
+ *    and the P group buffers are stored one after another.
+ *  - attention is non-causal softmax(q k^T * scale) v over all N tokens with
+ *    scale = 1/sqrt(D) unless given; no mask except the padding slots.
+ *
+ * Element type: bf16, given as its 16-bit pattern.  The oracle widens each
+ * bf16 value exactly to double.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_to_f64(uint16_t x) {
+    uint32_t u = (uint32_t)x << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/*
+ * Pack (sequence-sharded -> head-sharded): the send-buffer reorder plus the
+ * all-to-all of the page section "Splitting one generation across four GPUs".
+ * Rank r's tokens for head group j land in group j's buffer at token index
+ * r*Nl + n:
+ *     xh[j][b][r*Nl + n][hh][c] = xs[r][b][n][j*Hl + hh][c]
+ * xs: [P][B][Nl][H][D] words; xh: [P][B][P*Nl][Hl][D] words.
+ * Returns 0, or -1 when P does not divide H (page section "Tuning cost and
+ * GPU count").
+ */
+int sp_oracle_pack(const uint16_t *xs, uint16_t *xh, int64_t B, int64_t N,
+                   int64_t H, int64_t D, int64_t P) {
+    if (P < 1 || H % P != 0) return -1;
+    int64_t Hl = H / P, Nl = (N + P - 1) / P, Np = P * Nl;
+    for (int64_t j = 0; j < P; ++j)
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t r = 0; r < P; ++r)
+                for (int64_t n = 0; n < Nl; ++n)
+                    for (int64_t hh = 0; hh < Hl; ++hh)
+                        for (int64_t c = 0; c < D; ++c) {
+                            int64_t src = (((r * B + b) * Nl + n) * H + (j * Hl + hh)) * D + c;
+                            int64_t dst = (((j * B + b) * Np + (r * Nl + n)) * Hl + hh) * D + c;
+                            xh[dst] = xs[src];
+                        }
+    return 0;
+}
+
+/*
+ * Unpack (head-sharded -> sequence-sharded): "the shards return to their own
+ * GPUs" in the same page section; the inverse of the pack:
+ *     os[r][b][n][j*Hl + hh][c] = oh[j][b][r*Nl + n][hh][c]
+ */
+int sp_oracle_unpack(const uint16_t *oh, uint16_t *os, int64_t B, int64_t N,
+                     int64_t H, int64_t D, int64_t P) {
+    if (P < 1 || H % P != 0) return -1;
+    int64_t Hl = H / P, Nl = (N + P - 1) / P, Np = P * Nl;
+    for (int64_t r = 0; r < P; ++r)
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t n = 0; n < Nl; ++n)
+                for (int64_t j = 0; j < P; ++j)
+                    for (int64_t hh = 0; hh < Hl; ++hh)
+                        for (int64_t c = 0; c < D; ++c) {
+                            int64_t src = (((j * B + b) * Np + (r * Nl + n)) * Hl + hh) * D + c;
+                            int64_t dst = (((r * B + b) * Nl + n) * H + (j * Hl + hh)) * D + c;
+                            os[dst] = oh[src];
+                        }
+    return 0;
+}
+
+/*
+ * Attention for a list of query rows of the unsharded problem.
+ *
+ * For query row i of batch b and head h, with scores
+ *     s_k = scale * sum_c q[b][i][h][c] * k[b][k][h][c]      (k = 0 .. N-1)
+ * the two-pass exact softmax
+ *     m = max_k s_k,  w_k = exp(s_k - m),  l = sum_k w_k
+ * gives
+ *     o[c] = (sum_k w_k * v[b][k][h][c]) / l,   lse = m + ln(l).
+ * This is the plain definition softmax(q K^T scale) V of "attention over the
+ * full sequence" for one head; the sequence-parallel result equals it for
+ * every degree (LTX-2 README, Capabilities table).
+ *
+ * q, k, v: logical [B][N][H][D] bf16 words.  rows: nrows triples (b, h, i).
+ * out_o: nrows x D doubles; out_lse: nrows doubles (may be NULL).
+ */
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int64_t B, N, H, D;
+    double scale;
+    int64_t nrows;
+    const int64_t *rows;
+    double *out_o, *out_lse;
+    int64_t next;
+    pthread_mutex_t lock;
+    int failed;
+} attn_job_t;
+
+static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
+    int64_t b = J->rows[3 * r], h = J->rows[3 * r + 1], i = J->rows[3 * r + 2];
+    int64_t N = J->N, H = J->H, D = J->D;
+    const uint16_t *qi = J->q + ((b * N + i) * H + h) * D;
+    double m = -INFINITY;
+    for (int64_t kk = 0; kk < N; ++kk) {
+        const uint16_t *kr = J->k + ((b * N + kk) * H + h) * D;
+        double dot = 0.0;
+        for (int64_t c = 0; c < D; ++c) dot += bf16_to_f64(qi[c]) * bf16_to_f64(kr[c]);
+        s[kk] = J->scale * dot;
+        if (s[kk] > m) m = s[kk];
+    }
+    double *o = J->out_o + r * D;
+    for (int64_t c = 0; c < D; ++c) o[c] = 0.0;
+    double l = 0.0;
+    for (int64_t kk = 0; kk < N; ++kk) {
+        double w = exp(s[kk] - m);
+        l += w;
+        const uint16_t *vr = J->v + ((b * N + kk) * H + h) * D;
+        for (int64_t c = 0; c < D; ++c) o[c] += w * bf16_to_f64(vr[c]);
+    }
+    for (int64_t c = 0; c < D; ++c) o[c] /= l;
+    if (J->out_lse) J->out_lse[r] = m + log(l);
+}
+
+static void *attention_worker(void *arg) {
+    attn_job_t *J = (attn_job_t *)arg;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(J->N > 0 ? J->N : 1));
+    if (!s) {
+        pthread_mutex_lock(&J->lock);
+        J->failed = 1;
+        pthread_mutex_unlock(&J->lock);
+        return NULL;
+    }
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t r = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (r >= J->nrows) break;
+        attention_one_row(J, r, s);
+    }
+    free(s);
+    return NULL;
+}
+
+/* Returns 0 on success, -1 on bad arguments, -2 when out of host memory.
+ * Rows are handed to up to nthreads threads in list order; callers that sort
+ * the list by (b, h) let the threads share each head's K/V in cache. */
+int sp_oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             int64_t B, int64_t N, int64_t H, int64_t D, double scale,
+                             int64_t nrows, const int64_t *rows, double *out_o,
+                             double *out_lse, int nthreads) {
+    if (B < 1 || N < 1 || H < 1 || D < 1 || nrows < 0) return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 ||
+            rows[3 * r + 1] >= H || rows[3 * r + 2] < 0 || rows[3 * r + 2] >= N)
+            return -1;
+    }
+    if (!(scale > 0.0)) scale = 1.0 / sqrt((double)D);
+    attn_job_t J;
+    J.q = q; J.k = k; J.v = v;
+    J.B = B; J.N = N; J.H = H; J.D = D;
+    J.scale = scale;
+    J.nrows = nrows; J.rows = rows;
+    J.out_o = out_o; J.out_lse = out_lse;
+    J.next = 0;
+    J.failed = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 512) nthreads = 512;
+    pthread_t th[512];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t) {
+        if (pthread_create(&th[started], NULL, attention_worker, &J) != 0) break;
+        ++started;
+    }
+    attention_worker(&J);
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    pthread_mutex_destroy(&J.lock);
+    return J.failed ? -2 : 0;
+}

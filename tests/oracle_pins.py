@@ -1,0 +1,264 @@
+"""Checks that pin the fp64 oracle to facts other than its own code.
+
+Each check takes an optional ``lib`` (a bound oracle library) so that the
+mutant tests can run the same checks against copies of the oracle with a
+planted mistake and show that some check fails.  Every check raises
+AssertionError on failure.
+
+Facts used:
+* page facts: after the exchange, head group j holds the full sequence for
+  heads j*Hl .. j*Hl+Hl-1 (fal.ai WAN 2.2 page, "Splitting one generation
+  across four GPUs"); the degree must divide the head count ("Tuning cost and
+  GPU count"); the shards return to their owners afterwards.
+* library routines: numpy's reshape/transpose for the permutation and
+  numpy fp64 matmul/exp for softmax(q K^T scale) V on small problems;
+  scipy's logsumexp for the LSE.
+* closed forms and invariants of softmax attention: rows of the softmax sum
+  to one; V = 1 gives O = 1; Q = 0 gives the mean of V; N = 1 gives V; a
+  dominant key selects its value row; invariance under a key permutation and
+  under a common shift of all keys; linearity in V; a two-token example.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import logsumexp
+
+import oracle
+import synth
+
+RNG_SEED = 1234
+
+
+def _codes(shape, rng):
+    """Distinct-ish 16-bit payloads; pack/unpack move words without reading
+    them, so any bit pattern serves as a tag."""
+    n = int(np.prod(shape))
+    base = rng.permutation(65536)[: min(n, 65536)].astype(np.uint16)
+    return np.resize(base, n).reshape(shape)
+
+
+def _small_ints_bf16(shape, rng, lo=-3, hi=4):
+    """Small integers, exact in bf16 and closed under the sums the checks use."""
+    return synth.f32_to_bf16(rng.integers(lo, hi, size=shape).astype(np.float32))
+
+
+def _bf16_normal(shape, rng, mul=1.0):
+    return synth.f32_to_bf16((rng.standard_normal(shape) * mul).astype(np.float32))
+
+
+def _f64(x):
+    return synth.bf16_to_f32(x).astype(np.float64)
+
+
+PACK_SHAPES = [(1, 16, 4, 8, 2), (2, 13, 6, 8, 3), (3, 10, 8, 16, 4),
+               (1, 7, 4, 8, 4), (2, 9, 8, 8, 8), (1, 5, 2, 8, 1)]
+
+
+def check_pack_heads_for_full_sequence(lib=None):
+    """Group j's buffer holds the full sequence for heads j*Hl..(j+1)*Hl-1,
+    tokens in order; padding slots stay zero."""
+    rng = np.random.default_rng(RNG_SEED)
+    for (B, N, H, D, P) in PACK_SHAPES:
+        X = _codes((B, N, H, D), rng)
+        X[X == 0] = 1  # keep zero for the padding check
+        xh = oracle.pack(synth.to_seq_shards(X, P), N, lib=lib)
+        Hl = H // P
+        for j in range(P):
+            assert np.array_equal(xh[j][:, :N], X[:, :, j * Hl:(j + 1) * Hl]), (B, N, H, D, P, j)
+            assert not xh[j][:, N:].any()
+
+
+def check_pack_matches_numpy_transpose(lib=None):
+    """Library formulation: per-rank shards viewed as [P][B][Nl][P][Hl][D],
+    moved to [P(group)][B][P(rank)][Nl][Hl][D] by numpy."""
+    rng = np.random.default_rng(RNG_SEED + 1)
+    for (B, N, H, D, P) in PACK_SHAPES:
+        Nl = -(-N // P)
+        xs = _codes((P, B, Nl, H, D), rng)
+        ref = xs.reshape(P, B, Nl, P, H // P, D).transpose(3, 1, 0, 2, 4, 5)
+        ref = ref.reshape(P, B, P * Nl, H // P, D)
+        assert np.array_equal(oracle.pack(xs, N, lib=lib), ref)
+
+
+def check_unpack_returns_shards(lib=None):
+    """The shards return to their owners: unpack(pack(x)) = x, and a
+    head-sharded result built from a logical tensor unpacks to its shards."""
+    rng = np.random.default_rng(RNG_SEED + 2)
+    for (B, N, H, D, P) in PACK_SHAPES:
+        Nl = -(-N // P)
+        xs = _codes((P, B, Nl, H, D), rng)
+        assert np.array_equal(oracle.unpack(oracle.pack(xs, N, lib=lib), N, H, lib=lib), xs)
+        X = _codes((B, N, H, D), rng)
+        Hl = H // P
+        oh = np.zeros((P, B, P * Nl, Hl, D), dtype=np.uint16)
+        for j in range(P):
+            oh[j][:, :N] = X[:, :, j * Hl:(j + 1) * Hl]
+        os_ = oracle.unpack(oh, N, H, lib=lib)
+        assert np.array_equal(synth.from_seq_shards(os_, N), X)
+        assert np.array_equal(os_, synth.to_seq_shards(X, P))
+
+
+def check_pack_degree_one_is_copy(lib=None):
+    rng = np.random.default_rng(RNG_SEED + 3)
+    xs = _codes((1, 2, 11, 4, 8), rng)
+    assert np.array_equal(oracle.pack(xs, 11, lib=lib), xs)
+    assert np.array_equal(oracle.unpack(xs, 11, 4, lib=lib), xs)
+
+
+# ---------------------------------------------------------------- attention
+
+def _np_attention(q, k, v, scale=None):
+    """numpy fp64 softmax(q K^T scale) V per (b, h); returns O, LSE."""
+    qf, kf, vf = _f64(q), _f64(k), _f64(v)
+    B, N, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    O = np.empty((B, N, H, D))
+    L = np.empty((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            s = (qf[b, :, h] @ kf[b, :, h].T) * scale
+            L[b, h] = logsumexp(s, axis=1)
+            p = np.exp(s - L[b, h][:, None])
+            O[b, :, h] = p @ vf[b, :, h]
+    return O, L
+
+
+ATTN_SHAPES = [(1, 1, 1, 16), (2, 37, 3, 16), (1, 130, 2, 64), (1, 64, 2, 128)]
+
+
+def check_attention_matches_numpy(lib=None):
+    rng = np.random.default_rng(RNG_SEED + 10)
+    for (B, N, H, D) in ATTN_SHAPES:
+        q, k, v = (_bf16_normal((B, N, H, D), rng, m) for m in (1.0, 1.5, 1.0))
+        O, L = oracle.attention_full(q, k, v, lib=lib, threads=2)
+        On, Ln = _np_attention(q, k, v)
+        assert np.max(np.abs(O - On)) < 1e-12, (B, N, H, D)
+        assert np.max(np.abs(L - Ln)) < 1e-12, (B, N, H, D)
+
+
+def check_softmax_rows_sum_to_one(lib=None):
+    """sum_k exp(s_ik - LSE_i) = 1 with s computed by numpy."""
+    rng = np.random.default_rng(RNG_SEED + 11)
+    B, N, H, D = 1, 200, 2, 32
+    q, k, v = (_bf16_normal((B, N, H, D), rng, 2.0) for _ in range(3))
+    _, L = oracle.attention_full(q, k, v, lib=lib, threads=2)
+    qf, kf = _f64(q), _f64(k)
+    for h in range(H):
+        s = (qf[0, :, h] @ kf[0, :, h].T) / math.sqrt(D)
+        tot = np.exp(s - L[0, h][:, None]).sum(axis=1)
+        assert np.max(np.abs(tot - 1.0)) < 1e-12
+
+
+def check_closed_forms(lib=None):
+    rng = np.random.default_rng(RNG_SEED + 12)
+    B, N, H, D = 1, 50, 2, 16
+    q, k = _bf16_normal((B, N, H, D), rng), _bf16_normal((B, N, H, D), rng)
+    v = _bf16_normal((B, N, H, D), rng)
+    # V = 1 -> O = 1 for every row.
+    ones = synth.f32_to_bf16(np.ones((B, N, H, D), dtype=np.float32))
+    O, _ = oracle.attention_full(q, k, ones, lib=lib, threads=2)
+    assert np.max(np.abs(O - 1.0)) < 1e-13
+    # Q = 0 -> uniform weights -> O = mean_k V and LSE = ln N.
+    zeros = np.zeros((B, N, H, D), dtype=np.uint16)
+    O, L = oracle.attention_full(zeros, k, v, lib=lib, threads=2)
+    mean = _f64(v).mean(axis=1)  # [B][H][D]
+    assert np.max(np.abs(O - mean[:, None])) < 1e-13
+    assert np.max(np.abs(L - math.log(N))) < 1e-13
+    # N = 1 -> O = V.
+    O, L = oracle.attention_full(q[:, :1], k[:, :1], v[:, :1], lib=lib, threads=1)
+    assert np.array_equal(O, _f64(v[:, :1]))
+
+
+def check_dominant_key(lib=None):
+    """A key aligned with q and scaled far above the rest takes all weight."""
+    rng = np.random.default_rng(RNG_SEED + 13)
+    B, N, H, D = 1, 40, 1, 16
+    q = _small_ints_bf16((B, N, H, D), rng, 1, 3)          # entries 1..2
+    k = _small_ints_bf16((B, N, H, D), rng, -1, 2)          # entries -1..1
+    v = _bf16_normal((B, N, H, D), rng)
+    star = 17
+    k[0, star, 0] = synth.f32_to_bf16(np.full(D, 64.0, dtype=np.float32))
+    O, _ = oracle.attention_full(q, k, v, lib=lib, threads=2)
+    # logit gap >= (64*16 - 2*16)/4 = 248 -> other weights < N*e^-248.
+    assert np.max(np.abs(O[0, :, 0] - _f64(v[0, star, 0])[None])) < 1e-12
+
+
+def check_invariances(lib=None):
+    rng = np.random.default_rng(RNG_SEED + 14)
+    B, N, H, D = 2, 33, 2, 16
+    q = _small_ints_bf16((B, N, H, D), rng)
+    k = _small_ints_bf16((B, N, H, D), rng)
+    v1 = _small_ints_bf16((B, N, H, D), rng)
+    v2 = _small_ints_bf16((B, N, H, D), rng)
+    scale = 0.125
+    O, L = oracle.attention_full(q, k, v1, scale, lib=lib, threads=2)
+    # Permuting the key/value tokens together changes nothing.
+    perm = rng.permutation(N)
+    Op, _ = oracle.attention_full(q, k[:, perm], v1[:, perm], scale, lib=lib, threads=2)
+    assert np.max(np.abs(Op - O)) < 1e-12
+    # Permuting the queries permutes the rows.
+    Oq, _ = oracle.attention_full(q[:, perm], k, v1, scale, lib=lib, threads=2)
+    assert np.max(np.abs(Oq - O[:, perm])) < 1e-12
+    # A common shift u of all keys adds scale*q.u to every score of a row:
+    # O unchanged, LSE shifted by exactly that amount.
+    u = rng.integers(-2, 3, size=D).astype(np.float32)
+    ks = synth.f32_to_bf16(synth.bf16_to_f32(k) + u)
+    Os, Ls = oracle.attention_full(q, ks, v1, scale, lib=lib, threads=2)
+    assert np.max(np.abs(Os - O)) < 1e-12
+    shift = scale * np.einsum("bnhd,d->bhn", _f64(q), u.astype(np.float64))
+    assert np.max(np.abs(Ls - (L + shift))) < 1e-11
+    # Linear in V.
+    v12 = synth.f32_to_bf16(synth.bf16_to_f32(v1) + synth.bf16_to_f32(v2))
+    O2, _ = oracle.attention_full(q, k, v2, scale, lib=lib, threads=2)
+    O12, _ = oracle.attention_full(q, k, v12, scale, lib=lib, threads=2)
+    assert np.max(np.abs(O12 - (O + O2))) < 1e-12
+    # Scores scale with K: (2K, scale/2) gives the same result.
+    k2 = synth.f32_to_bf16(synth.bf16_to_f32(k) * 2)
+    Ok, Lk = oracle.attention_full(q, k2, v1, scale / 2, lib=lib, threads=2)
+    assert np.max(np.abs(Ok - O)) < 1e-12 and np.max(np.abs(Lk - L)) < 1e-12
+    # scale <= 0 means 1/sqrt(D).
+    Od, _ = oracle.attention_full(q, k, v1, 0.0, lib=lib, threads=2)
+    Oe, _ = oracle.attention_full(q, k, v1, 1.0 / math.sqrt(D), lib=lib, threads=2)
+    assert np.array_equal(Od, Oe)
+
+
+def check_two_token_example(lib=None):
+    """Worked by hand: D = 4, scale = 1/2, one head.  q = (2,0,0,0),
+    k0 = (1,0,0,0), k1 = (0,0,0,0): scores (1, 0), weights e/(e+1) and
+    1/(e+1); v0 = (1,2,3,4), v1 = (-1,0,0,8)."""
+    f = lambda a: synth.f32_to_bf16(np.array(a, dtype=np.float32))
+    q = f([[[[2, 0, 0, 0]], [[0, 0, 0, 0]]]])
+    k = f([[[[1, 0, 0, 0]], [[0, 0, 0, 0]]]])
+    v = f([[[[1, 2, 3, 4]], [[-1, 0, 0, 8]]]])
+    O, L = oracle.attention_full(q, k, v, lib=lib, threads=1)
+    e = math.e
+    w0, w1 = e / (e + 1), 1 / (e + 1)
+    want0 = [w0 * 1 + w1 * -1, w0 * 2, w0 * 3, w0 * 4 + w1 * 8]
+    assert np.max(np.abs(O[0, 0, 0] - want0)) < 1e-15
+    assert abs(L[0, 0, 0] - math.log(e + 1)) < 1e-15
+    # query 1 is all zeros: uniform over the two keys.
+    assert np.max(np.abs(O[0, 1, 0] - [0, 1, 1.5, 6])) < 1e-15
+    assert abs(L[0, 0, 1] - math.log(2)) < 1e-15
+
+
+def check_rows_api(lib=None):
+    """attention_rows on a subset equals the same rows of attention_full."""
+    rng = np.random.default_rng(RNG_SEED + 15)
+    B, N, H, D = 2, 70, 3, 16
+    q, k, v = (_bf16_normal((B, N, H, D), rng) for _ in range(3))
+    O, L = oracle.attention_full(q, k, v, lib=lib, threads=3)
+    rows = np.array([[1, 2, 69], [0, 0, 0], [1, 0, 35]], dtype=np.int64)
+    o, l = oracle.attention_rows(q, k, v, rows, lib=lib, threads=2)
+    for r, (b, h, i) in enumerate(rows):
+        assert np.array_equal(o[r], O[b, i, h]) and l[r] == L[b, h, i]
+
+
+PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
+               check_unpack_returns_shards, check_pack_degree_one_is_copy]
+ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one,
+                    check_closed_forms, check_dominant_key, check_invariances,
+                    check_two_token_example, check_rows_api]
+ALL_CHECKS = PACK_CHECKS + ATTENTION_CHECKS
