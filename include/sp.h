@@ -1,0 +1,137 @@
+/*
+ * sp.h -- C ABI of libsp, Ulysses sequence-parallel self-attention on one
+ * B200 (sm_100a) with P virtual ranks.
+ *
+ * The method (fal.ai, "Generate video with WAN 2.2 across four GPUs",
+ * section "Splitting one generation across four GPUs"): the token sequence
+ * of one generation is split across P ranks; at each attention layer an
+ * all-to-all trades tokens for heads so that every rank sees the full
+ * sequence for H/P of the H heads, attention runs per head over all tokens,
+ * and the outputs return to the ranks that own the tokens.  The result is
+ * numerically the single-GPU result (LTX-2 "Multi-GPU Inference" README,
+ * Capabilities table).  On one GPU the exchange is a permutation in HBM
+ * (sp_pack / sp_unpack) or disappears into the attention kernel's addressing
+ * (sp_attention_seqsharded).
+ *
+ * Notation: B batch, N true token count, H heads, D head dim, P degree,
+ * Hl = H/P, Nl = ceil(N/P), Np = P*Nl.  Elements are bf16 (16-bit words).
+ *
+ * Layouts (all dense, row-major, innermost last):
+ *   sequence-sharded  xs : [P][B][Nl][H][D]   rank r holds tokens r*Nl .. r*Nl+Nl-1
+ *   head-sharded      xh : [P][B][Np][Hl][D]  group j holds heads j*Hl .. j*Hl+Hl-1
+ *   log-sum-exp      lse : [B][H][Np] fp32 (natural log), optional
+ * Token slots t >= N are padding: they must be zero in xs for the pack to be
+ * an exact copy of a zero-padded sequence; attention ignores them as keys and
+ * writes zero output rows (lse = -inf) for them as queries.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates no device
+ * memory and keeps no pointer after a call returns.
+ * Asynchrony: every call that takes a stream only enqueues work on it (NULL
+ * means the legacy default stream) and does not synchronise, except
+ * sp_device_status.
+ * Errors: argument errors are returned before anything is enqueued and leave
+ * the outputs untouched.  A failed launch returns SP_ERR_CUDA.  A kernel that
+ * gives up on a bounded wait records SP_ERR_TIMEOUT in a device status word,
+ * which sp_device_status reports.  Nothing throws across this ABI.
+ * Requirements: device pointers 16-byte aligned; D in {64, 128};
+ * H % P == 0; N >= 1; B >= 1; element counts below 2^31 per tensor row
+ * index space.
+ */
+#ifndef SP_H_
+#define SP_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SP_OK = 0,
+  SP_ERR_NULL = 1,                /* a required pointer is NULL */
+  SP_ERR_SHAPE = 2,               /* B, N, H, D or P out of range */
+  SP_ERR_HEADS_NOT_DIVISIBLE = 3, /* H % P != 0 */
+  SP_ERR_ALIGN = 4,               /* a device pointer is not 16-byte aligned */
+  SP_ERR_UNSUPPORTED_D = 5,       /* D not in {64, 128} */
+  SP_ERR_CUDA = 6,                /* a CUDA runtime/driver call failed */
+  SP_ERR_TIMEOUT = 7              /* a kernel gave up on a bounded wait */
+} sp_status;
+
+/* One problem.  scale <= 0 selects 1/sqrt(D). */
+typedef struct {
+  int32_t B, N, H, D, P;
+  float scale;
+} sp_shape;
+
+/* Np = ceil(N/P) * P, the padded token count of both layouts; -1 when
+ * N < 1 or P < 1. */
+int64_t sp_padded_tokens(int32_t N, int32_t P);
+
+/* Validates a shape against the rules above; the degree rule ("the Ulysses
+ * degree must divide the attention head count", fal.ai page, section
+ * "Tuning cost and GPU count") gives SP_ERR_HEADS_NOT_DIVISIBLE. */
+sp_status sp_check_shape(const sp_shape *shape);
+
+/* Pack: sequence-sharded -> head-sharded, the send reorder plus all-to-all
+ * of the page section "Splitting one generation across four GPUs":
+ *   xh[j][b][r*Nl + n][hh][c] = xs[r][b][n][j*Hl + hh][c]
+ * xs: device, [P][B][Nl][H][D] bf16, read only.  xh: device,
+ * [P][B][Np][Hl][D] bf16, written in full.  Bit-exact copy.  xs and xh must
+ * not overlap. */
+sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream);
+
+/* Unpack: head-sharded -> sequence-sharded ("the shards return to their own
+ * GPUs", same section); the inverse of sp_pack:
+ *   os[r][b][n][j*Hl + hh][c] = oh[j][b][r*Nl + n][hh][c]
+ * oh: device, [P][B][Np][Hl][D] bf16, read only.  os: device,
+ * [P][B][Nl][H][D] bf16, written in full.  Bit-exact copy. */
+sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *stream);
+
+/* Attention per head group on head-sharded tensors: for every batch b,
+ * group j, local head hh (global head h = j*Hl + hh) and query token i < N,
+ *   oh[j][b][i][hh] = sum_{k<N} softmax_k(q_i . k_k * scale) v_k
+ * non-causal, keys k >= N masked; "each GPU sees the full sequence" for its
+ * heads (same section).  Accumulation in fp32, probabilities rounded to
+ * bf16 before the P*V product, output rounded to nearest-even bf16.  Rows
+ * i in [N, Np) are written as zero.  The result for a given (b, h, i) does
+ * not depend on P.
+ * qh, kh, vh: device [P][B][Np][Hl][D] bf16, read only.  oh: device, same
+ * shape, written.  lse: device fp32 [B][H][Np] or NULL. */
+sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh,
+                       float *lse, const sp_shape *shape, void *stream);
+
+/* Fused sequence-parallel attention: sp_unpack(sp_attention(sp_pack(q),
+ * sp_pack(k), sp_pack(v))) in one kernel that reads Q/K/V tiles straight
+ * from the sequence-sharded buffers and writes O into the sequence-sharded
+ * layout; no intermediate buffers.  Bit-identical to the three-call path.
+ * qs, ks, vs: device [P][B][Nl][H][D] bf16, read only.  os: device, same
+ * shape, written.  lse: device fp32 [B][H][Np] or NULL.  Supports B == 1 or
+ * P == 1 (the layouts in which a token tile is one strided block); other
+ * shapes return SP_ERR_SHAPE (use the three-call path). */
+sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs,
+                                  void *os, float *lse, const sp_shape *shape,
+                                  void *stream);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * SP_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
+ * SP_ERR_CUDA if the stream reports an error, else SP_OK. */
+sp_status sp_device_status(void *stream);
+
+/* Self-test of the bounded waits: enqueues one small kernel that waits on a
+ * shared-memory barrier nothing will complete, with a limit of limit_ns
+ * nanoseconds (clamped to 1 s).  The wait runs out, the kernel records
+ * SP_ERR_TIMEOUT in the device status word and returns; the next
+ * sp_device_status call reports it.  No GPU fault is involved. */
+sp_status sp_selftest_wait_timeout(uint64_t limit_ns, void *stream);
+
+/* Number of kernels this library has enqueued since it was loaded. */
+uint64_t sp_launch_count(void);
+
+/* Static description of a status code; never NULL. */
+const char *sp_status_str(sp_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP_H_ */

@@ -1,0 +1,110 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+symbol include/sp.h declares, and its host-side checks reject bad arguments
+before anything is enqueued (no compute call is made here)."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+import video_dit_sequence_b200 as sp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from video_dit_sequence_b200 import build
+    build.build()
+    return sp.load()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(sp_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert names >= {"sp_pack", "sp_unpack", "sp_attention", "sp_attention_seqsharded"}
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(sp.EXPORTED) == names
+
+
+def test_padded_tokens(lib):
+    assert sp.padded_tokens(75600, 4) == 75600
+    assert sp.padded_tokens(75601, 8) == 75608
+    assert sp.padded_tokens(75601, 2) == 75602
+    assert sp.padded_tokens(1024, 2) == 1024
+    assert sp.padded_tokens(0, 2) == -1 and sp.padded_tokens(5, 0) == -1
+
+
+def test_degree_rule_golden(lib):
+    with open(os.path.join(ROOT, "tests", "golden", "degree_rule.json")) as f:
+        g = json.load(f)
+    for c in g["valid"]:
+        assert sp.check_shape(sp.Shape(1, 4096, c["heads"], 128, c["degree"])) == sp.SP_OK
+        assert sp.Shape(1, 4096, c["heads"], 128, c["degree"]).Hl == c["heads_per_rank"]
+    for c in g["invalid"]:
+        assert sp.check_shape(sp.Shape(1, 4096, c["heads"], 128, c["degree"])) == \
+            sp.SP_ERR_HEADS_NOT_DIVISIBLE
+
+
+def test_shape_errors(lib):
+    ok = sp.Shape(1, 75600, 40, 128, 4)
+    assert sp.check_shape(ok) == sp.SP_OK
+    assert sp.check_shape(sp.Shape(1, 0, 40, 128, 4)) == sp.SP_ERR_SHAPE
+    assert sp.check_shape(sp.Shape(0, 10, 40, 128, 4)) == sp.SP_ERR_SHAPE
+    assert sp.check_shape(sp.Shape(1, 10, 40, 96, 4)) == sp.SP_ERR_UNSUPPORTED_D
+    assert sp.check_shape(sp.Shape(1, 10, 40, 64, 3)) == sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    assert lib.sp_check_shape(None) == sp.SP_ERR_NULL
+    for code in range(8):
+        assert isinstance(sp.status_str(code), str) and sp.status_str(code)
+
+
+def _call(fn, *ptrs, shape):
+    s = shape.c()
+    return fn(*[ctypes.c_void_p(p) if p else None for p in ptrs], ctypes.byref(s), None)
+
+
+def test_argument_errors_return_before_launch(lib):
+    """Fake device addresses are only checked, never touched: every one of
+    these calls must return its error without reaching the GPU."""
+    shape = sp.Shape(1, 1024, 4, 64, 2)
+    A, B_ = 0x10000, 0x20000
+    assert _call(lib.sp_pack, 0, B_, shape=shape) == sp.SP_ERR_NULL
+    assert _call(lib.sp_unpack, A, 0, shape=shape) == sp.SP_ERR_NULL
+    assert _call(lib.sp_pack, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN
+    assert _call(lib.sp_unpack, A, B_ + 2, shape=shape) == sp.SP_ERR_ALIGN
+    bad = sp.Shape(1, 1024, 6, 64, 4)
+    assert _call(lib.sp_pack, A, B_, shape=bad) == sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    s = shape.c()
+    att = lambda fn, q, k, v, o, lse=None, shp=shape: fn(
+        *[ctypes.c_void_p(x) if x else None for x in (q, k, v, o, lse)],
+        ctypes.byref(shp.c()), None)
+    for fn in (lib.sp_attention, lib.sp_attention_seqsharded):
+        assert att(fn, A, A, 0, B_) == sp.SP_ERR_NULL
+        assert att(fn, A, A, A + 4, B_) == sp.SP_ERR_ALIGN
+        assert att(fn, A, A, A, B_, 0x30002) == sp.SP_ERR_ALIGN
+        assert att(fn, A, A, A, B_, shp=sp.Shape(1, 1024, 4, 80, 2)) == sp.SP_ERR_UNSUPPORTED_D
+        assert att(fn, A, A, A, B_, shp=sp.Shape(1, 1024, 4, 64, 3)) == \
+            sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    # the fused kernel covers B == 1 or P == 1
+    assert att(lib.sp_attention_seqsharded, A, A, A, B_, shp=sp.Shape(2, 1024, 4, 64, 2)) == \
+        sp.SP_ERR_SHAPE
+    assert lib.sp_launch_count() == 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    torch = pytest.importorskip("torch")
+    shape = sp.Shape(1, 16, 2, 64, 2)
+    x = torch.zeros(shape.seq_sharded, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        sp.pack(x, x, shape)

@@ -1,0 +1,285 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Permutations: bit-exact.  Attention: within the bars in gpu_util, and
+bit-identical across degrees P and between the fused and the three-call
+path.  Large problems check sampled query rows (always including rows 0,
+N-1 and every shard boundary) in the launch configuration the benchmark
+times (the fused sequence-sharded kernel)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import assert_parity, compare, to_dev, to_host
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, never run there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import video_dit_sequence_b200 as sp  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    sp.load()
+    yield
+    assert sp.device_status() == sp.SP_OK
+
+
+def _status_ok():
+    assert sp.device_status() == sp.SP_OK
+
+
+def _random_logical(B, N, H, D, seed, k_mul=1.0):
+    cfg = synth.Config("t", synth.Shape(B, N, H, D, 1), seed=seed, k_mul=k_mul)
+    return synth.qkv_logical(cfg)
+
+
+def _run_fused(q, k, v, P, lse=False):
+    B, N, H, D = q.shape
+    shape = sp.Shape(B, N, H, D, P)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    os_ = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    l = torch.full(shape.lse_shape, float("nan"), dtype=torch.float32, device="cuda") if lse else None
+    sp.attention_seqsharded(qs, ks, vs, os_, shape, lse=l)
+    _status_ok()
+    return to_host(os_), (l.cpu().numpy() if lse else None)
+
+
+def _run_unfused(q, k, v, P, lse=False):
+    B, N, H, D = q.shape
+    shape = sp.Shape(B, N, H, D, P)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    hs = shape.head_sharded
+    qh, kh, vh = (torch.empty(hs, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    oh = torch.full(hs, float("nan"), dtype=torch.bfloat16, device="cuda")
+    os_ = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    l = torch.full(shape.lse_shape, float("nan"), dtype=torch.float32, device="cuda") if lse else None
+    sp.pack(qs, qh, shape)
+    sp.pack(ks, kh, shape)
+    sp.pack(vs, vh, shape)
+    sp.attention(qh, kh, vh, oh, shape, lse=l)
+    sp.unpack(oh, os_, shape)
+    _status_ok()
+    return to_host(os_), (l.cpu().numpy() if lse else None)
+
+
+def _rows_all(B, N, H):
+    b, h, i = np.meshgrid(np.arange(B), np.arange(H), np.arange(N), indexing="ij")
+    return np.stack([b.ravel(), h.ravel(), i.ravel()], axis=1)
+
+
+def _check_rows(os_host, q, k, v, rows, P, where):
+    B, N, H, D = q.shape
+    O = synth.from_seq_shards(os_host.reshape(P, B, -1, H, D), N)
+    ref, _ = oracle.attention_rows(q, k, v, rows)
+    got = O[rows[:, 0], rows[:, 2], rows[:, 1]]
+    m = compare(got, ref, rows[:, 1])
+    assert_parity(m, where)
+    return m
+
+
+# ------------------------------------------------------------------ permutations
+
+PERM_SHAPES = [(1, 1024, 4, 64, 2), (2, 1000, 8, 64, 4), (3, 77, 6, 128, 3),
+               (1, 4096, 40, 128, 8), (1, 75601 // 50, 40, 128, 8), (2, 9, 8, 128, 8),
+               (1, 300, 40, 128, 1), (4, 130, 2, 64, 2)]
+
+
+@pytest.mark.parametrize("B,N,H,D,P", PERM_SHAPES)
+def test_pack_unpack_bit_exact(B, N, H, D, P):
+    shape = sp.Shape(B, N, H, D, P)
+    X = synth.normal_bf16(100 + N, 0, 0, B * N * H * D).reshape(B, N, H, D)
+    xs = synth.to_seq_shards(X, P)
+    want_h = oracle.pack(xs, N)
+    d_xs = to_dev(xs)
+    d_xh = torch.full(shape.head_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.pack(d_xs, d_xh, shape)
+    got_h = to_host(d_xh)
+    assert np.array_equal(got_h.reshape(want_h.shape), want_h)
+    # unpack of an arbitrary head-sharded buffer
+    oh = synth.normal_bf16(200 + N, 1, 0, int(np.prod(shape.head_sharded))).reshape(shape.head_sharded)
+    want_s = oracle.unpack(oh, N, H)
+    d_os = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.unpack(to_dev(oh), d_os, shape)
+    assert np.array_equal(to_host(d_os).reshape(want_s.shape), want_s)
+    # and the round trip on the device
+    d_back = torch.empty_like(d_xs)
+    sp.unpack(d_xh, d_back, shape)
+    assert torch.equal(d_back.view(torch.int16), d_xs.view(torch.int16))
+    _status_ok()
+
+
+@pytest.mark.parametrize("name", ["720p", "sweep-N75601-P8"])
+def test_pack_full_size_bit_exact(name):
+    cfg = synth.CONFIGS.get(name) or synth.sweep_config(75601, 8)
+    s = cfg.shape
+    shape = sp.Shape(s.B, s.N, s.H, s.D, s.P)
+    q = synth.logical_tensor(cfg, synth.TID_Q)
+    xs = synth.to_seq_shards(q, s.P)
+    want = oracle.pack(xs, s.N)
+    d_xh = torch.empty(shape.head_sharded, dtype=torch.bfloat16, device="cuda")
+    sp.pack(to_dev(xs), d_xh, shape)
+    assert np.array_equal(to_host(d_xh).reshape(want.shape), want)
+    want_s = oracle.unpack(want, s.N, s.H)
+    d_os = torch.empty(shape.seq_sharded, dtype=torch.bfloat16, device="cuda")
+    sp.unpack(d_xh, d_os, shape)
+    assert np.array_equal(to_host(d_os).reshape(want_s.shape), want_s)
+    _status_ok()
+
+
+# ------------------------------------------------------------------ attention, small
+
+def test_tiny_config_every_row():
+    cfg = synth.CONFIGS["tiny"]
+    s = cfg.shape
+    q, k, v = synth.qkv_logical(cfg)
+    fused, lse_f = _run_fused(q, k, v, s.P, lse=True)
+    unfused, lse_u = _run_unfused(q, k, v, s.P, lse=True)
+    assert np.array_equal(fused, unfused)
+    assert np.array_equal(lse_f, lse_u)
+    rows = _rows_all(s.B, s.N, s.H)
+    _check_rows(fused, q, k, v, rows, s.P, "tiny")
+    _, lse_ref = oracle.attention_full(q, k, v)
+    assert np.max(np.abs(lse_f[:, :, : s.N] - lse_ref)) < 1e-2
+
+
+@pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 255, 256, 257, 383, 513])
+@pytest.mark.parametrize("D", [64, 128])
+def test_ragged_lengths(N, D):
+    B, H, P = 1, 2, 2
+    q, k, v = _random_logical(B, N, H, D, seed=N * 7 + D)
+    out, lse = _run_fused(q, k, v, P, lse=True)
+    _check_rows(out, q, k, v, _rows_all(B, N, H), P, f"N={N} D={D}")
+    O_all = out.reshape(P, B, -1, H, D).transpose(1, 0, 2, 3, 4).reshape(B, -1, H, D)
+    assert not O_all[:, N:].any(), "padding rows must be zero"
+    assert np.all(np.isneginf(lse[:, :, N:]))
+    un, lse_u = _run_unfused(q, k, v, P, lse=True)
+    assert np.array_equal(out, un) and np.array_equal(lse, lse_u)
+
+
+def test_batch_and_degree_one_fused_and_unfused():
+    B, N, H, D = 3, 300, 4, 128
+    q, k, v = _random_logical(B, N, H, D, seed=77)
+    f1, _ = _run_fused(q, k, v, 1)
+    u2, _ = _run_unfused(q, k, v, 2)
+    u1, _ = _run_unfused(q, k, v, 1)
+    assert np.array_equal(f1, u1)
+    assert np.array_equal(synth.from_seq_shards(u2.reshape(2, B, -1, H, D), N),
+                          synth.from_seq_shards(f1.reshape(1, B, -1, H, D), N))
+    _check_rows(f1, q, k, v, _rows_all(B, N, H), 1, "B=3")
+
+
+@pytest.mark.parametrize("N", [1000, 4096])
+def test_degrees_bit_identical(N):
+    """SP output equals single-GPU output bit for bit, for every degree."""
+    B, H, D = 1, 8, 128
+    q, k, v = _random_logical(B, N, H, D, seed=N)
+    ref, _ = _run_fused(q, k, v, 1)
+    ref_l = synth.from_seq_shards(ref.reshape(1, B, -1, H, D), N)
+    for P in (2, 4, 8):
+        for run in (_run_fused, _run_unfused):
+            out, _ = run(q, k, v, P)
+            got = synth.from_seq_shards(out.reshape(P, B, -1, H, D), N)
+            assert np.array_equal(got, ref_l), (P, run.__name__)
+    rows = synth.sampled_rows(synth.Config("x", synth.Shape(B, N, H, D, 8), seed=3), 64)
+    rr = np.array([(0, h, i) for h in range(H) for i in rows], dtype=np.int64)
+    _check_rows(ref, q, k, v, rr, 1, f"N={N}")
+
+
+def test_closed_forms_on_gpu():
+    B, N, H, D, P = 1, 700, 4, 128, 2
+    q, k, v = _random_logical(B, N, H, D, seed=5)
+    ones = synth.f32_to_bf16(np.ones((B, N, H, D), np.float32))
+    out, _ = _run_fused(q, k, ones, P)
+    O = synth.from_seq_shards(out.reshape(P, B, -1, H, D), N)
+    assert np.all(synth.bf16_to_f32(O) == 1.0), "V = 1 must give O = 1 exactly"
+    out, _ = _run_fused(q[:, :1], k[:, :1], v[:, :1], 1)
+    assert np.array_equal(out.reshape(1, 1, H, D), v[:, :1]), "N = 1 must give O = V"
+    zeros = np.zeros_like(q)
+    out, _ = _run_fused(zeros, k, v, P)
+    O = synth.bf16_to_f32(synth.from_seq_shards(out.reshape(P, B, -1, H, D), N))
+    mean = synth.bf16_to_f32(v).astype(np.float64).mean(axis=1)
+    assert np.max(np.abs(O - mean[:, None])) < 2e-3
+
+
+def test_lse_rows_sum_to_one():
+    """sum_k exp(s_ik - LSE_i) recomputed in fp64 from the bf16 inputs."""
+    B, N, H, D, P = 1, 2000, 2, 128, 2
+    q, k, v = _random_logical(B, N, H, D, seed=9, k_mul=1.5)
+    _, lse = _run_fused(q, k, v, P, lse=True)
+    qf, kf = (synth.bf16_to_f32(x).astype(np.float64) for x in (q, k))
+    for h in range(H):
+        s = qf[0, :, h] @ kf[0, :, h].T / math.sqrt(D)
+        tot = np.exp(s - lse[0, h, :N, None]).sum(axis=1)
+        assert np.max(np.abs(tot - 1.0)) < 1e-3
+
+
+def test_dominant_key_selects_value_row():
+    B, N, H, D, P = 1, 1000, 2, 128, 2
+    q, k, v = _random_logical(B, N, H, D, seed=11)
+    q = synth.f32_to_bf16(np.abs(synth.bf16_to_f32(q)) + 0.5)
+    k = synth.f32_to_bf16(np.clip(synth.bf16_to_f32(k), -1, 1))
+    k[0, 613] = synth.f32_to_bf16(np.full((H, D), 64.0, np.float32))
+    out, _ = _run_fused(q, k, v, P)
+    O = synth.bf16_to_f32(synth.from_seq_shards(out.reshape(P, B, -1, H, D), N))
+    want = synth.bf16_to_f32(v[0, 613])
+    assert np.max(np.abs(O[0] - want[None])) < 1e-2
+
+
+def test_wait_timeout_is_reported_not_hung():
+    sp.selftest_wait_timeout(1_000_000)  # 1 ms
+    assert sp.device_status() == sp.SP_ERR_TIMEOUT
+    assert sp.device_status() == sp.SP_OK
+
+
+# ------------------------------------------------------------------ full sizes
+
+def _sampled_check(cfg, per_head, fused=True, extra_P=()):
+    s = cfg.shape
+    q, k, v = synth.qkv_logical(cfg)
+    out, _ = (_run_fused if fused else _run_unfused)(q, k, v, s.P)
+    rows = synth.sampled_rows(cfg, per_head, extra_P=extra_P)
+    rr = np.array([(0, h, i) for h in range(s.H) for i in rows], dtype=np.int64)
+    return _check_rows(out, q, k, v, rr, s.P, cfg.name), out, (q, k, v)
+
+
+@pytest.mark.parametrize("name", ["480p", "720p", "1344x768"])
+def test_full_size_configs_sampled_rows(name):
+    cfg = synth.CONFIGS[name]
+    per_head = 12 if name == "1344x768" else 16
+    _sampled_check(cfg, per_head)
+
+
+def test_720p_unfused_equals_fused():
+    cfg = synth.CONFIGS["720p"]
+    s = cfg.shape
+    q, k, v = synth.qkv_logical(cfg)
+    f, _ = _run_fused(q, k, v, s.P)
+    u, _ = _run_unfused(q, k, v, s.P)
+    assert np.array_equal(f, u)
+
+
+def test_sweep_degrees_bit_identical_and_sampled():
+    """Layout sweep: N in {4096, 32760, 75600, 75601}, P in {1, 2, 4, 8};
+    every P bit-identical to P = 1; P = 1 checked against the oracle."""
+    for N in synth.SWEEP_N:
+        base = synth.sweep_config(N, 1)
+        q, k, v = synth.qkv_logical(base)
+        ref = None
+        for P in synth.SWEEP_P:
+            out, _ = _run_fused(q, k, v, P)
+            got = synth.from_seq_shards(out.reshape(P, 1, -1, 40, 128), N)
+            if ref is None:
+                ref = got
+                rows = synth.sampled_rows(base, 6, extra_P=synth.SWEEP_P)
+                rr = np.array([(0, h, i) for h in range(40) for i in rows], dtype=np.int64)
+                _check_rows(out, q, k, v, rr, 1, f"sweep N={N}")
+            else:
+                assert np.array_equal(got, ref), (N, P)

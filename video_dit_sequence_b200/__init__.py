@@ -1,0 +1,259 @@
+"""Ulysses sequence-parallel self-attention on one B200 (sm_100a).
+
+Python binding of ``libsp.so`` (C ABI in ``include/sp.h``).  This module only
+marshals arguments: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is
+no CPU or PyTorch fallback: without the built library, or without a CUDA
+device, the calls raise.
+
+The method (fal.ai, "Generate video with WAN 2.2 across four GPUs", section
+"Splitting one generation across four GPUs"): P ranks each hold N/P tokens
+of the sequence for all H heads; an all-to-all trades tokens for heads, each
+rank attends over the full sequence for H/P heads, and the outputs return to
+the token owners.  With P virtual ranks on one GPU the exchange is
+``pack`` / ``unpack``; ``attention_seqsharded`` fuses all three steps.
+
+Layouts (bf16, contiguous):
+  sequence-sharded  [P][B][Nl][H][D]    Nl = ceil(N/P)
+  head-sharded      [P][B][Np][Hl][D]   Np = P*Nl, Hl = H/P
+  lse (optional)    [B][H][Np] float32
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libsp.so")
+
+SP_OK = 0
+SP_ERR_NULL = 1
+SP_ERR_SHAPE = 2
+SP_ERR_HEADS_NOT_DIVISIBLE = 3
+SP_ERR_ALIGN = 4
+SP_ERR_UNSUPPORTED_D = 5
+SP_ERR_CUDA = 6
+SP_ERR_TIMEOUT = 7
+
+EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
+            "sp_attention", "sp_attention_seqsharded", "sp_device_status",
+            "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout")
+
+
+class sp_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("N", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("P", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class SpError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Loads libsp.so (built by ``python -m video_dit_sequence_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m video_dit_sequence_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sp_p = ctypes.c_void_p, ctypes.POINTER(sp_shape)
+    lib.sp_padded_tokens.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    lib.sp_padded_tokens.restype = ctypes.c_int64
+    lib.sp_check_shape.argtypes = [sp_p]
+    lib.sp_check_shape.restype = ctypes.c_int
+    for name in ("sp_pack", "sp_unpack"):
+        f = getattr(lib, name)
+        f.argtypes = [vp, vp, sp_p, vp]
+        f.restype = ctypes.c_int
+    for name in ("sp_attention", "sp_attention_seqsharded"):
+        f = getattr(lib, name)
+        f.argtypes = [vp, vp, vp, vp, vp, sp_p, vp]
+        f.restype = ctypes.c_int
+    lib.sp_device_status.argtypes = [vp]
+    lib.sp_device_status.restype = ctypes.c_int
+    lib.sp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+    lib.sp_selftest_wait_timeout.restype = ctypes.c_int
+    lib.sp_launch_count.argtypes = []
+    lib.sp_launch_count.restype = ctypes.c_uint64
+    lib.sp_status_str.argtypes = [ctypes.c_int]
+    lib.sp_status_str.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    return load().sp_status_str(int(status)).decode()
+
+
+@dataclasses.dataclass(frozen=True)
+class Shape:
+    """Problem shape; scale <= 0 selects 1/sqrt(D)."""
+    B: int
+    N: int
+    H: int
+    D: int
+    P: int
+    scale: float = 0.0
+
+    @property
+    def Hl(self) -> int:
+        return self.H // self.P
+
+    @property
+    def Nl(self) -> int:
+        return -(-self.N // self.P)
+
+    @property
+    def Np(self) -> int:
+        return self.Nl * self.P
+
+    @property
+    def seq_sharded(self):
+        return (self.P, self.B, self.Nl, self.H, self.D)
+
+    @property
+    def head_sharded(self):
+        return (self.P, self.B, self.Np, self.Hl, self.D)
+
+    @property
+    def lse_shape(self):
+        return (self.B, self.H, self.Np)
+
+    def c(self) -> sp_shape:
+        return sp_shape(self.B, self.N, self.H, self.D, self.P, float(self.scale))
+
+
+def padded_tokens(N: int, P: int) -> int:
+    return int(load().sp_padded_tokens(N, P))
+
+
+def check_shape(shape: Shape) -> int:
+    """Returns the library's status code for a shape (0 = valid)."""
+    s = shape.c()
+    return int(load().sp_check_shape(ctypes.byref(s)))
+
+
+def launch_count() -> int:
+    return int(load().sp_launch_count())
+
+
+# ---------------------------------------------------------------- tensors
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t, shape, name, dtype=None):
+    torch = _torch()
+    if t is None:
+        return None
+    dtype = dtype or torch.bfloat16
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape) and t.numel() != math.prod(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != SP_OK:
+        raise SpError(status, where)
+
+
+def pack(xs, xh, shape: Shape, stream=None):
+    """Sequence-sharded -> head-sharded (bit-exact permutation)."""
+    s = shape.c()
+    _check(load().sp_pack(_ptr(xs, shape.seq_sharded, "xs"), _ptr(xh, shape.head_sharded, "xh"),
+                          ctypes.byref(s), _stream(stream, xs.device)), "sp_pack")
+
+
+def unpack(oh, os_, shape: Shape, stream=None):
+    """Head-sharded -> sequence-sharded (bit-exact permutation)."""
+    s = shape.c()
+    _check(load().sp_unpack(_ptr(oh, shape.head_sharded, "oh"), _ptr(os_, shape.seq_sharded, "os"),
+                            ctypes.byref(s), _stream(stream, oh.device)), "sp_unpack")
+
+
+def attention(qh, kh, vh, oh, shape: Shape, lse=None, stream=None):
+    """Full-sequence attention per head group on head-sharded tensors."""
+    torch = _torch()
+    s = shape.c()
+    hs = shape.head_sharded
+    _check(load().sp_attention(
+        _ptr(qh, hs, "qh"), _ptr(kh, hs, "kh"), _ptr(vh, hs, "vh"), _ptr(oh, hs, "oh"),
+        _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
+        _stream(stream, qh.device)), "sp_attention")
+
+
+def attention_seqsharded(qs, ks, vs, os_, shape: Shape, lse=None, stream=None):
+    """Fused pack + attention + unpack on sequence-sharded tensors."""
+    torch = _torch()
+    s = shape.c()
+    ss = shape.seq_sharded
+    _check(load().sp_attention_seqsharded(
+        _ptr(qs, ss, "qs"), _ptr(ks, ss, "ks"), _ptr(vs, ss, "vs"), _ptr(os_, ss, "os"),
+        _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
+        _stream(stream, qs.device)), "sp_attention_seqsharded")
+
+
+def device_status(stream=None, device=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status."""
+    return int(load().sp_device_status(_stream(stream, device)))
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None, device=None):
+    """Enqueues a kernel whose bounded wait must run out (see sp.h)."""
+    _check(load().sp_selftest_wait_timeout(int(limit_ns), _stream(stream, device)),
+           "sp_selftest_wait_timeout")
+
+
+def ulysses_attention(q, k, v, P: int, scale: float = 0.0, fused: bool = True):
+    """User-level call: q, k, v are [B, N, H, D] bf16 CUDA tensors (logical,
+    unsharded); returns O [B, N, H, D].  The tensors are laid out as P
+    sequence shards (zero-padded to Np tokens), attended with P virtual ranks
+    and read back.  fused=False runs pack -> attention -> unpack."""
+    torch = _torch()
+    B, N, H, D = q.shape
+    shape = Shape(B, N, H, D, P, scale)
+    Nl, Np = shape.Nl, shape.Np
+
+    def shards(x):
+        buf = torch.zeros((B, Np, H, D), dtype=x.dtype, device=x.device)
+        buf[:, :N] = x
+        return buf.view(B, P, Nl, H, D).transpose(0, 1).contiguous()
+
+    qs, ks, vs = shards(q), shards(k), shards(v)
+    os_ = torch.empty_like(qs)
+    if fused and (B == 1 or P == 1):
+        attention_seqsharded(qs, ks, vs, os_, shape)
+    else:
+        hs = shape.head_sharded
+        qh, kh, vh, oh = (torch.empty(hs, dtype=q.dtype, device=q.device) for _ in range(4))
+        pack(qs, qh, shape)
+        pack(ks, kh, shape)
+        pack(vs, vh, shape)
+        attention(qh, kh, vh, oh, shape)
+        unpack(oh, os_, shape)
+    return os_.transpose(0, 1).reshape(B, Np, H, D)[:, :N]

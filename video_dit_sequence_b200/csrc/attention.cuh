@@ -1,0 +1,379 @@
+// attention.cuh -- full-sequence, non-causal bf16 attention per head on
+// tcgen05 tensor cores (sm_100a).
+//
+// What it computes (fal.ai "Generate video with WAN 2.2 across four GPUs",
+// section "Splitting one generation across four GPUs": after the exchange
+// each rank attends over the full sequence for its heads):
+//   O[i] = sum_{k<N} softmax_k(q_i . k_k * scale) v_k      for i < N,
+//   O[i] = 0                                               for N <= i < Np.
+// The softmax is evaluated online, one 128-key tile at a time (flash
+// attention), which reaches the two-pass result up to rounding.
+//
+// One CTA owns two 128-row query tiles of one (batch, head).  Roles:
+//   warps 0-3  softmax for query tile 0 (one thread per query row)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q once, then K_j, V_j into a ring of smem slots
+//   warp  9    TMEM allocator and the single MMA-issuing thread
+// Tensor memory (512 columns x 128 lanes, fp32): S_t at columns 128t,
+// O_t at columns 256 + D*t.  The softmax writes P_t (bf16, two per column)
+// over the first 64 columns of S_t, and the P*V product reads it from there.
+// Per key tile j the MMA thread issues, in this order,
+//   O_0 += P_0 V_j,  S_0 = Q_0 K_{j+1}^T,  O_1 += P_1 V_j,  S_1 = Q_1 K_{j+1}^T
+// so the tensor core works on one query tile while the other one's softmax
+// runs.  tcgen05 operations from one thread execute in issue order, so an S
+// write never overtakes the P read before it, and the commit that signals
+// "S_{t,j+1} ready" also covers the O_t update before it: when a softmax
+// thread sees S ready it may rescale O_t in place.
+//
+// Online softmax with a lazily updated row maximum: the running reference
+// m (log2 units) moves only when a tile's maximum exceeds it by more than 8,
+// so probabilities stay <= 2^8 and O is rescaled rarely.  The arithmetic of
+// a row depends only on its own scores and the fixed key-tile order, never on
+// P, the layout, or the CTA it runs in: outputs are bit-identical across
+// degrees and between the fused and the three-call path.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace sp {
+
+struct AttnParams {
+  int32_t N;            // true tokens (keys and queries)
+  int32_t Np;           // rows that exist in the output buffer per (batch, head)
+  int32_t H;            // global heads
+  int32_t B;
+  int32_t hsplit;       // heads per tensor-map "batch" slot (Hl or H)
+  int32_t num_kv_tiles; // ceil(N / 128)
+  float scale_log2e;    // scale * log2(e)
+  __nv_bfloat16 *o;     // output base
+  int64_t o_row;        // elements between consecutive tokens
+  int64_t o_batch;      // elements between tensor-map batch slots
+  float *lse;           // [B][H][Np] or null
+  int32_t *status;      // device status word
+};
+
+constexpr int32_t kStatusTimeout = 7;
+
+template <int D>
+struct AttnCfg {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int kBM = 128;                   // query rows per tile
+  static constexpr int kBN = 128;                   // keys per tile
+  static constexpr int kHalves = D / 64;            // 128-byte column blocks per row
+  static constexpr int kBlockBytes = 128 * 128;     // 128 rows x 64 bf16 (one swizzle block)
+  static constexpr int kTileBytes = kHalves * kBlockBytes;
+  static constexpr int kStages = 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  static constexpr int kNumBar = 1 + 2 * kStages + 6;
+  static constexpr int kOffMisc = kOffBar + kNumBar * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256;
+  static constexpr uint32_t kColO1 = 256 + D;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+attention_kernel(const __grid_constant__ CUtensorMap tmQ,
+                 const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t *sptr = smem_raw + (sbase - raw);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int hg = blockIdx.y;            // global head
+  const int b = blockIdx.z;
+  const int map_head = hg % p.hsplit;
+  const int map_batch = (hg / p.hsplit) * p.B + b;
+  const int q0 = blockIdx.x * 2 * C::kBM;
+  const int T = p.num_kv_tiles;
+
+  const uint32_t bar_q = sbase + C::kOffBar;
+  const uint32_t bar_kv_full = bar_q + 8;
+  const uint32_t bar_kv_empty = bar_kv_full + 8 * C::kStages;
+  const uint32_t bar_s = bar_kv_empty + 8 * C::kStages;  // [2]
+  const uint32_t bar_p = bar_s + 16;                      // [2]
+  const uint32_t bar_o = bar_p + 16;                      // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + C::kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(sptr + C::kOffMisc + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_kv_full + 8 * s, 1);
+      mbar_init(bar_kv_empty + 8 * s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s + 8 * t, 1);
+      mbar_init(bar_p + 8 * t, 128);
+      mbar_init(bar_o + 8 * t, 1);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_kv = policy_evict_last();
+      mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int h = 0; h < C::kHalves; ++h)
+          tma_load_4d(sbase + C::kOffQ + t * C::kTileBytes + h * C::kBlockBytes, &tmQ, bar_q,
+                      h * 64, map_head, q0 + t * C::kBM, map_batch, pol_q);
+      int it = 0;
+      for (int j = 0; j < T && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          if (!mbar_wait(bar_kv_empty + 8 * s, ph ^ 1u, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_kv_full + 8 * s, C::kTileBytes);
+          const CUtensorMap *m = kv == 0 ? &tmK : &tmV;
+          for (int h = 0; h < C::kHalves; ++h)
+            tma_load_4d(sbase + C::kOffKV + s * C::kTileBytes + h * C::kBlockBytes, m,
+                        bar_kv_full + 8 * s, h * 64, map_head, j * C::kBN, map_batch, pol_kv);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t qa = sbase + C::kOffQ + t * C::kTileBytes;
+        const uint32_t kb = sbase + C::kOffKV + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          umma_ss(tmem + (t ? C::kColS1 : 0u), make_sdesc_sw128(qa + off, 16, 1024),
+                  make_sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool first) {
+        const uint32_t vb = sbase + C::kOffKV + slot * C::kTileBytes;
+        const uint32_t pcol = t ? C::kColS1 : 0u;
+        const uint32_t ocol = t ? C::kColO1 : C::kColO0;
+#pragma unroll
+        for (int kk = 0; kk < C::kBN / 16; ++kk) {
+          umma_ts(tmem + ocol, tmem + pcol + kk * 8,
+                  make_sdesc_sw128(vb + kk * 16 * 128, C::kBlockBytes, 1024), idesc_pv,
+                  (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      int it = 0;
+      ok = mbar_wait(bar_q, 0, abort_flag, kWaitLimitNs) &&
+           mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        umma_commit(bar_s);
+        issue_s(1, 0);
+        umma_commit(bar_s + 8);
+        umma_commit(bar_kv_empty);
+        it = 1;
+      }
+      for (int j = 0; j < T && ok; ++j) {
+        const int sv = it % C::kStages;
+        ok = mbar_wait(bar_kv_full + 8 * sv, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
+        ++it;
+        if (!ok) break;
+        ok = mbar_wait(bar_p, j & 1, abort_flag, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, sv, j == 0);
+        int sk = 0;
+        if (j + 1 < T) {
+          sk = it % C::kStages;
+          ok = mbar_wait(bar_kv_full + 8 * sk, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
+          ++it;
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, sk);
+          umma_commit(bar_s);
+        } else {
+          umma_commit(bar_o);
+        }
+        ok = mbar_wait(bar_p + 8, j & 1, abort_flag, kWaitLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, sv, j == 0);
+        umma_commit(bar_kv_empty + 8 * sv);
+        if (j + 1 < T) {
+          issue_s(1, sk);
+          umma_commit(bar_s + 8);
+          umma_commit(bar_kv_empty + 8 * sk);
+        } else {
+          umma_commit(bar_o + 8);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- softmax
+    const int t = warp >> 2;           // query tile
+    const int wq = warp & 3;           // TMEM lane quarter this warp may access
+    const int row = wq * 32 + lane;    // row within the tile
+    const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + (t ? C::kColS1 : 0u);
+    const uint32_t tO = tmem + lane_bits + (t ? C::kColO1 : C::kColO0);
+    const float sl2 = p.scale_log2e;
+    const int tail = p.N - (T - 1) * C::kBN;   // valid keys in the last tile, 1..128
+    float m_ref = -INFINITY;                   // reference maximum, log2 units
+    float l = 0.f;
+    for (int j = 0; j < T; ++j) {
+      // Warp-uniform exit: the TMEM accesses below are warp-collective.
+      const bool got = mbar_wait(bar_s + 8 * t, j & 1, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld32(tS + 0, &s[0]);
+      tmem_ld32(tS + 32, &s[32]);
+      tmem_ld32(tS + 64, &s[64]);
+      tmem_ld32(tS + 96, &s[96]);
+      tmem_wait_ld();
+      if (j == T - 1 && tail < C::kBN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= tail) s[c] = 0xFF800000u;  // -inf
+      }
+      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
+      float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(s[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const bool need = mx > m_ref + 8.0f;
+      const bool warp_rescale = __any_sync(0xffffffffu, need);
+      const float alpha = need ? ex2(m_ref - mx) : 1.0f;
+      if (need) {
+        l *= alpha;
+        m_ref = mx;
+      }
+      const float neg_m = -m_ref;
+      float ls0 = 0.f, ls1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, neg_m));
+        const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, neg_m));
+        ls0 += p0;
+        ls1 += p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l += ls0 + ls1;
+      tmem_st32(tS + 0, &pk[0]);
+      tmem_st32(tS + 32, &pk[32]);
+      // Rescale O_t (only after the first tile; O_t is not yet written
+      // before it).  Warp-uniform because TMEM access is warp-collective;
+      // rows that keep their reference multiply by exactly 1.
+      if (warp_rescale && j > 0) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_p + 8 * t);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait(bar_o + 8 * t, 0, abort_flag, kWaitLimitNs);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const int token = q0 + t * C::kBM + row;
+      const bool valid = token < p.N;
+      const bool exists = token < p.Np;
+      const float inv_l = valid ? 1.0f / l : 0.0f;
+      __nv_bfloat16 *dst = p.o + static_cast<int64_t>(map_batch) * p.o_batch +
+                           static_cast<int64_t>(token) * p.o_row + static_cast<int64_t>(map_head) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = valid ? pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                     __uint_as_float(o[2 * i + 1]) * inv_l)
+                       : 0u;  // padding rows: +0.0 words
+        if (exists) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (p.lse != nullptr && exists) {
+        const float v = valid ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        p.lse[(static_cast<int64_t>(b) * p.H + hg) * p.Np + token] = v;
+      }
+    } else {
+      ok = false;
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  if (!ok) {
+    *abort_flag = 1;
+    atomicExch(p.status, kStatusTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    // Let copies and MMAs already in flight land before the CTA's shared and
+    // tensor memory are released (bounded: 50 us).
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 50000ull) {
+    }
+  }
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace sp

@@ -1,0 +1,119 @@
+// permute.cuh -- the Ulysses token<->head exchange on one GPU.
+//
+// With P virtual ranks in one HBM, the all-to-all of "Splitting one
+// generation across four GPUs" (fal.ai, "Generate video with WAN 2.2 across
+// four GPUs") is a pure permutation of 16-bit words:
+//   pack   : xh[j][b][r*Nl + n][hh][:] = xs[r][b][n][j*Hl + hh][:]
+//   unpack : os[r][b][n][j*Hl + hh][:] = oh[j][b][r*Nl + n][hh][:]
+// Both move contiguous runs of Hl*D words (>= 128 bytes), so every thread
+// copies 16-byte vectors and consecutive threads touch consecutive vectors of
+// one run on both sides.  The destination is walked linearly (vector v of
+// the kernel writes bytes 16v .. 16v+15 of the output); the source address
+// comes from the index arithmetic above, with invariant-divisor
+// multiplications in place of integer division.
+#pragma once
+#include <cstdint>
+
+namespace sp {
+
+// Quotient / remainder by a fixed divisor d >= 1 for numerators n < 2^31:
+// q = (mulhi(n, m) + n) >> s with s = ceil(log2 d) and
+// m = floor(2^32 (2^s - d) / d) + 1 (Granlund & Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994, section 4).
+struct FastDiv {
+  uint32_t d, m, s;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  f.s = s;
+  f.m = static_cast<uint32_t>((((1ull << s) - d) << 32) / d + 1ull);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+  return (__umulhi(n, f.m) + n) >> f.s;
+}
+
+struct PermuteParams {
+  const uint4 *src;
+  uint4 *dst;
+  uint32_t total_vec;      // output vectors (16 B each), < 2^31
+  FastDiv vr;              // vectors per run: Hl*D/8
+  FastDiv nl;              // Nl
+  FastDiv p;               // P
+  FastDiv bdiv;            // B
+  FastDiv pvr;             // P * vectors per run (unpack: vectors per output row)
+  uint32_t H_vec;          // vectors per sequence-sharded token row: H*D/8
+  uint32_t Hl_vec;         // vectors per head-sharded token row: Hl*D/8
+  uint32_t Nl, Np, B, P;
+};
+
+constexpr int kPermThreads = 256;
+constexpr int kPermUnroll = 4;
+
+// Loads bypass L1 (each byte is read once); stores stream.
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void st_stream(uint4 *p, const uint4 &v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};"
+               ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Source vector of pack for output vector v: output row R = v / Vr holds
+// (j, b, r, n) with R = ((j*B + b)*P + r)*Nl + n; vector k = v % Vr of it.
+__device__ __forceinline__ uint64_t pack_src(uint32_t v, const PermuteParams &p) {
+  uint32_t R = fdiv(v, p.vr);
+  uint32_t k = v - R * p.vr.d;
+  uint32_t blk = fdiv(R, p.nl);
+  uint32_t n = R - blk * p.Nl;
+  uint32_t jb = fdiv(blk, p.p);
+  uint32_t r = blk - jb * p.P;
+  uint32_t j = fdiv(jb, p.bdiv);
+  uint32_t b = jb - j * p.B;
+  return (static_cast<uint64_t>(r * p.B + b) * p.Nl + n) * p.H_vec +
+         static_cast<uint64_t>(j) * p.Hl_vec + k;
+}
+
+// Source vector of unpack for output vector v: output row R = v / (P*Vr)
+// holds (r, b, n) with R = (r*B + b)*Nl + n; within it, run j = w / Vr and
+// vector k = w % Vr, w = v % (P*Vr).
+__device__ __forceinline__ uint64_t unpack_src(uint32_t v, const PermuteParams &p) {
+  uint32_t R = fdiv(v, p.pvr);
+  uint32_t w = v - R * p.pvr.d;
+  uint32_t j = fdiv(w, p.vr);
+  uint32_t k = w - j * p.vr.d;
+  uint32_t rb = fdiv(R, p.nl);
+  uint32_t n = R - rb * p.Nl;
+  uint32_t r = fdiv(rb, p.bdiv);
+  uint32_t b = rb - r * p.B;
+  return (static_cast<uint64_t>(j * p.B + b) * p.Np + r * p.Nl + n) * p.Hl_vec + k;
+}
+
+template <bool kPack>
+__global__ void __launch_bounds__(kPermThreads)
+permute_kernel(const PermuteParams p) {
+  const uint32_t base = blockIdx.x * (kPermThreads * kPermUnroll) + threadIdx.x;
+  uint4 v[kPermUnroll];
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    uint32_t o = base + u * kPermThreads;
+    if (o < p.total_vec) v[u] = ld_stream(p.src + (kPack ? pack_src(o, p) : unpack_src(o, p)));
+  }
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    uint32_t o = base + u * kPermThreads;
+    if (o < p.total_vec) st_stream(p.dst + o, v[u]);
+  }
+}
+
+}  // namespace sp

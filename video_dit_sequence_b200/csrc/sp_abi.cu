@@ -1,0 +1,297 @@
+// sp_abi.cu -- the C ABI declared in include/sp.h: argument checks, TMA
+// descriptor construction and kernel launches.  One translation unit holds
+// every kernel so that the device status word needs no relocatable code.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attention.cuh"
+#include "permute.cuh"
+#include "sp.h"
+
+namespace {
+
+__device__ int32_t g_status = 0;
+
+std::atomic<uint64_t> g_launches{0};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sp_status check_common(const sp_shape *s) {
+  if (s == nullptr) return SP_ERR_NULL;
+  if (s->B < 1 || s->N < 1 || s->H < 1 || s->P < 1 || s->D < 1) return SP_ERR_SHAPE;
+  if (s->H % s->P != 0) return SP_ERR_HEADS_NOT_DIVISIBLE;
+  if (s->D != 64 && s->D != 128) return SP_ERR_UNSUPPORTED_D;
+  if (s->P > 65535 || s->B > 65535 || s->H > 65535) return SP_ERR_SHAPE;
+  const int64_t Nl = (static_cast<int64_t>(s->N) + s->P - 1) / s->P;
+  const int64_t elems = static_cast<int64_t>(s->P) * s->B * Nl * s->H * s->D;
+  // permute kernels index 16-byte vectors with 32-bit integers below 2^31
+  if (elems / 8 >= (int64_t(1) << 31)) return SP_ERR_SHAPE;
+  return SP_OK;
+}
+
+sp_status launch_status(cudaError_t e) {
+  if (e != cudaSuccess) return SP_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return SP_OK;
+}
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+
+// Device address of g_status on the current device (looked up once per
+// device; host code must not use the symbol itself as a pointer).
+int32_t *status_ptr() {
+  static int32_t *ptrs[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> g(g_mu);
+  if (ptrs[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) == cudaSuccess) ptrs[dev] = static_cast<int32_t *>(p);
+  }
+  return ptrs[dev];
+}
+
+sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, bool pack) {
+  sp_status st = check_common(s);
+  if (st != SP_OK) return st;
+  if (src == nullptr || dst == nullptr) return SP_ERR_NULL;
+  if (!aligned16(src) || !aligned16(dst)) return SP_ERR_ALIGN;
+  const uint32_t P = s->P, B = s->B, H = s->H, D = s->D;
+  const uint32_t Hl = H / P;
+  const uint32_t Nl = (s->N + P - 1) / P;
+  sp::PermuteParams p;
+  p.src = static_cast<const uint4 *>(src);
+  p.dst = static_cast<uint4 *>(dst);
+  p.total_vec = static_cast<uint32_t>(static_cast<uint64_t>(P) * B * Nl * H * D / 8);
+  p.vr = sp::make_fastdiv(Hl * D / 8);
+  p.nl = sp::make_fastdiv(Nl);
+  p.p = sp::make_fastdiv(P);
+  p.bdiv = sp::make_fastdiv(B);
+  p.pvr = sp::make_fastdiv(P * Hl * D / 8);
+  p.H_vec = H * D / 8;
+  p.Hl_vec = Hl * D / 8;
+  p.Nl = Nl;
+  p.Np = Nl * P;
+  p.B = B;
+  p.P = P;
+  const uint32_t per_block = sp::kPermThreads * sp::kPermUnroll;
+  const uint32_t blocks = (p.total_vec + per_block - 1) / per_block;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (pack)
+    sp::permute_kernel<true><<<blocks, sp::kPermThreads, 0, cs>>>(p);
+  else
+    sp::permute_kernel<false><<<blocks, sp::kPermThreads, 0, cs>>>(p);
+  return launch_status(cudaGetLastError());
+}
+
+// Tensor map over one of Q/K/V, viewed as [Bx][N rows][Hx heads][D] with
+// the given row and batch strides (elements).  Rows >= N read as zero.
+bool make_map(CUtensorMap *m, const void *base, int D, int Hx, int N, int Bx, int64_t row_el,
+              int64_t batch_el) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hx),
+                        static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(Bx)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(row_el) * 2,
+                           static_cast<cuuint64_t>(batch_el) * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                             const sp::AttnParams &p, int B, cudaStream_t cs) {
+  using C = sp::AttnCfg<D>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(sp::attention_kernel<D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+  }
+  dim3 grid((p.N + 2 * C::kBM - 1) / (2 * C::kBM), p.H, B);
+  sp::attention_kernel<D><<<grid, C::kThreads, C::kSmemBytes, cs>>>(q, k, v, p);
+  return cudaGetLastError();
+}
+
+// Shared launch path.  The head-sharded and the sequence-sharded layouts are
+// both [slots][rows][heads-per-slot][D] with different strides; the kernel
+// finds (slot, head-in-slot) of global head h as (h / hsplit * B + b,
+// h % hsplit).
+sp_status attention(const void *q, const void *k, const void *v, void *o, float *lse,
+                    const sp_shape *s, void *stream, bool seqsharded) {
+  sp_status st = check_common(s);
+  if (st != SP_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SP_ERR_NULL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
+    return SP_ERR_ALIGN;
+  const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
+  const int Hl = H / P;
+  const int Nl = (N + P - 1) / P;
+  const int Np = Nl * P;
+  int Hx, Bx, hsplit;
+  int64_t row_el, batch_el;
+  if (seqsharded) {
+    if (B > 1 && P > 1) return SP_ERR_SHAPE;
+    Hx = H;
+    hsplit = H;
+    Bx = B;
+    row_el = static_cast<int64_t>(H) * D;
+    batch_el = static_cast<int64_t>(Nl) * H * D;  // P == 1 when B > 1
+  } else {
+    Hx = Hl;
+    hsplit = Hl;
+    Bx = P * B;
+    row_el = static_cast<int64_t>(Hl) * D;
+    batch_el = static_cast<int64_t>(Np) * Hl * D;
+  }
+  int32_t *status = status_ptr();
+  if (status == nullptr) return SP_ERR_CUDA;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, Hx, N, Bx, row_el, batch_el) ||
+      !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el) ||
+      !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el))
+    return SP_ERR_CUDA;
+  sp::AttnParams p;
+  p.N = N;
+  p.Np = Np;
+  p.H = H;
+  p.B = B;
+  p.hsplit = hsplit;
+  p.num_kv_tiles = (N + 127) / 128;
+  const float scale = s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2e = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.o_row = row_el;
+  p.o_batch = batch_el;
+  p.lse = lse;
+  p.status = status;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  cudaError_t e = D == 64 ? launch_attention<64>(mq, mk, mv, p, B, cs)
+                          : launch_attention<128>(mq, mk, mv, p, B, cs);
+  return launch_status(e);
+}
+
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int32_t *status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sp::mbar_init(sp::smem_u32(&bar), 1);
+    abort_flag = 0;
+    sp::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: the wait must give up after limit_ns.
+    if (!sp::mbar_wait(sp::smem_u32(&bar), 0, &abort_flag, limit_ns))
+      atomicExch(status, sp::kStatusTimeout);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+sp_status sp_selftest_wait_timeout(uint64_t limit_ns, void *stream) {
+  if (limit_ns > 1000000000ull) limit_ns = 1000000000ull;
+  int32_t *status = status_ptr();
+  if (status == nullptr) return SP_ERR_CUDA;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status);
+  return launch_status(cudaGetLastError());
+}
+
+int64_t sp_padded_tokens(int32_t N, int32_t P) {
+  if (N < 1 || P < 1) return -1;
+  return ((static_cast<int64_t>(N) + P - 1) / P) * P;
+}
+
+sp_status sp_check_shape(const sp_shape *shape) { return check_common(shape); }
+
+sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream) {
+  return permute(xs, xh, shape, stream, true);
+}
+
+sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *stream) {
+  return permute(oh, os, shape, stream, false);
+}
+
+sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh, float *lse,
+                       const sp_shape *shape, void *stream) {
+  return attention(qh, kh, vh, oh, lse, shape, stream, false);
+}
+
+sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs, void *os,
+                                  float *lse, const sp_shape *shape, void *stream) {
+  return attention(qs, ks, vs, os, lse, shape, stream, true);
+}
+
+sp_status sp_device_status(void *stream) {
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return SP_ERR_CUDA;
+  int32_t *status = status_ptr();
+  if (status == nullptr) return SP_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return SP_ERR_CUDA;
+  if (v != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SP_ERR_CUDA;
+    return v == sp::kStatusTimeout ? SP_ERR_TIMEOUT : SP_ERR_CUDA;
+  }
+  return SP_OK;
+}
+
+uint64_t sp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *sp_status_str(sp_status status) {
+  switch (status) {
+    case SP_OK: return "ok";
+    case SP_ERR_NULL: return "a required pointer is NULL";
+    case SP_ERR_SHAPE: return "shape out of range";
+    case SP_ERR_HEADS_NOT_DIVISIBLE: return "the degree P must divide the head count H";
+    case SP_ERR_ALIGN: return "a device pointer is not 16-byte aligned";
+    case SP_ERR_UNSUPPORTED_D: return "head dim D must be 64 or 128";
+    case SP_ERR_CUDA: return "CUDA error";
+    case SP_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"
