@@ -1,0 +1,360 @@
+#!/usr/bin/env python3
+"""Benchmark of Ulysses sequence-parallel attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 720p]
+                    [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of synthetic
+input: the fused sequence-parallel attention (pack + per-head-group
+attention + unpack in one kernel, sp_attention_seqsharded) on the
+720p/81-frame-shaped workload (75,600 tokens, 40 heads, d = 128, P = 4
+virtual ranks).  The JSON line's value is algorithmic attention TFLOP/s,
+4*B*N^2*H*D per step, summed over ranks, divided by the slowest rank's
+device time for the K timed steps.  The three unfused rows (pack of Q, K and
+V; attention on head-sharded tensors; unpack of O) are timed in the same run
+and reported under "rows" (GB/s for the permutations).  Q+K+V are 2.3 GB,
+far larger than the 126 MB L2, so no L2 flush is done between steps.
+
+With --gpus N > 1 (launched by torchrun, one rank per GPU) every rank runs
+the same single-GPU problem on its own GPU: independent problems, no
+data-path collective, weak scaling.
+
+--impl reference times the fp64 CPU oracle on the host cores instead, each
+step a bounded sample (query rows) of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SP attention TFLOP/s & % bf16 tensor peak at 75.6k tokens; pack/unpack GB/s"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(cfg):
+    s = cfg.shape
+    g = "x".join(str(x) for x in cfg.grid) if cfg.grid[0] else "-"
+    return {"workload": f"{cfg.name}-shaped Ulysses SP attention, latent grid {g} = {s.N} tokens",
+            "B": s.B, "N": s.N, "H": s.H, "D": s.D, "P": s.P,
+            "causal": False, "inputs": "bf16 i.i.d. N(0,1), seeded",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+def oracle_sample(cfg, q, k, v, seconds, max_rows_per_head=64, threads=None):
+    """Times the fp64 oracle on sampled query rows (all heads) until about
+    `seconds` of CPU work; returns (TFLOP/s, rows, seconds, threads)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    s = cfg.shape
+    threads = threads or synth.host_threads()
+    rows = synth.sampled_rows(cfg, max_rows_per_head)
+    per_row_flops = 4.0 * s.N * s.D
+    done, spent, i = 0, 0.0, 0
+    while spent < seconds and i < len(rows):
+        batch = rows[i:i + max(1, threads // s.H + 1)]
+        rr = np.array([(0, h, t) for t in batch for h in range(s.H)], dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, rr, threads=threads)
+        spent += time.perf_counter() - t0
+        done += len(rr)
+        i += len(batch)
+    return done * per_row_flops / spent / 1e12, done, spent, threads
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(", ") for r in self.file.read().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle on the host cores."""
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = synth.CONFIGS[args.config]
+    q, k, v = synth.qkv_logical(cfg)
+    per_step = max(1.0, args.ref_step_seconds)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, q, k, v, per_step / 4, max_rows_per_head=2)
+    vals, rows_done, secs, thr = [], 0, 0.0, 1
+    for _ in range(args.steps):
+        val, r, sp_, thr = oracle_sample(cfg, q, k, v, per_step, max_rows_per_head=8)
+        vals.append(val)
+        rows_done += r
+        secs += sp_
+    value = rows_done * 4.0 * cfg.shape.N * cfg.shape.D / secs / 1e12
+    sample = (f"{rows_done} query rows over {args.steps} steps (all {cfg.shape.H} heads, "
+              f"full {cfg.shape.N}-key softmax each), fp64")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(cfg),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import video_dit_sequence_b200 as sp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sp.load()
+    cfg = synth.CONFIGS[args.config]
+    s = cfg.shape
+    shape = sp.Shape(s.B, s.N, s.H, s.D, s.P)
+    flops = s.flops()
+    q, k, v = synth.qkv_logical(cfg)
+
+    def pinned(a):
+        return torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(a, s.P)).view(np.int16)
+                                ).view(torch.bfloat16).pin_memory()
+
+    hq, hk, hv = pinned(q), pinned(k), pinned(v)
+    ho = torch.empty(shape.seq_sharded, dtype=torch.bfloat16).pin_memory()
+    qs, ks, vs = (h.to(dev) for h in (hq, hk, hv))
+    os_ = torch.empty(shape.seq_sharded, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sp.attention_seqsharded(qs, ks, vs, os_, shape, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if sp.device_status(stream) != sp.SP_OK:
+        raise SystemExit("device status not ok after warm-up")
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = str(local)
+    sampler = ClockSampler(uuid)
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = sp.launch_count()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    launches = sp.launch_count() - n0
+    clocks = sampler.stop()
+    if sp.device_status(stream) != sp.SP_OK:
+        raise SystemExit("device status not ok after the timed steps")
+    t_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([t_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    else:
+        t_max = t_ms
+    value = world * args.steps * flops / (t_max * 1e-3) / 1e12
+    per_launch_ms = t_ms / args.steps
+
+    # ---- unfused rows: pack (Q, K, V), attention on head-sharded, unpack (O)
+    hs = shape.head_sharded
+    qh, kh, vh, oh = (torch.empty(hs, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    os2 = torch.empty_like(os_)
+    reps = max(3, args.steps)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    tensor_bytes = 2.0 * math.prod(shape.seq_sharded)
+    pk, pkq = peaks()
+    t_pack = timed(lambda: sp.pack(qs, qh, shape, stream=stream))
+    t_unpack = timed(lambda: sp.unpack(oh, os2, shape, stream=stream))
+    t_attn = timed(lambda: sp.attention(qh, kh, vh, oh, shape, stream=stream))
+    if sp.device_status(stream) != sp.SP_OK:
+        raise SystemExit("device status not ok after the unfused rows")
+    pack_gbs = 2 * tensor_bytes / (t_pack * 1e-3) / 1e9
+    unpack_gbs = 2 * tensor_bytes / (t_unpack * 1e-3) / 1e9
+    rows = {
+        "pack": {"ms": t_pack, "GB/s": pack_gbs, "frac_hbm": pack_gbs / pk["hbm_gbs"],
+                 "bytes": 2 * tensor_bytes, "per": "one tensor (Q, K or V), read + write"},
+        "unpack": {"ms": t_unpack, "GB/s": unpack_gbs, "frac_hbm": unpack_gbs / pk["hbm_gbs"],
+                   "bytes": 2 * tensor_bytes, "per": "O, read + write"},
+        "attention_head_sharded": {"ms": t_attn, "TFLOP/s": flops / (t_attn * 1e-3) / 1e12},
+        "unfused_step_ms": 3 * t_pack + t_attn + t_unpack,
+        "fused_step_ms": per_launch_ms,
+    }
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        def e2e_step():
+            qs.copy_(hq, non_blocking=True)
+            ks.copy_(hk, non_blocking=True)
+            vs.copy_(hv, non_blocking=True)
+            sp.attention_seqsharded(qs, ks, vs, os_, shape, stream=stream)
+            ho.copy_(os_, non_blocking=True)
+        e2e_step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        te = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([te], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            te = float(t.item())
+        e2e = {"value": world * args.steps * flops / (te * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(3 * tensor_bytes), "d2h_bytes_per_step": int(tensor_bytes),
+               "ms_per_step": te / args.steps}
+        if sp.device_status(stream) != sp.SP_OK:
+            raise SystemExit("device status not ok after e2e")
+
+    achieved = flops / (per_launch_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attention_kernel<128> (sp_attention_seqsharded)",
+                "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"],
+                "peak_kind": f"{pkq} bf16 dense (burst)",
+                "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
+                "traffic": args.traffic_bytes,
+                "flops_per_launch": flops}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, r, secs, thr = oracle_sample(cfg, q, k, v, args.cpu_seconds)
+        cpu = {"value": val, "unit": UNIT, "cores": thr, "kind": "oracle",
+               "sample": f"{r} query rows ({r // s.H} per head x {s.H} heads), each a full "
+                         f"{s.N}-key fp64 softmax row, {secs:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": max(3, args.warmup),
+                "ms_per_step": t_max / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": workload_desc(cfg), "e2e": e2e, "gpu_launches": int(launches),
+                "clocks": clocks, "roofline": roofline, "cpu_baseline": cpu, "rows": rows}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="720p")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per launch of the attention kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
