@@ -69,7 +69,7 @@ struct AttnCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kNumBar = 1 + 2 * kStages + 6;
+  static constexpr int kNumBar = 1 + 2 * kStages + 8;
   static constexpr int kOffMisc = kOffBar + kNumBar * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr int kThreads = 320;
@@ -80,6 +80,7 @@ struct AttnCfg {
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+
 
 template <int D>
 __global__ void __launch_bounds__(320, 1)
@@ -105,8 +106,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t bar_kv_full = bar_q + 8;
   const uint32_t bar_kv_empty = bar_kv_full + 8 * C::kStages;
   const uint32_t bar_s = bar_kv_empty + 8 * C::kStages;  // [2]
-  const uint32_t bar_p = bar_s + 16;                      // [2]
-  const uint32_t bar_o = bar_p + 16;                      // [2]
+  const uint32_t bar_p = bar_s + 16;                      // [2 tiles][2 key halves]
+  const uint32_t bar_o = bar_p + 32;                      // [2]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sptr + C::kOffMisc + 4);
 
@@ -118,7 +119,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s + 8 * t, 1);
-      mbar_init(bar_p + 8 * t, 128);
+      mbar_init(bar_p + 16 * t, 128);
+      mbar_init(bar_p + 16 * t + 8, 128);
       mbar_init(bar_o + 8 * t, 1);
     }
     *abort_flag = 0;
@@ -180,16 +182,26 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                   make_sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool first) {
+      // O_t += P_t[:, 64h .. 64h+63] V_j[64h .. 64h+63, :] for key half h.
+      auto issue_pv_half = [&](int t, int slot, bool first, int h) {
         const uint32_t vb = sbase + C::kOffKV + slot * C::kTileBytes;
         const uint32_t pcol = t ? C::kColS1 : 0u;
         const uint32_t ocol = t ? C::kColO1 : C::kColO0;
 #pragma unroll
-        for (int kk = 0; kk < C::kBN / 16; ++kk) {
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
           umma_ts(tmem + ocol, tmem + pcol + kk * 8,
                   make_sdesc_sw128(vb + kk * 16 * 128, C::kBlockBytes, 1024), idesc_pv,
                   (first && kk == 0) ? 0u : 1u);
         }
+      };
+      // Waits for each half of P_t, then issues that half's PV MMAs.
+      auto issue_pv = [&](int t, int slot, bool first, int j) -> bool {
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(bar_p + 16 * t + 8 * h, j & 1, abort_flag, kWaitLimitNs)) return false;
+          tc_fence_after();
+          issue_pv_half(t, slot, first, h);
+        }
+        return true;
       };
       int it = 0;
       ok = mbar_wait(bar_q, 0, abort_flag, kWaitLimitNs) &&
@@ -208,10 +220,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         ok = mbar_wait(bar_kv_full + 8 * sv, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
         ++it;
         if (!ok) break;
-        ok = mbar_wait(bar_p, j & 1, abort_flag, kWaitLimitNs);
+        ok = issue_pv(0, sv, j == 0, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, sv, j == 0);
         int sk = 0;
         if (j + 1 < T) {
           sk = it % C::kStages;
@@ -224,10 +234,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         } else {
           umma_commit(bar_o);
         }
-        ok = mbar_wait(bar_p + 8, j & 1, abort_flag, kWaitLimitNs);
+        ok = issue_pv(1, sv, j == 0, j);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(1, sv, j == 0);
         umma_commit(bar_kv_empty + 8 * sv);
         if (j + 1 < T) {
           issue_s(1, sk);
@@ -270,16 +278,18 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int c = 0; c < 128; ++c)
           if (c >= tail) s[c] = 0xFF800000u;  // -inf
       }
-      float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-      float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+      // Row maximum: four independent chains of 3-input max.
+      float mc[4];
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(s[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(s[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(s[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(s[c + 3]));
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t *e = &s[32 * q];
+        float m = fmax3(__uint_as_float(e[0]), __uint_as_float(e[1]), __uint_as_float(e[2]));
+#pragma unroll
+        for (int c = 3; c < 31; c += 2)
+          m = fmax3(m, __uint_as_float(e[c]), __uint_as_float(e[c + 1]));
+        mc[q] = fmaxf(m, __uint_as_float(e[31]));
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * sl2;
       const bool need = mx > m_ref + 8.0f;
       const bool warp_rescale = __any_sync(0xffffffffu, need);
       const float alpha = need ? ex2(m_ref - mx) : 1.0f;
@@ -287,37 +297,53 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         l *= alpha;
         m_ref = mx;
       }
-      const float neg_m = -m_ref;
-      float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[64];
+      // p = 2^(s * scale * log2(e) - m_ref): two scores per packed FMA, ex2
+      // on the SFU.  Each half of the row's 128 probabilities is stored to TMEM
+      // (bf16, over the first 64 columns of S_t) and signalled on its own, so
+      // the PV MMAs of keys 0..63 can start while keys 64..127 are computed.
+      const uint64_t k_sl2 = f2_pack(sl2, sl2);
+      const uint64_t k_negm = f2_pack(-m_ref, -m_ref);
+      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), sl2, neg_m));
-        const float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), sl2, neg_m));
-        ls0 += p0;
-        ls1 += p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      l += ls0 + ls1;
-      tmem_st32(tS + 0, &pk[0]);
-      tmem_st32(tS + 32, &pk[32]);
-      // Rescale O_t (only after the first tile; O_t is not yet written
-      // before it).  Warp-uniform because TMEM access is warp-collective;
-      // rows that keep their reference multiply by exactly 1.
-      if (warp_rescale && j > 0) {
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + c, o);
+        for (int i = 0; i < 32; ++i) {
+          const int c = 64 * h + 2 * i;
+          const uint64_t x = f2_fma(f2_pack_bits(s[c], s[c + 1]), k_sl2, k_negm);
+          float p0, p1;
+          f2_unpack(x, p0, p1);
+          p0 = ex2(p0);
+          p1 = ex2(p1);
+          acc[i & 1] = f2_add(acc[i & 1], f2_pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
         }
+        if (h == 0 && warp_rescale && j > 0) {
+          // Rescale O_t by alpha before any PV MMA of this tile (warp-uniform
+          // because TMEM access is warp-collective; rows that keep their
+          // reference multiply by exactly 1).  O_t is complete: the commit
+          // that signalled S_t also covered the previous PV.
+#pragma unroll 1
+          for (int c = 0; c < D; c += 8) {
+            uint32_t o[8];
+            tmem_ld8(tO + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st8(tO + c, o);
+          }
+        }
+        tmem_st32(tS + 32 * h, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p + 16 * t + 8 * h);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p + 8 * t);
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(acc[0], a0, a1);
+        f2_unpack(acc[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
     }
     // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait(bar_o + 8 * t, 0, abort_flag, kWaitLimitNs);
