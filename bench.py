@@ -53,6 +53,41 @@ def peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+KERNEL_SOURCES = ("video_dit_sequence_b200/csrc/attention.cuh", "video_dit_sequence_b200/csrc/sm100.cuh")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "attention_kernel_dram_traffic.md")
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(cfg):
+    """DRAM bytes per launch of the attention kernel for this workload, from
+    the ncu record in profiles/, or None when the record is missing, is for
+    another workload, or was taken on a different kernel source."""
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            text = f.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != kernel_source_sha():
+        return None
+    try:
+        return float(fields[f"traffic_bytes_per_launch_{cfg.name}"])
+    except (KeyError, ValueError):
+        return None
+
+
 def workload_desc(cfg):
     s = cfg.shape
     g = "x".join(str(x) for x in cfg.grid) if cfg.grid[0] else "-"
@@ -186,6 +221,11 @@ def run_ours(args):
 
     sp.load()
     cfg = synth.CONFIGS[args.config]
+    if args.tokens:
+        # a smaller token count of the same layout (profiling captures)
+        import dataclasses
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}-N{args.tokens}",
+                                  shape=dataclasses.replace(cfg.shape, N=args.tokens))
     s = cfg.shape
     shape = sp.Shape(s.B, s.N, s.H, s.D, s.P)
     flops = s.flops()
@@ -317,7 +357,8 @@ def run_ours(args):
                 "frac": achieved / pk["bf16_tflops"],
                 "peak_kind": f"{pkq} bf16 dense (burst)",
                 "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
-                "traffic": args.traffic_bytes,
+                "traffic": args.traffic_bytes if args.traffic_bytes else recorded_traffic(cfg),
+                "kernel_source_sha256": kernel_source_sha(),
                 "flops_per_launch": flops}
 
     cpu = None
@@ -352,6 +393,8 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override N (same heads, head dim and degree); for profiling captures")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per launch of the attention kernel from an ncu capture")
     args = ap.parse_args()

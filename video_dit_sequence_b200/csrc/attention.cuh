@@ -172,25 +172,34 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);
+      // Shared-memory descriptors are built once; an operand's start address
+      // lives in the low 14 bits (address >> 4), so moving to another tile,
+      // slot or K step is one integer add (all addresses stay below 256 KB).
+      // This keeps the issuing thread far below the tensor core's 64 cycles
+      // per 128 x 128 x 16 MMA although it shares its SM sub-partition with
+      // two softmax warps.
+      const uint64_t dQ = make_sdesc_sw128(sbase + C::kOffQ, 16, 1024);
+      const uint64_t dK = make_sdesc_sw128(sbase + C::kOffKV, 16, 1024);
+      const uint64_t dV = make_sdesc_sw128(sbase + C::kOffKV, C::kBlockBytes, 1024);
       auto issue_s = [&](int t, int slot) {
-        const uint32_t qa = sbase + C::kOffQ + t * C::kTileBytes;
-        const uint32_t kb = sbase + C::kOffKV + slot * C::kTileBytes;
+        const uint64_t a0 = dQ + static_cast<uint32_t>((t * C::kTileBytes) >> 4);
+        const uint64_t b0 = dK + static_cast<uint32_t>((slot * C::kTileBytes) >> 4);
+        const uint32_t d = tmem + (t ? C::kColS1 : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          umma_ss(tmem + (t ? C::kColS1 : 0u), make_sdesc_sw128(qa + off, 16, 1024),
-                  make_sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4;
+          umma_ss(d, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t[:, 64h .. 64h+63] V_j[64h .. 64h+63, :] for key half h.
       auto issue_pv_half = [&](int t, int slot, bool first, int h) {
-        const uint32_t vb = sbase + C::kOffKV + slot * C::kTileBytes;
-        const uint32_t pcol = t ? C::kColS1 : 0u;
-        const uint32_t ocol = t ? C::kColO1 : C::kColO0;
+        const uint64_t b0 = dV + static_cast<uint32_t>((slot * C::kTileBytes) >> 4);
+        const uint32_t a0 = tmem + (t ? C::kColS1 : 0u);
+        const uint32_t d = tmem + (t ? C::kColO1 : C::kColO0);
 #pragma unroll
-        for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
-          umma_ts(tmem + ocol, tmem + pcol + kk * 8,
-                  make_sdesc_sw128(vb + kk * 16 * 128, C::kBlockBytes, 1024), idesc_pv,
+        for (int k = 0; k < 4; ++k) {
+          const int kk = 4 * h + k;
+          umma_ts(d, a0 + kk * 8, b0 + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_pv,
                   (first && kk == 0) ? 0u : 1u);
         }
       };
@@ -278,18 +287,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int c = 0; c < 128; ++c)
           if (c >= tail) s[c] = 0xFF800000u;  // -inf
       }
-      // Row maximum: four independent chains of 3-input max.
-      float mc[4];
+      // Row maximum: eight independent chains of 3-input max over 16
+      // scores each, then a short tree.
+      float mc[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t *e = &s[32 * q];
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t *e = &s[16 * q];
         float m = fmax3(__uint_as_float(e[0]), __uint_as_float(e[1]), __uint_as_float(e[2]));
 #pragma unroll
-        for (int c = 3; c < 31; c += 2)
+        for (int c = 3; c < 15; c += 2)
           m = fmax3(m, __uint_as_float(e[c]), __uint_as_float(e[c + 1]));
-        mc[q] = fmaxf(m, __uint_as_float(e[31]));
+        mc[q] = fmaxf(m, __uint_as_float(e[15]));
       }
-      const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * sl2;
+      const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
+                             fmaxf(mc[6], mc[7])) * sl2;
       const bool need = mx > m_ref + 8.0f;
       const bool warp_rescale = __any_sync(0xffffffffu, need);
       const float alpha = need ? ex2(m_ref - mx) : 1.0f;
