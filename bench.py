@@ -88,6 +88,24 @@ def recorded_traffic(cfg):
         return None
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's time: an all-reduce MAX over the default process
+    group (NCCL on the GPU machine, gloo in the CPU tests)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, steps: int, flops_per_step: float, t_max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs `steps` steps of its own problem;
+    the job takes as long as its slowest rank."""
+    return world * steps * flops_per_step / (t_max_ms * 1e-3) / 1e12
+
+
 def workload_desc(cfg):
     s = cfg.shape
     g = "x".join(str(x) for x in cfg.grid) if cfg.grid[0] else "-"
@@ -271,13 +289,8 @@ def run_ours(args):
     if sp.device_status(stream) != sp.SP_OK:
         raise SystemExit("device status not ok after the timed steps")
     t_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([t_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-    else:
-        t_max = t_ms
-    value = world * args.steps * flops / (t_max * 1e-3) / 1e12
+    t_max = max_over_ranks(t_ms, world, dev)
+    value = weak_scaling_value(world, args.steps, flops, t_max)
     per_launch_ms = t_ms / args.steps
 
     # ---- unfused rows: pack (Q, K, V), attention on head-sharded, unpack (O)
@@ -340,12 +353,8 @@ def run_ours(args):
         b.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        te = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([te], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            te = float(t.item())
-        e2e = {"value": world * args.steps * flops / (te * 1e-3) / 1e12, "unit": UNIT,
+        te = max_over_ranks(a.elapsed_time(b), world, dev)
+        e2e = {"value": weak_scaling_value(world, args.steps, flops, te), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * tensor_bytes), "d2h_bytes_per_step": int(tensor_bytes),
                "ms_per_step": te / args.steps}
         if sp.device_status(stream) != sp.SP_OK:

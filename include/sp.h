@@ -105,9 +105,10 @@ sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh,
  * from the sequence-sharded buffers and writes O into the sequence-sharded
  * layout; no intermediate buffers.  Bit-identical to the three-call path.
  * qs, ks, vs: device [P][B][Nl][H][D] bf16, read only.  os: device, same
- * shape, written.  lse: device fp32 [B][H][Np] or NULL.  Supports B == 1 or
- * P == 1 (the layouts in which a token tile is one strided block); other
- * shapes return SP_ERR_SHAPE (use the three-call path). */
+ * shape, written.  lse: device fp32 [B][H][Np] or NULL.  With B > 1 and
+ * P > 1 a token tile that crosses a shard boundary is gathered row by row
+ * (slower than the TMA path used for every other tile and shape); padding
+ * slots of qs/ks/vs must then be zero, as for sp_pack. */
 sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs,
                                   void *os, float *lse, const sp_shape *shape,
                                   void *stream);

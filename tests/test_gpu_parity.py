@@ -176,6 +176,26 @@ def test_batch_and_degree_one_fused_and_unfused():
     _check_rows(f1, q, k, v, _rows_all(B, N, H), 1, "B=3")
 
 
+@pytest.mark.parametrize("B,N,H,D,P", [(2, 1000, 8, 128, 4), (3, 300, 8, 64, 8),
+                                        (2, 1024, 4, 128, 2), (2, 9450, 8, 128, 8),
+                                        (4, 257, 2, 128, 2)])
+def test_fused_rank_major_batches(B, N, H, D, P):
+    """B > 1 with P > 1: rank-major shards, tiles that cross shard
+    boundaries (Nl = 250, 38 < 128, 512, 1182, 129); fused equals the
+    three-call path bit for bit, and P = 1, and the oracle."""
+    q, k, v = _random_logical(B, N, H, D, seed=B * N + P)
+    fused, lse_f = _run_fused(q, k, v, P, lse=True)
+    unfused, lse_u = _run_unfused(q, k, v, P, lse=True)
+    assert np.array_equal(fused, unfused)
+    assert np.array_equal(lse_f, lse_u)
+    one, _ = _run_fused(q, k, v, 1)
+    assert np.array_equal(synth.from_seq_shards(fused.reshape(P, B, -1, H, D), N),
+                          synth.from_seq_shards(one.reshape(1, B, -1, H, D), N))
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H)
+                     for i in sorted({0, N - 1, *range(0, N, max(1, N // 40))})], dtype=np.int64)
+    _check_rows(fused, q, k, v, rows, P, f"B={B} N={N} P={P}")
+
+
 @pytest.mark.parametrize("N", [1000, 4096])
 def test_degrees_bit_identical(N):
     """SP output equals single-GPU output bit for bit, for every degree."""

@@ -233,7 +233,8 @@ def ulysses_attention(q, k, v, P: int, scale: float = 0.0, fused: bool = True):
     """User-level call: q, k, v are [B, N, H, D] bf16 CUDA tensors (logical,
     unsharded); returns O [B, N, H, D].  The tensors are laid out as P
     sequence shards (zero-padded to Np tokens), attended with P virtual ranks
-    and read back.  fused=False runs pack -> attention -> unpack."""
+    and read back.  fused=False runs pack -> attention -> unpack instead of
+    the fused kernel."""
     torch = _torch()
     B, N, H, D = q.shape
     shape = Shape(B, N, H, D, P, scale)
@@ -246,7 +247,7 @@ def ulysses_attention(q, k, v, P: int, scale: float = 0.0, fused: bool = True):
 
     qs, ks, vs = shards(q), shards(k), shards(v)
     os_ = torch.empty_like(qs)
-    if fused and (B == 1 or P == 1):
+    if fused:
         attention_seqsharded(qs, ks, vs, os_, shape)
     else:
         hs = shape.head_sharded

@@ -51,6 +51,11 @@ struct AttnParams {
   __nv_bfloat16 *o;     // output base
   int64_t o_row;        // elements between consecutive tokens
   int64_t o_batch;      // elements between tensor-map batch slots
+  // Rank-major sequence shards with B > 1 and P > 1 ([P][B][Nl][H][D]):
+  // nl_split = Nl (else 0); token t lives in rank t / Nl at local row t % Nl.
+  int32_t nl_split;
+  int64_t o_rank;       // elements between rank slabs (B * Nl * H * D)
+  const __nv_bfloat16 *q, *k, *v;  // bases, for tiles that cross a shard boundary
   float *lse;           // [B][H][Np] or null
   int32_t *status;      // device status word
 };
@@ -138,35 +143,91 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
   bool ok = true;
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
+    // One elected lane issues the TMA loads.  In the rank-major layout a
+    // 128-token tile that crosses a shard boundary is two strided blocks,
+    // which one TMA box cannot describe: the whole warp copies such a tile
+    // with 16-byte loads into the same 128-byte-swizzled layout the TMA
+    // writes (16-byte chunk c of row r at chunk c ^ (r mod 8)), fences the
+    // generic-proxy writes for the async proxy, and arrives without bytes.
+    const uint64_t pol_q = policy_evict_first();
+    const uint64_t pol_kv = policy_evict_last();
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const uint64_t pol_q = policy_evict_first();
-      const uint64_t pol_kv = policy_evict_last();
-      mbar_arrive_expect_tx(bar_q, 2 * C::kTileBytes);
-      for (int t = 0; t < 2; ++t)
+    }
+    const int nl = p.nl_split;
+    auto tma_ok = [&](int t0) {
+      if (nl == 0) return true;
+      const int r0 = t0 / nl;
+      return t0 - r0 * nl + C::kBM <= nl;
+    };
+    auto tma_tile = [&](const CUtensorMap *m, uint32_t dst, uint32_t bar, int t0, uint64_t pol) {
+      if (nl == 0) {
         for (int h = 0; h < C::kHalves; ++h)
-          tma_load_4d(sbase + C::kOffQ + t * C::kTileBytes + h * C::kBlockBytes, &tmQ, bar_q,
-                      h * 64, map_head, q0 + t * C::kBM, map_batch, pol_q);
-      int it = 0;
-      for (int j = 0; j < T && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1;
-          if (!mbar_wait(bar_kv_empty + 8 * s, ph ^ 1u, abort_flag, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar_kv_full + 8 * s, C::kTileBytes);
-          const CUtensorMap *m = kv == 0 ? &tmK : &tmV;
-          for (int h = 0; h < C::kHalves; ++h)
-            tma_load_4d(sbase + C::kOffKV + s * C::kTileBytes + h * C::kBlockBytes, m,
-                        bar_kv_full + 8 * s, h * 64, map_head, j * C::kBN, map_batch, pol_kv);
-        }
+          tma_load_4d(dst + h * C::kBlockBytes, m, bar, h * 64, map_head, t0, map_batch, pol);
+      } else {
+        const int r0 = t0 / nl;
+        for (int h = 0; h < C::kHalves; ++h)
+          tma_load_5d(dst + h * C::kBlockBytes, m, bar, h * 64, map_head, t0 - r0 * nl, b, r0,
+                      pol);
       }
+    };
+    auto copy_tile = [&](const __nv_bfloat16 *base, uint32_t dst, int t0) {
+      constexpr int kChunks = D / 8;  // 16-byte chunks per token row
+      for (int idx = lane; idx < C::kBM * kChunks; idx += 32) {
+        const int r = idx / kChunks, cc = idx % kChunks;
+        const int tok = t0 + r;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (tok < p.N) {
+          const int rk = tok / nl, n = tok - rk * nl;
+          const int64_t off = ((static_cast<int64_t>(rk) * p.B + b) * nl + n) * p.H * D +
+                              static_cast<int64_t>(map_head) * D + cc * 8;
+          val = ld_global_nc_v4(base + off);
+        }
+        st_shared_v4(dst + (cc >> 3) * C::kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4), val);
+      }
+      fence_proxy_async_smem();
+    };
+    // Q: both tiles complete one barrier.
+    uint32_t q_tx = 0;
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t dst = sbase + C::kOffQ + t * C::kTileBytes;
+      if (tma_ok(q0 + t * C::kBM)) q_tx += C::kTileBytes;
+      else copy_tile(p.q, dst, q0 + t * C::kBM);
     }
     __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, q_tx);
+      for (int t = 0; t < 2; ++t)
+        if (tma_ok(q0 + t * C::kBM))
+          tma_tile(&tmQ, sbase + C::kOffQ + t * C::kTileBytes, bar_q, q0 + t * C::kBM, pol_q);
+    }
+    int it = 0;
+    for (int j = 0; j < T && ok; ++j) {
+      for (int kv = 0; kv < 2; ++kv, ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        const bool free_slot = mbar_wait(bar_kv_empty + 8 * s, ph ^ 1u, abort_flag, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, free_slot)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = sbase + C::kOffKV + s * C::kTileBytes;
+        const uint32_t bar = bar_kv_full + 8 * s;
+        if (tma_ok(j * C::kBN)) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar, C::kTileBytes);
+            tma_tile(kv == 0 ? &tmK : &tmV, dst, bar, j * C::kBN, pol_kv);
+          }
+        } else {
+          copy_tile(kv == 0 ? p.k : p.v, dst, j * C::kBN);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar);
+        }
+        __syncwarp();
+      }
+    }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
@@ -364,8 +425,15 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       const bool valid = token < p.N;
       const bool exists = token < p.Np;
       const float inv_l = valid ? 1.0f / l : 0.0f;
-      __nv_bfloat16 *dst = p.o + static_cast<int64_t>(map_batch) * p.o_batch +
-                           static_cast<int64_t>(token) * p.o_row + static_cast<int64_t>(map_head) * D;
+      int64_t row_off;
+      if (p.nl_split) {
+        const int rk = token / p.nl_split, n = token - rk * p.nl_split;
+        row_off = static_cast<int64_t>(rk) * p.o_rank + static_cast<int64_t>(b) * p.o_batch +
+                  static_cast<int64_t>(n) * p.o_row;
+      } else {
+        row_off = static_cast<int64_t>(map_batch) * p.o_batch + static_cast<int64_t>(token) * p.o_row;
+      }
+      __nv_bfloat16 *dst = p.o + row_off + static_cast<int64_t>(map_head) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];

@@ -128,6 +128,27 @@ bool make_map(CUtensorMap *m, const void *base, int D, int Hx, int N, int Bx, in
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over rank-major sequence shards [P][B][Nl][H][D] (B > 1 and
+// P > 1), dims inner to outer (D, H, Nl, B, P).  Used only for token tiles
+// that lie inside one shard; the box is 128 rows (or Nl when smaller, in
+// which case no tile uses the map).
+bool make_map5(CUtensorMap *m, const void *base, int D, int H, int Nl, int B, int P) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(H) * D * 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(Nl), static_cast<cuuint64_t>(B),
+                        static_cast<cuuint64_t>(P)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * 2, row, row * Nl,
+                           row * Nl * static_cast<cuuint64_t>(B)};
+  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(Nl < 128 ? Nl : 128), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const sp::AttnParams &p, int B, cudaStream_t cs) {
@@ -169,13 +190,13 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   const int Np = Nl * P;
   int Hx, Bx, hsplit;
   int64_t row_el, batch_el;
+  const bool rank_major = seqsharded && B > 1 && P > 1;
   if (seqsharded) {
-    if (B > 1 && P > 1) return SP_ERR_SHAPE;
     Hx = H;
     hsplit = H;
     Bx = B;
     row_el = static_cast<int64_t>(H) * D;
-    batch_el = static_cast<int64_t>(Nl) * H * D;  // P == 1 when B > 1
+    batch_el = static_cast<int64_t>(Nl) * H * D;  // one rank's [B][Nl] rows
   } else {
     Hx = Hl;
     hsplit = Hl;
@@ -186,10 +207,15 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   int32_t *status = status_ptr();
   if (status == nullptr) return SP_ERR_CUDA;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, Hx, N, Bx, row_el, batch_el) ||
-      !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el) ||
-      !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el))
+  if (rank_major) {
+    if (!make_map5(&mq, q, D, H, Nl, B, P) || !make_map5(&mk, k, D, H, Nl, B, P) ||
+        !make_map5(&mv, v, D, H, Nl, B, P))
+      return SP_ERR_CUDA;
+  } else if (!make_map(&mq, q, D, Hx, N, Bx, row_el, batch_el) ||
+             !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el) ||
+             !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el)) {
     return SP_ERR_CUDA;
+  }
   sp::AttnParams p;
   p.N = N;
   p.Np = Np;
@@ -204,6 +230,11 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   p.o_batch = batch_el;
   p.lse = lse;
   p.status = status;
+  p.nl_split = rank_major ? Nl : 0;
+  p.o_rank = static_cast<int64_t>(B) * Nl * H * D;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.k = static_cast<const __nv_bfloat16 *>(k);
+  p.v = static_cast<const __nv_bfloat16 *>(v);
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   cudaError_t e = D == 64 ? launch_attention<64>(mq, mk, mv, p, B, cs)
                           : launch_attention<128>(mq, mk, mv, p, B, cs);
