@@ -7,6 +7,9 @@ with it.
 
 What it computes, and the passages it follows:
 
+* ``exchange_pack`` / ``exchange_unpack`` -- the same exchange seen from one
+  rank when every rank is its own GPU: the send-buffer reorder in front of
+  the all-to-all and the reverse reorder after the return all-to-all.
 * ``pack`` / ``unpack`` -- the token<->head all-to-all of the fal.ai page
   "Generate video with WAN 2.2 across four GPUs", section "Splitting one
   generation across four GPUs" (each GPU sees the full sequence for its share
@@ -49,7 +52,8 @@ def _bind(path: str):
     lib = ctypes.CDLL(path)
     i64 = ctypes.c_int64
     vp = ctypes.c_void_p
-    for name in ("sp_oracle_pack", "sp_oracle_unpack"):
+    for name in ("sp_oracle_pack", "sp_oracle_unpack", "sp_oracle_exchange_pack",
+                 "sp_oracle_exchange_unpack"):
         f = getattr(lib, name)
         f.argtypes = [vp, vp, i64, i64, i64, i64, i64]
         f.restype = ctypes.c_int
@@ -111,6 +115,32 @@ def unpack(oh: np.ndarray, N: int, H: int, lib=None) -> np.ndarray:
     oh = np.ascontiguousarray(oh)
     out = np.empty((P, B, Nl, H, D), dtype=np.uint16)
     rc = (lib or _load()).sp_oracle_unpack(oh.ctypes.data, out.ctypes.data, B, N, H, D, P)
+    assert rc == 0
+    return out
+
+
+def exchange_pack(xs_r: np.ndarray, N: int, P: int, lib=None) -> np.ndarray:
+    """One rank's shard [B][Nl][H][D] -> its P send chunks [P][B][Nl][Hl][D]."""
+    assert xs_r.dtype == np.uint16 and xs_r.ndim == 4
+    B, Nl, H, D = xs_r.shape
+    assert Nl == _dims(N, P)[0]
+    if H % P:
+        raise ValueError("the Ulysses degree must divide the head count")
+    xs_r = np.ascontiguousarray(xs_r)
+    out = np.empty((P, B, Nl, H // P, D), dtype=np.uint16)
+    rc = (lib or _load()).sp_oracle_exchange_pack(xs_r.ctypes.data, out.ctypes.data, B, N, H, D, P)
+    assert rc == 0
+    return out
+
+
+def exchange_unpack(recv: np.ndarray, N: int, H: int, lib=None) -> np.ndarray:
+    """The P chunks returned to one rank [P][B][Nl][Hl][D] -> its shard [B][Nl][H][D]."""
+    assert recv.dtype == np.uint16 and recv.ndim == 5
+    P, B, Nl, Hl, D = recv.shape
+    assert Nl == _dims(N, P)[0] and Hl * P == H
+    recv = np.ascontiguousarray(recv)
+    out = np.empty((B, Nl, H, D), dtype=np.uint16)
+    rc = (lib or _load()).sp_oracle_exchange_unpack(recv.ctypes.data, out.ctypes.data, B, N, H, D, P)
     assert rc == 0
     return out
 

@@ -95,6 +95,49 @@ int sp_oracle_unpack(const uint16_t *oh, uint16_t *os, int64_t B, int64_t N,
 }
 
 /*
+ * Exchange pack on one rank (the send-buffer reorder in front of the
+ * all-to-all of "Splitting one generation across four GPUs" when every rank
+ * is its own GPU): rank r's shard xs_r [B][Nl][H][D] becomes P send chunks,
+ * chunk j holding r's tokens for head group j:
+ *     send[j][b][n][hh][c] = xs_r[b][n][j*Hl + hh][c]
+ * After the all-to-all, rank j holds chunk j of every rank r in rank order,
+ * [P][B][Nl][Hl][D]: the full sequence for its heads.
+ */
+int sp_oracle_exchange_pack(const uint16_t *xs_r, uint16_t *send, int64_t B, int64_t N,
+                            int64_t H, int64_t D, int64_t P) {
+    if (P < 1 || H % P != 0) return -1;
+    int64_t Hl = H / P, Nl = (N + P - 1) / P;
+    for (int64_t j = 0; j < P; ++j)
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t n = 0; n < Nl; ++n)
+                for (int64_t hh = 0; hh < Hl; ++hh)
+                    for (int64_t c = 0; c < D; ++c)
+                        send[(((j * B + b) * Nl + n) * Hl + hh) * D + c] =
+                            xs_r[((b * Nl + n) * H + (j * Hl + hh)) * D + c];
+    return 0;
+}
+
+/*
+ * Exchange unpack on one rank ("the shards return to their own GPUs"): the
+ * P chunks received back from the head groups, recv[j][b][n][hh][c] (group
+ * j's output for this rank's tokens), become the shard [B][Nl][H][D]:
+ *     os_r[b][n][j*Hl + hh][c] = recv[j][b][n][hh][c]
+ */
+int sp_oracle_exchange_unpack(const uint16_t *recv, uint16_t *os_r, int64_t B, int64_t N,
+                              int64_t H, int64_t D, int64_t P) {
+    if (P < 1 || H % P != 0) return -1;
+    int64_t Hl = H / P, Nl = (N + P - 1) / P;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t n = 0; n < Nl; ++n)
+            for (int64_t j = 0; j < P; ++j)
+                for (int64_t hh = 0; hh < Hl; ++hh)
+                    for (int64_t c = 0; c < D; ++c)
+                        os_r[((b * Nl + n) * H + (j * Hl + hh)) * D + c] =
+                            recv[(((j * B + b) * Nl + n) * Hl + hh) * D + c];
+    return 0;
+}
+
+/*
  * Attention for a list of query rows of the unsharded problem.
  *
  * For query row i of batch b and head h, with scores

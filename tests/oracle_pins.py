@@ -107,6 +107,43 @@ def check_pack_degree_one_is_copy(lib=None):
     assert np.array_equal(oracle.unpack(xs, 11, 4, lib=lib), xs)
 
 
+def check_exchange_chunks_hold_head_groups(lib=None):
+    """On rank r, send chunk j holds r's tokens for heads j*Hl..(j+1)*Hl-1;
+    the return reorder puts every group's chunk back at its heads."""
+    rng = np.random.default_rng(RNG_SEED + 4)
+    for (B, N, H, D, P) in PACK_SHAPES:
+        Nl, Hl = -(-N // P), H // P
+        X = _codes((B, N, H, D), rng)
+        X[X == 0] = 1  # keep zero for the padding check
+        xs = synth.to_seq_shards(X, P)
+        for r in range(P):
+            send = oracle.exchange_pack(xs[r], N, P, lib=lib)
+            lo, hi = r * Nl, max(r * Nl, min(N, (r + 1) * Nl))
+            for j in range(P):
+                assert np.array_equal(send[j][:, : hi - lo], X[:, lo:hi, j * Hl:(j + 1) * Hl])
+                assert not send[j][:, hi - lo:].any()  # padding slots stay zero
+            assert np.array_equal(oracle.exchange_unpack(send, N, H, lib=lib), xs[r])
+
+
+def check_exchange_matches_numpy_and_single_gpu_pack(lib=None):
+    """numpy formulation ([B*Nl][P][Hl*D] -> [P][B*Nl][Hl*D]); and the
+    all-to-all of the P ranks' chunks (chunk j of rank r to rank j, in rank
+    order) is exactly the one-GPU head-sharded pack for B = 1."""
+    rng = np.random.default_rng(RNG_SEED + 5)
+    for (B, N, H, D, P) in PACK_SHAPES:
+        Nl, Hl = -(-N // P), H // P
+        xs = _codes((P, B, Nl, H, D), rng)
+        sends = [oracle.exchange_pack(xs[r], N, P, lib=lib) for r in range(P)]
+        for r in range(P):
+            ref = xs[r].reshape(B * Nl, P, Hl * D).transpose(1, 0, 2).reshape(P, B, Nl, Hl, D)
+            assert np.array_equal(sends[r], ref)
+        if B == 1:
+            xh = oracle.pack(xs, N, lib=lib)
+            for j in range(P):
+                recv_j = np.concatenate([sends[r][j] for r in range(P)], axis=1)
+                assert np.array_equal(recv_j, xh[j])
+
+
 # ---------------------------------------------------------------- attention
 
 def _np_attention(q, k, v, scale=None):
@@ -257,7 +294,9 @@ def check_rows_api(lib=None):
 
 
 PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
-               check_unpack_returns_shards, check_pack_degree_one_is_copy]
+               check_unpack_returns_shards, check_pack_degree_one_is_copy,
+               check_exchange_chunks_hold_head_groups,
+               check_exchange_matches_numpy_and_single_gpu_pack]
 ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one,
                     check_closed_forms, check_dominant_key, check_invariances,
                     check_two_token_example, check_rows_api]

@@ -18,6 +18,12 @@ MUTANTS = [
     ("pack-wrong-local-head",
      "(j * Hl + hh)) * D + c;\n                            int64_t dst",
      "(j * Hl + (Hl - 1 - hh))) * D + c;\n                            int64_t dst"),
+    ("exchange-pack-wrong-head",
+     "xs_r[((b * Nl + n) * H + (j * Hl + hh)) * D + c];",
+     "xs_r[((b * Nl + n) * H + (hh * P + j)) * D + c];"),
+    ("exchange-unpack-wrong-chunk",
+     "recv[(((j * B + b) * Nl + n) * Hl + hh) * D + c];",
+     "recv[((((P - 1 - j) * B + b) * Nl + n) * Hl + hh) * D + c];"),
     ("scale-dropped", "s[kk] = J->scale * dot;", "s[kk] = dot;"),
     ("lse-sign", "m + log(l)", "m - log(l)"),
     ("no-normalisation", "o[c] /= l;", "o[c] /= 1.0;"),
