@@ -17,7 +17,10 @@ far larger than the 126 MB L2, so no L2 flush is done between steps.
 
 With --gpus N > 1 (launched by torchrun, one rank per GPU) every rank runs
 the same single-GPU problem on its own GPU: independent problems, no
-data-path collective, weak scaling.
+data-path collective, weak scaling.  --mode ulysses instead splits the one
+problem across the N GPUs the way the method does (P = N ranks, NCCL
+all-to-all of the sequence shards, each GPU attends H/N heads over the whole
+sequence, all-to-all back): strong scaling.
 
 --impl reference times the fp64 CPU oracle on the host cores instead, each
 step a bounded sample (query rows) of the same workload.
@@ -213,6 +216,115 @@ def run_reference(args):
     return 0
 
 
+def run_ulysses(args):
+    """--mode ulysses with N > 1: the multi-GPU form, one rank per GPU."""
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import video_dit_sequence_b200 as sp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # one rank without torchrun: a single-member group, the exchange a self-copy
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29533")
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev,
+                            rank=rank, world_size=world)
+    sp.load()
+    cfg = synth.CONFIGS[args.config]
+    s = cfg.shape
+    if s.H % world:
+        raise SystemExit(f"the degree {world} must divide the head count {s.H}")
+    shape = sp.Shape(s.B, s.N, s.H, s.D, world)
+    flops = s.flops()
+    q, k, v = synth.qkv_logical(cfg)
+
+    def pinned_shard(a):
+        shard = np.ascontiguousarray(synth.to_seq_shards(a, world)[rank])
+        return torch.from_numpy(shard.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+    hq, hk, hv = (pinned_shard(a) for a in (q, k, v))
+    ho = torch.empty(shape.rank_shard, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv = (h.to(dev) for h in (hq, hk, hv))
+    stream = torch.cuda.current_stream(dev)
+    a2a = sp.nccl_all_to_all()
+    out = [None]
+
+    def step():
+        out[0] = sp.ulysses_attention_distributed(dq, dk, dv, shape, a2a)
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        return a.elapsed_time(b)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if sp.device_status(stream) != sp.SP_OK:
+        raise SystemExit("device status not ok after warm-up")
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = str(local)
+    sampler = ClockSampler(uuid)
+    time.sleep(0.3)
+    n0 = sp.launch_count()
+    t_ms = timed(step)
+    launches = sp.launch_count() - n0
+    clocks = sampler.stop()
+    t_max = max_over_ranks(t_ms, world, dev)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        step()
+        ho.copy_(out[0], non_blocking=True)
+
+    te = max_over_ranks(timed(e2e_step), world, dev)
+    if sp.device_status(stream) != sp.SP_OK:
+        raise SystemExit("device status not ok after the timed steps")
+    pk, pkq = peaks()
+    per_gpu = flops / world / (t_max / args.steps * 1e-3) / 1e12
+    shard_bytes = 2 * math.prod(shape.rank_shard)
+    if rank == 0:
+        line = {"metric": METRIC, "value": args.steps * flops / (t_max * 1e-3) / 1e12,
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+                "ms_per_step": t_max / args.steps, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": dict(workload_desc(cfg), P=world, parallelism=f"ulysses{world}",
+                               exchange="NCCL all_to_all_single"),
+                "e2e": {"value": args.steps * flops / (te * 1e-3) / 1e12, "unit": UNIT,
+                        "h2d_bytes_per_step": int(3 * shard_bytes),
+                        "d2h_bytes_per_step": int(shard_bytes)},
+                "gpu_launches": int(launches), "clocks": clocks,
+                "roofline": {"bound": "tensor", "kernel": "whole step per GPU",
+                             "achieved": per_gpu, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": per_gpu / pk["bf16_tflops"],
+                             "peak_kind": f"{pkq} bf16 dense (burst)", "traffic": None},
+                "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -397,6 +509,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--mode", choices=["replicas", "ulysses"], default="replicas",
+                    help="N > 1 only: independent problems per GPU (default) or one problem "
+                         "split across the GPUs with the Ulysses all-to-all")
     ap.add_argument("--config", default="720p")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
@@ -409,6 +524,8 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode == "ulysses":
+        return run_ulysses(args)
     return run_ours(args)
 
 

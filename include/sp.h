@@ -87,6 +87,28 @@ sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream)
  * [P][B][Nl][H][D] bf16, written in full.  Bit-exact copy. */
 sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *stream);
 
+/* Exchange pack on one rank, for the form in which every rank is its own
+ * GPU: the send-buffer reorder in front of the all-to-all (same page
+ * section).  Rank r's shard becomes P send chunks, chunk j holding r's
+ * tokens for head group j:
+ *   send[j][b][n][hh][c] = xs_r[b][n][j*Hl + hh][c]
+ * After an all-to-all that delivers chunk j of every rank to rank j, in rank
+ * order, rank j holds [P][B][Nl][Hl][D]: the sequence-sharded layout of its
+ * Hl heads, which sp_attention_seqsharded with shape {B, N, Hl, D, P}
+ * attends directly.
+ * xs_r: device [B][Nl][H][D] bf16, read only.  send: device
+ * [P][B][Nl][Hl][D] bf16, written in full.  shape: the global problem
+ * (H % P == 0).  Bit-exact copy. */
+sp_status sp_exchange_pack(const void *xs_r, void *send, const sp_shape *shape, void *stream);
+
+/* Exchange unpack on one rank ("the shards return to their own GPUs"): the
+ * P chunks returned by the head groups, chunk j = group j's output for this
+ * rank's tokens, become the rank's shard:
+ *   os_r[b][n][j*Hl + hh][c] = recv[j][b][n][hh][c]
+ * recv: device [P][B][Nl][Hl][D] bf16, read only.  os_r: device
+ * [B][Nl][H][D] bf16, written in full.  Bit-exact copy. */
+sp_status sp_exchange_unpack(const void *recv, void *os_r, const sp_shape *shape, void *stream);
+
 /* Attention per head group on head-sharded tensors: for every batch b,
  * group j, local head hh (global head h = j*Hl + hh) and query token i < N,
  *   oh[j][b][i][hh] = sum_{k<N} softmax_k(q_i . k_k * scale) v_k
@@ -108,7 +130,9 @@ sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh,
  * shape, written.  lse: device fp32 [B][H][Np] or NULL.  With B > 1 and
  * P > 1 a token tile that crosses a shard boundary is gathered row by row
  * (slower than the TMA path used for every other tile and shape); padding
- * slots of qs/ks/vs must then be zero, as for sp_pack. */
+ * slots of qs/ks/vs must then be zero, as for sp_pack.  P describes only
+ * how the tokens are sharded (no heads are split), so H % P == 0 is not
+ * required here. */
 sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs,
                                   void *os, float *lse, const sp_shape *shape,
                                   void *stream);

@@ -94,8 +94,16 @@ def test_argument_errors_return_before_launch(lib):
         assert att(fn, A, A, A + 4, B_) == sp.SP_ERR_ALIGN
         assert att(fn, A, A, A, B_, 0x30002) == sp.SP_ERR_ALIGN
         assert att(fn, A, A, A, B_, shp=sp.Shape(1, 1024, 4, 80, 2)) == sp.SP_ERR_UNSUPPORTED_D
-        assert att(fn, A, A, A, B_, shp=sp.Shape(1, 1024, 4, 64, 3)) == \
-            sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    # heads are split only by the head-sharded call; the fused call shards
+    # tokens alone and accepts any degree
+    assert att(lib.sp_attention, A, A, A, B_, shp=sp.Shape(1, 1024, 4, 64, 3)) == \
+        sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    assert lib.sp_check_shape(ctypes.byref(sp.Shape(1, 1024, 4, 64, 3).c())) == \
+        sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    for fn in (lib.sp_exchange_pack, lib.sp_exchange_unpack):
+        assert _call(fn, 0, B_, shape=shape) == sp.SP_ERR_NULL
+        assert _call(fn, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN
+        assert _call(fn, A, B_, shape=bad) == sp.SP_ERR_HEADS_NOT_DIVISIBLE
     assert lib.sp_launch_count() == 0
 
 

@@ -134,6 +134,64 @@ def test_pack_full_size_bit_exact(name):
     _status_ok()
 
 
+EXCHANGE_SHAPES = [(1, 1024, 4, 64, 2), (2, 1000, 8, 128, 4), (3, 77, 6, 128, 3),
+                   (1, 4096, 40, 128, 8), (2, 9, 8, 128, 8)]
+
+
+@pytest.mark.parametrize("B,N,H,D,P", EXCHANGE_SHAPES)
+def test_exchange_pack_unpack_bit_exact(B, N, H, D, P):
+    shape = sp.Shape(B, N, H, D, P)
+    X = synth.normal_bf16(300 + N, 0, 0, B * N * H * D).reshape(B, N, H, D)
+    xs = synth.to_seq_shards(X, P)
+    for r in range(P):
+        want = oracle.exchange_pack(xs[r], N, P)
+        d_send = torch.full(shape.send_chunks, float("nan"), dtype=torch.bfloat16, device="cuda")
+        sp.exchange_pack(to_dev(xs[r]), d_send, shape)
+        assert np.array_equal(to_host(d_send).reshape(want.shape), want)
+        recv = synth.normal_bf16(400 + r, 1, 0, int(np.prod(shape.send_chunks))).reshape(shape.send_chunks)
+        want_u = oracle.exchange_unpack(recv, N, H)
+        d_os = torch.full(shape.rank_shard, float("nan"), dtype=torch.bfloat16, device="cuda")
+        sp.exchange_unpack(to_dev(recv), d_os, shape)
+        assert np.array_equal(to_host(d_os).reshape(want_u.shape), want_u)
+    _status_ok()
+
+
+def _virtual_ranks_ulysses(q, k, v, P):
+    """The multi-GPU form run as P virtual ranks in lockstep on one GPU: each
+    rank's phases in turn, the all-to-all as copies between their buffers
+    (no kernel waits on another)."""
+    B, N, H, D = q.shape
+    shape = sp.Shape(B, N, H, D, P)
+    shards = [to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v)]
+    ranks = [sp.UlyssesRank(shape) for _ in range(P)]
+    sends = [ranks[r].send_qkv(shards[0][r], shards[1][r], shards[2][r]) for r in range(P)]
+
+    def all_to_all(bufs):  # bufs[r][j] = rank r's chunk for rank j
+        return [torch.stack([bufs[r][j] for r in range(P)]).contiguous() for j in range(P)]
+
+    recv = [all_to_all([sends[r][t] for r in range(P)]) for t in range(3)]
+    outs = [ranks[j].attend(recv[0][j], recv[1][j], recv[2][j]) for j in range(P)]
+    back = all_to_all(outs)
+    res = torch.stack([ranks[r].finish(back[r]) for r in range(P)])
+    _status_ok()
+    return to_host(res)
+
+
+@pytest.mark.parametrize("B,N,H,D,P", [(1, 1024, 4, 64, 2), (1, 3000, 8, 128, 4),
+                                        (2, 1000, 8, 128, 4), (1, 4099, 40, 128, 8),
+                                        (3, 300, 16, 64, 8)])
+def test_multi_gpu_form_on_virtual_ranks(B, N, H, D, P):
+    """Exchange pack -> all-to-all -> per-group fused attention -> all-to-all
+    -> exchange unpack gives the one-GPU result bit for bit."""
+    q, k, v = _random_logical(B, N, H, D, seed=7 * N + P)
+    got = _virtual_ranks_ulysses(q, k, v, P)
+    one, _ = _run_fused(q, k, v, P)
+    assert np.array_equal(got.reshape(one.shape), one)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H)
+                     for i in sorted({0, N - 1, *range(0, N, max(1, N // 24))})], dtype=np.int64)
+    _check_rows(got, q, k, v, rows, P, f"virtual ranks B={B} N={N} P={P}")
+
+
 # ------------------------------------------------------------------ attention, small
 
 def test_tiny_config_every_row():

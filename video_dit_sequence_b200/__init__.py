@@ -40,7 +40,8 @@ SP_ERR_TIMEOUT = 7
 
 EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_attention", "sp_attention_seqsharded", "sp_device_status",
-            "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout")
+            "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout",
+            "sp_exchange_pack", "sp_exchange_unpack")
 
 
 class sp_shape(ctypes.Structure):
@@ -71,7 +72,7 @@ def load(path: str = LIB_PATH):
     lib.sp_padded_tokens.restype = ctypes.c_int64
     lib.sp_check_shape.argtypes = [sp_p]
     lib.sp_check_shape.restype = ctypes.c_int
-    for name in ("sp_pack", "sp_unpack"):
+    for name in ("sp_pack", "sp_unpack", "sp_exchange_pack", "sp_exchange_unpack"):
         f = getattr(lib, name)
         f.argtypes = [vp, vp, sp_p, vp]
         f.restype = ctypes.c_int
@@ -124,6 +125,21 @@ class Shape:
     @property
     def head_sharded(self):
         return (self.P, self.B, self.Np, self.Hl, self.D)
+
+    @property
+    def rank_shard(self):
+        """One rank's shard when every rank is its own GPU: [B][Nl][H][D]."""
+        return (self.B, self.Nl, self.H, self.D)
+
+    @property
+    def send_chunks(self):
+        """One rank's P exchange chunks: [P][B][Nl][Hl][D]."""
+        return (self.P, self.B, self.Nl, self.Hl, self.D)
+
+    def head_group(self) -> "Shape":
+        """The problem one head group attends after the exchange: Hl heads
+        over the whole sequence, still in P token shards."""
+        return Shape(self.B, self.N, self.Hl, self.D, self.P, self.scale)
 
     @property
     def lse_shape(self):
@@ -216,6 +232,88 @@ def attention_seqsharded(qs, ks, vs, os_, shape: Shape, lse=None, stream=None):
         _ptr(qs, ss, "qs"), _ptr(ks, ss, "ks"), _ptr(vs, ss, "vs"), _ptr(os_, ss, "os"),
         _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
         _stream(stream, qs.device)), "sp_attention_seqsharded")
+
+
+def exchange_pack(xs_r, send, shape: Shape, stream=None):
+    """One rank's shard [B][Nl][H][D] -> its P send chunks [P][B][Nl][Hl][D]."""
+    s = shape.c()
+    _check(load().sp_exchange_pack(_ptr(xs_r, shape.rank_shard, "xs_r"),
+                                   _ptr(send, shape.send_chunks, "send"), ctypes.byref(s),
+                                   _stream(stream, xs_r.device)), "sp_exchange_pack")
+
+
+def exchange_unpack(recv, os_r, shape: Shape, stream=None):
+    """The P chunks returned to one rank [P][B][Nl][Hl][D] -> its shard."""
+    s = shape.c()
+    _check(load().sp_exchange_unpack(_ptr(recv, shape.send_chunks, "recv"),
+                                     _ptr(os_r, shape.rank_shard, "os_r"), ctypes.byref(s),
+                                     _stream(stream, recv.device)), "sp_exchange_unpack")
+
+
+class UlyssesRank:
+    """One rank of Ulysses attention when every rank is its own GPU (the
+    form of fal.ai's "Splitting one generation across four GPUs").
+
+    The step has three local phases around two all-to-alls:
+      send_qkv(q, k, v)   shard [B][Nl][H][D] -> three [P][B][Nl][Hl][D]
+                          chunk sets (sp_exchange_pack)
+      -- all-to-all: chunk j of every rank to rank j, in rank order --
+      attend(q, k, v)     this rank's head group over the whole sequence, on
+                          the received rank-major shards (fused attention,
+                          Hl heads, P token shards); the output is already
+                          in chunk order for the way back
+      -- all-to-all back --
+      finish(back)        P returned chunks -> this rank's output shard
+                          (sp_exchange_unpack)
+    Keeping the phases apart lets the caller choose the exchange (NCCL over
+    NVLink, or a copy between virtual ranks on one GPU)."""
+
+    def __init__(self, shape: Shape):
+        self.shape = shape
+
+    def send_qkv(self, q, k, v, stream=None):
+        torch = _torch()
+        out = []
+        for x in (q, k, v):
+            send = torch.empty(self.shape.send_chunks, dtype=x.dtype, device=x.device)
+            exchange_pack(x, send, self.shape, stream)
+            out.append(send)
+        return out
+
+    def attend(self, q, k, v, lse=None, stream=None):
+        torch = _torch()
+        o = torch.empty_like(q)
+        attention_seqsharded(q, k, v, o, self.shape.head_group(), lse=lse, stream=stream)
+        return o
+
+    def finish(self, back, stream=None):
+        torch = _torch()
+        out = torch.empty(self.shape.rank_shard, dtype=back.dtype, device=back.device)
+        exchange_unpack(back, out, self.shape, stream)
+        return out
+
+
+def nccl_all_to_all(group=None):
+    """Exchange through torch.distributed: chunk j of this rank's [P][...]
+    buffer goes to rank j; the result holds every rank's chunk in rank order."""
+    import torch.distributed as dist
+
+    def exchange(send):
+        torch = _torch()
+        recv = torch.empty_like(send)
+        dist.all_to_all_single(recv, send, group=group)
+        return recv
+    return exchange
+
+
+def ulysses_attention_distributed(q, k, v, shape: Shape, all_to_all=None):
+    """One rank's Ulysses attention step: q, k, v are this rank's shards
+    [B][Nl][H][D] (rank = position in the group of shape.P ranks); returns
+    the output shard.  all_to_all defaults to NCCL over the default group."""
+    all_to_all = all_to_all or nccl_all_to_all()
+    rank = UlyssesRank(shape)
+    rq, rk, rv = (all_to_all(x) for x in rank.send_qkv(q, k, v))
+    return rank.finish(all_to_all(rank.attend(rq, rk, rv)))
 
 
 def device_status(stream=None, device=None) -> int:

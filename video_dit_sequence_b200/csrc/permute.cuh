@@ -5,7 +5,11 @@
 // four GPUs") is a pure permutation of 16-bit words:
 //   pack   : xh[j][b][r*Nl + n][hh][:] = xs[r][b][n][j*Hl + hh][:]
 //   unpack : os[r][b][n][j*Hl + hh][:] = oh[j][b][r*Nl + n][hh][:]
-// Both move contiguous runs of Hl*D words (>= 128 bytes), so every thread
+// With one GPU per rank the same exchange is, on each rank, a reorder into P
+// send chunks before the all-to-all and the reverse after the return one:
+//   exchange pack   : send[j][b][n][hh][:]  = xs_r[b][n][j*Hl + hh][:]
+//   exchange unpack : os_r[b][n][j*Hl + hh][:] = recv[j][b][n][hh][:]
+// All four move contiguous runs of Hl*D words (>= 128 bytes), so every thread
 // copies 16-byte vectors and consecutive threads touch consecutive vectors of
 // one run on both sides.  The destination is walked linearly (vector v of
 // the kernel writes bytes 16v .. 16v+15 of the output); the source address
@@ -47,6 +51,7 @@ struct PermuteParams {
   FastDiv p;               // P
   FastDiv bdiv;            // B
   FastDiv pvr;             // P * vectors per run (unpack: vectors per output row)
+  FastDiv bnl;             // B * Nl (exchange modes)
   uint32_t H_vec;          // vectors per sequence-sharded token row: H*D/8
   uint32_t Hl_vec;         // vectors per head-sharded token row: Hl*D/8
   uint32_t Nl, Np, B, P;
@@ -99,7 +104,37 @@ __device__ __forceinline__ uint64_t unpack_src(uint32_t v, const PermuteParams &
   return (static_cast<uint64_t>(j * p.B + b) * p.Np + r * p.Nl + n) * p.Hl_vec + k;
 }
 
-template <bool kPack>
+// Exchange pack, output vector v: send row R = v / Vr = j*(B*Nl) + bn,
+// vector k = v % Vr; the source row is bn of the rank's shard.
+__device__ __forceinline__ uint64_t exchange_pack_src(uint32_t v, const PermuteParams &p) {
+  uint32_t R = fdiv(v, p.vr);
+  uint32_t k = v - R * p.vr.d;
+  uint32_t j = fdiv(R, p.bnl);
+  uint32_t bn = R - j * p.bnl.d;
+  return static_cast<uint64_t>(bn) * p.H_vec + static_cast<uint64_t>(j) * p.Hl_vec + k;
+}
+
+// Exchange unpack, output vector v: shard row bn = v / (P*Vr); within it
+// run j = w / Vr and vector k = w % Vr, w = v % (P*Vr).
+__device__ __forceinline__ uint64_t exchange_unpack_src(uint32_t v, const PermuteParams &p) {
+  uint32_t bn = fdiv(v, p.pvr);
+  uint32_t w = v - bn * p.pvr.d;
+  uint32_t j = fdiv(w, p.vr);
+  uint32_t k = w - j * p.vr.d;
+  return (static_cast<uint64_t>(j) * p.bnl.d + bn) * p.Hl_vec + k;
+}
+
+enum PermuteMode { kModePack = 0, kModeUnpack = 1, kModeExchangePack = 2, kModeExchangeUnpack = 3 };
+
+template <int kMode>
+__device__ __forceinline__ uint64_t permute_src(uint32_t v, const PermuteParams &p) {
+  if (kMode == kModePack) return pack_src(v, p);
+  if (kMode == kModeUnpack) return unpack_src(v, p);
+  if (kMode == kModeExchangePack) return exchange_pack_src(v, p);
+  return exchange_unpack_src(v, p);
+}
+
+template <int kMode>
 __global__ void __launch_bounds__(kPermThreads)
 permute_kernel(const PermuteParams p) {
   const uint32_t base = blockIdx.x * (kPermThreads * kPermUnroll) + threadIdx.x;
@@ -107,7 +142,7 @@ permute_kernel(const PermuteParams p) {
 #pragma unroll
   for (int u = 0; u < kPermUnroll; ++u) {
     uint32_t o = base + u * kPermThreads;
-    if (o < p.total_vec) v[u] = ld_stream(p.src + (kPack ? pack_src(o, p) : unpack_src(o, p)));
+    if (o < p.total_vec) v[u] = ld_stream(p.src + permute_src<kMode>(o, p));
   }
 #pragma unroll
   for (int u = 0; u < kPermUnroll; ++u) {

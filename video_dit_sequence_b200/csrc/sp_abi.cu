@@ -41,10 +41,11 @@ EncodeTiledFn encode_fn() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-sp_status check_common(const sp_shape *s) {
+// heads_split: the call splits heads into P groups, so P must divide H.
+sp_status check_common(const sp_shape *s, bool heads_split = true) {
   if (s == nullptr) return SP_ERR_NULL;
   if (s->B < 1 || s->N < 1 || s->H < 1 || s->P < 1 || s->D < 1) return SP_ERR_SHAPE;
-  if (s->H % s->P != 0) return SP_ERR_HEADS_NOT_DIVISIBLE;
+  if (heads_split && s->H % s->P != 0) return SP_ERR_HEADS_NOT_DIVISIBLE;
   if (s->D != 64 && s->D != 128) return SP_ERR_UNSUPPORTED_D;
   if (s->P > 65535 || s->B > 65535 || s->H > 65535) return SP_ERR_SHAPE;
   const int64_t Nl = (static_cast<int64_t>(s->N) + s->P - 1) / s->P;
@@ -77,7 +78,7 @@ int32_t *status_ptr() {
   return ptrs[dev];
 }
 
-sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, bool pack) {
+sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, int mode) {
   sp_status st = check_common(s);
   if (st != SP_OK) return st;
   if (src == nullptr || dst == nullptr) return SP_ERR_NULL;
@@ -88,12 +89,15 @@ sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, b
   sp::PermuteParams p;
   p.src = static_cast<const uint4 *>(src);
   p.dst = static_cast<uint4 *>(dst);
-  p.total_vec = static_cast<uint32_t>(static_cast<uint64_t>(P) * B * Nl * H * D / 8);
+  const bool exchange = mode == sp::kModeExchangePack || mode == sp::kModeExchangeUnpack;
+  // one rank's shard (exchange modes) or all P shards
+  p.total_vec = static_cast<uint32_t>(static_cast<uint64_t>(exchange ? 1 : P) * B * Nl * H * D / 8);
   p.vr = sp::make_fastdiv(Hl * D / 8);
   p.nl = sp::make_fastdiv(Nl);
   p.p = sp::make_fastdiv(P);
   p.bdiv = sp::make_fastdiv(B);
   p.pvr = sp::make_fastdiv(P * Hl * D / 8);
+  p.bnl = sp::make_fastdiv(B * Nl);
   p.H_vec = H * D / 8;
   p.Hl_vec = Hl * D / 8;
   p.Nl = Nl;
@@ -103,10 +107,16 @@ sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, b
   const uint32_t per_block = sp::kPermThreads * sp::kPermUnroll;
   const uint32_t blocks = (p.total_vec + per_block - 1) / per_block;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (pack)
-    sp::permute_kernel<true><<<blocks, sp::kPermThreads, 0, cs>>>(p);
-  else
-    sp::permute_kernel<false><<<blocks, sp::kPermThreads, 0, cs>>>(p);
+  switch (mode) {
+    case sp::kModePack: sp::permute_kernel<sp::kModePack><<<blocks, sp::kPermThreads, 0, cs>>>(p); break;
+    case sp::kModeUnpack: sp::permute_kernel<sp::kModeUnpack><<<blocks, sp::kPermThreads, 0, cs>>>(p); break;
+    case sp::kModeExchangePack:
+      sp::permute_kernel<sp::kModeExchangePack><<<blocks, sp::kPermThreads, 0, cs>>>(p);
+      break;
+    default:
+      sp::permute_kernel<sp::kModeExchangeUnpack><<<blocks, sp::kPermThreads, 0, cs>>>(p);
+      break;
+  }
   return launch_status(cudaGetLastError());
 }
 
@@ -178,7 +188,9 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
 // h % hsplit).
 sp_status attention(const void *q, const void *k, const void *v, void *o, float *lse,
                     const sp_shape *s, void *stream, bool seqsharded) {
-  sp_status st = check_common(s);
+  // The fused call shards tokens only; heads are never split, so it takes
+  // any P (the per-rank call of the multi-GPU form has Hl heads and P shards).
+  sp_status st = check_common(s, !seqsharded);
   if (st != SP_OK) return st;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SP_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
@@ -277,11 +289,19 @@ int64_t sp_padded_tokens(int32_t N, int32_t P) {
 sp_status sp_check_shape(const sp_shape *shape) { return check_common(shape); }
 
 sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream) {
-  return permute(xs, xh, shape, stream, true);
+  return permute(xs, xh, shape, stream, sp::kModePack);
 }
 
 sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *stream) {
-  return permute(oh, os, shape, stream, false);
+  return permute(oh, os, shape, stream, sp::kModeUnpack);
+}
+
+sp_status sp_exchange_pack(const void *xs_r, void *send, const sp_shape *shape, void *stream) {
+  return permute(xs_r, send, shape, stream, sp::kModeExchangePack);
+}
+
+sp_status sp_exchange_unpack(const void *recv, void *os_r, const sp_shape *shape, void *stream) {
+  return permute(recv, os_r, shape, stream, sp::kModeExchangeUnpack);
 }
 
 sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh, float *lse,
