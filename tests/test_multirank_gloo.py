@@ -140,3 +140,51 @@ def test_multi_gpu_exchange_routing_over_gloo(world, shape_args):
         assert p.exitcode == 0
     got = dict(q.get(timeout=5) for _ in range(world))
     assert all(got[r] for r in range(world)), got
+
+
+def _dead_peer_main(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import datetime
+    import time
+
+    import torch
+    import torch.distributed as dist
+
+    import video_dit_sequence_b200 as sp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        # this rank fails between steps: it leaves before the exchange
+        q.put((rank, "left"))
+        q.close()
+        q.join_thread()
+        os._exit(0)
+    send = torch.zeros((world, 4), dtype=torch.bfloat16)
+    t0 = time.monotonic()
+    try:
+        sp.nccl_all_to_all()(send)
+        q.put((rank, "no error"))
+    except Exception as e:  # the group's timeout ends the exchange with an error
+        q.put((rank, f"error after {time.monotonic() - t0:.1f}s: {type(e).__name__}"))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+@pytest.mark.timeout(120)
+def test_exchange_with_a_dead_peer_errors_instead_of_hanging():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dead_peer_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(90)
+        assert p.exitcode is not None, "a rank hung"
+    got = dict(q.get(timeout=5) for _ in range(world))
+    assert got[1] == "left"
+    assert got[0].startswith("error after"), got[0]
+    assert float(got[0].split()[2].rstrip("s:")) < 60
