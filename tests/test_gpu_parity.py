@@ -271,6 +271,42 @@ def test_degrees_bit_identical(N):
     _check_rows(ref, q, k, v, rr, 1, f"N={N}")
 
 
+def test_host_pipeline_matches_direct_calls():
+    """Three problems through HostPipeline (transfers overlapped with compute
+    on three streams, two device buffer sets) give the direct results."""
+    B, N, H, D, P = 1, 1500, 4, 128, 2
+    shape = sp.Shape(B, N, H, D, P)
+    pipe = sp.HostPipeline(shape, depth=2)
+    outs, wants = [], []
+    for i in range(3):
+        q, k, v = _random_logical(B, N, H, D, seed=500 + i)
+        host = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, P)).view(np.int16))
+                .view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+        ho = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16).pin_memory()
+        pipe.submit(*host, ho)
+        outs.append(ho)
+        wants.append(_run_fused(q, k, v, P)[0])
+    pipe.synchronize()
+    _status_ok()
+    for got, want in zip(outs, wants):
+        assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
+
+
+@pytest.mark.parametrize("scale", [0.05, 0.2])
+def test_explicit_scale(scale):
+    B, N, H, D, P = 1, 900, 2, 64, 2
+    q, k, v = _random_logical(B, N, H, D, seed=int(scale * 100))
+    shape = sp.Shape(B, N, H, D, P, scale)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    os_ = torch.empty_like(qs)
+    sp.attention_seqsharded(qs, ks, vs, os_, shape)
+    _status_ok()
+    O = synth.from_seq_shards(to_host(os_).reshape(shape.seq_sharded), N)
+    rows = _rows_all(B, N, H)
+    ref, _ = oracle.attention_rows(q, k, v, rows, scale=scale)
+    assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]), f"scale={scale}")
+
+
 def test_closed_forms_on_gpu():
     B, N, H, D, P = 1, 700, 4, 128, 2
     q, k, v = _random_logical(B, N, H, D, seed=5)

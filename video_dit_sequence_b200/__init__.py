@@ -316,6 +316,62 @@ def ulysses_attention_distributed(q, k, v, shape: Shape, all_to_all=None):
     return rank.finish(all_to_all(rank.attend(rq, rk, rv)))
 
 
+class HostPipeline:
+    """Fused attention on host-resident problems, with the transfers hidden
+    behind the compute.
+
+    submit(hq, hk, hv, ho) takes pinned host tensors in the sequence-sharded
+    layout ([P][B][Nl][H][D] bf16) and enqueues, on three streams: the copy of
+    the inputs into one of `depth` device buffer sets, the fused attention on
+    that set, and the copy of the output back into `ho`.  A buffer set is
+    reused only after the output it held has left the device, so step i+1's
+    inputs travel while step i computes and step i's output travels while
+    step i+1 computes.  Nothing here synchronises the host; synchronize()
+    waits for everything submitted."""
+
+    def __init__(self, shape: Shape, device=None, depth: int = 2):
+        torch = _torch()
+        self.shape = shape
+        self.device = torch.device(device or "cuda")
+        self.h2d = torch.cuda.Stream(self.device)
+        self.compute = torch.cuda.Stream(self.device)
+        self.d2h = torch.cuda.Stream(self.device)
+        ss = shape.seq_sharded
+        self.sets = [tuple(torch.empty(ss, dtype=torch.bfloat16, device=self.device)
+                           for _ in range(4)) for _ in range(depth)]
+        self.freed = [None] * depth     # event: the set's last output has left
+        self.count = 0
+
+    def submit(self, hq, hk, hv, ho):
+        torch = _torch()
+        i = self.count % len(self.sets)
+        self.count += 1
+        dq, dk, dv, do = self.sets[i]
+        if self.freed[i] is not None:
+            self.h2d.wait_event(self.freed[i])
+        with torch.cuda.stream(self.h2d):
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+        arrived = torch.cuda.Event()
+        arrived.record(self.h2d)
+        self.compute.wait_event(arrived)
+        attention_seqsharded(dq, dk, dv, do, self.shape, stream=self.compute)
+        done = torch.cuda.Event()
+        done.record(self.compute)
+        self.d2h.wait_event(done)
+        with torch.cuda.stream(self.d2h):
+            ho.copy_(do, non_blocking=True)
+        freed = torch.cuda.Event()
+        freed.record(self.d2h)
+        self.freed[i] = freed
+        return freed
+
+    def synchronize(self):
+        for st in (self.h2d, self.compute, self.d2h):
+            st.synchronize()
+
+
 def device_status(stream=None, device=None) -> int:
     """Synchronises the stream and returns (and clears) the device status."""
     return int(load().sp_device_status(_stream(stream, device)))
