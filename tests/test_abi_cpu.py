@@ -113,3 +113,12 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(shape.seq_sharded, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         sp.pack(x, x, shape)
+
+
+def test_binding_refuses_mixed_devices(lib):
+    torch = pytest.importorskip("torch")
+    shape = sp.Shape(1, 16, 2, 64, 2)
+    a = torch.zeros(shape.seq_sharded, dtype=torch.bfloat16)
+    b = torch.zeros(shape.head_sharded, dtype=torch.bfloat16, device="meta")
+    with pytest.raises((ValueError, TypeError)):
+        sp.pack(a, b, shape)

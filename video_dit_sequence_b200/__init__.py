@@ -190,7 +190,30 @@ def _stream(stream, device):
     torch = _torch()
     if stream is None:
         stream = torch.cuda.current_stream(device)
+    elif stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _resolve_device(stream, device):
+    torch = _torch()
+    if stream is not None:
+        return stream.device
+    d = torch.device(device) if device is not None else torch.device("cuda")
+    return d if d.index is not None else torch.device("cuda", torch.cuda.current_device())
+
+
+def _same_device(*tensors):
+    """All operands must live on one CUDA device; the call runs with that
+    device current (the library resolves its per-device state from it)."""
+    torch = _torch()
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"operands on several devices: {sorted(map(str, devs))}")
+    dev = devs.pop()
+    if dev.type != "cuda":
+        raise TypeError("operands must be CUDA tensors")
+    return torch.cuda.device(dev)
 
 
 def _check(status: int, where: str):
@@ -201,15 +224,17 @@ def _check(status: int, where: str):
 def pack(xs, xh, shape: Shape, stream=None):
     """Sequence-sharded -> head-sharded (bit-exact permutation)."""
     s = shape.c()
-    _check(load().sp_pack(_ptr(xs, shape.seq_sharded, "xs"), _ptr(xh, shape.head_sharded, "xh"),
-                          ctypes.byref(s), _stream(stream, xs.device)), "sp_pack")
+    with _same_device(xs, xh):
+        _check(load().sp_pack(_ptr(xs, shape.seq_sharded, "xs"), _ptr(xh, shape.head_sharded, "xh"),
+                              ctypes.byref(s), _stream(stream, xs.device)), "sp_pack")
 
 
 def unpack(oh, os_, shape: Shape, stream=None):
     """Head-sharded -> sequence-sharded (bit-exact permutation)."""
     s = shape.c()
-    _check(load().sp_unpack(_ptr(oh, shape.head_sharded, "oh"), _ptr(os_, shape.seq_sharded, "os"),
-                            ctypes.byref(s), _stream(stream, oh.device)), "sp_unpack")
+    with _same_device(oh, os_):
+        _check(load().sp_unpack(_ptr(oh, shape.head_sharded, "oh"), _ptr(os_, shape.seq_sharded, "os"),
+                                ctypes.byref(s), _stream(stream, oh.device)), "sp_unpack")
 
 
 def attention(qh, kh, vh, oh, shape: Shape, lse=None, stream=None):
@@ -217,10 +242,11 @@ def attention(qh, kh, vh, oh, shape: Shape, lse=None, stream=None):
     torch = _torch()
     s = shape.c()
     hs = shape.head_sharded
-    _check(load().sp_attention(
-        _ptr(qh, hs, "qh"), _ptr(kh, hs, "kh"), _ptr(vh, hs, "vh"), _ptr(oh, hs, "oh"),
-        _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
-        _stream(stream, qh.device)), "sp_attention")
+    with _same_device(qh, kh, vh, oh, lse):
+        _check(load().sp_attention(
+            _ptr(qh, hs, "qh"), _ptr(kh, hs, "kh"), _ptr(vh, hs, "vh"), _ptr(oh, hs, "oh"),
+            _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
+            _stream(stream, qh.device)), "sp_attention")
 
 
 def attention_seqsharded(qs, ks, vs, os_, shape: Shape, lse=None, stream=None):
@@ -228,26 +254,29 @@ def attention_seqsharded(qs, ks, vs, os_, shape: Shape, lse=None, stream=None):
     torch = _torch()
     s = shape.c()
     ss = shape.seq_sharded
-    _check(load().sp_attention_seqsharded(
-        _ptr(qs, ss, "qs"), _ptr(ks, ss, "ks"), _ptr(vs, ss, "vs"), _ptr(os_, ss, "os"),
-        _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
-        _stream(stream, qs.device)), "sp_attention_seqsharded")
+    with _same_device(qs, ks, vs, os_, lse):
+        _check(load().sp_attention_seqsharded(
+            _ptr(qs, ss, "qs"), _ptr(ks, ss, "ks"), _ptr(vs, ss, "vs"), _ptr(os_, ss, "os"),
+            _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
+            _stream(stream, qs.device)), "sp_attention_seqsharded")
 
 
 def exchange_pack(xs_r, send, shape: Shape, stream=None):
     """One rank's shard [B][Nl][H][D] -> its P send chunks [P][B][Nl][Hl][D]."""
     s = shape.c()
-    _check(load().sp_exchange_pack(_ptr(xs_r, shape.rank_shard, "xs_r"),
-                                   _ptr(send, shape.send_chunks, "send"), ctypes.byref(s),
-                                   _stream(stream, xs_r.device)), "sp_exchange_pack")
+    with _same_device(xs_r, send):
+        _check(load().sp_exchange_pack(_ptr(xs_r, shape.rank_shard, "xs_r"),
+                                       _ptr(send, shape.send_chunks, "send"), ctypes.byref(s),
+                                       _stream(stream, xs_r.device)), "sp_exchange_pack")
 
 
 def exchange_unpack(recv, os_r, shape: Shape, stream=None):
     """The P chunks returned to one rank [P][B][Nl][Hl][D] -> its shard."""
     s = shape.c()
-    _check(load().sp_exchange_unpack(_ptr(recv, shape.send_chunks, "recv"),
-                                     _ptr(os_r, shape.rank_shard, "os_r"), ctypes.byref(s),
-                                     _stream(stream, recv.device)), "sp_exchange_unpack")
+    with _same_device(recv, os_r):
+        _check(load().sp_exchange_unpack(_ptr(recv, shape.send_chunks, "recv"),
+                                         _ptr(os_r, shape.rank_shard, "os_r"), ctypes.byref(s),
+                                         _stream(stream, recv.device)), "sp_exchange_unpack")
 
 
 class UlyssesRank:
@@ -373,14 +402,21 @@ class HostPipeline:
 
 
 def device_status(stream=None, device=None) -> int:
-    """Synchronises the stream and returns (and clears) the device status."""
-    return int(load().sp_device_status(_stream(stream, device)))
+    """Synchronises the stream and returns (and clears) the status word of
+    the stream's device."""
+    torch = _torch()
+    dev = _resolve_device(stream, device)
+    with torch.cuda.device(dev):
+        return int(load().sp_device_status(_stream(stream, dev)))
 
 
 def selftest_wait_timeout(limit_ns: int, stream=None, device=None):
     """Enqueues a kernel whose bounded wait must run out (see sp.h)."""
-    _check(load().sp_selftest_wait_timeout(int(limit_ns), _stream(stream, device)),
-           "sp_selftest_wait_timeout")
+    torch = _torch()
+    dev = _resolve_device(stream, device)
+    with torch.cuda.device(dev):
+        _check(load().sp_selftest_wait_timeout(int(limit_ns), _stream(stream, dev)),
+               "sp_selftest_wait_timeout")
 
 
 def ulysses_attention(q, k, v, P: int, scale: float = 0.0, fused: bool = True):
