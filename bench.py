@@ -432,6 +432,16 @@ def run_ours(args):
     sp.pack(vs, vh, shape, stream=stream)
     t_attn = timed(lambda: sp.attention(qh, kh, vh, oh, shape, stream=stream))
     t_unpack = timed(lambda: sp.unpack(oh, os2, shape, stream=stream))
+    # FP8 variant of the fused step: the same problem with E4M3 Q/K/V
+    t_fp8 = None
+    if not args.no_fp8:
+        q8, k8, v8, d8 = synth.fp8_qkv(cfg)
+        dev8 = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, s.P))).to(dev)
+                for x in (q8, k8, v8)]
+        desc8 = torch.from_numpy(d8).to(dev)
+        o8 = torch.empty_like(os_)
+        t_fp8 = timed(lambda: sp.attention_fp8_seqsharded(*dev8, desc8, o8, shape, stream=stream))
+        del dev8, o8
     if sp.device_status(stream) != sp.SP_OK:
         raise SystemExit("device status not ok after the unfused rows")
     pack_gbs = 2 * tensor_bytes / (t_pack * 1e-3) / 1e9
@@ -442,6 +452,9 @@ def run_ours(args):
         "unpack": {"ms": t_unpack, "GB/s": unpack_gbs, "frac_hbm": unpack_gbs / pk["hbm_gbs"],
                    "bytes": 2 * tensor_bytes, "per": "O, read + write"},
         "attention_head_sharded": {"ms": t_attn, "TFLOP/s": flops / (t_attn * 1e-3) / 1e12},
+        "fused_fp8": None if t_fp8 is None else {
+            "ms": t_fp8, "TFLOP/s": flops / (t_fp8 * 1e-3) / 1e12,
+            "inputs": "E4M3 Q/K/V, per-(batch, head) scales; bf16 output"},
         "unfused_step_ms": 3 * t_pack + t_attn + t_unpack,
         "fused_step_ms": per_launch_ms,
     }
@@ -521,6 +534,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 row")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override N (same heads, head dim and degree); for profiling captures")
     ap.add_argument("--traffic-bytes", type=float, default=None,

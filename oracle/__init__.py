@@ -14,6 +14,8 @@ What it computes, and the passages it follows:
   "Generate video with WAN 2.2 across four GPUs", section "Splitting one
   generation across four GPUs" (each GPU sees the full sequence for its share
   of the heads, then the shards return).  Index formulas in ``sp_oracle.c``.
+* ``attention_rows_e4m3`` -- the same attention on 8-bit (E4M3) inputs with
+  per-(batch, head) scale factors, for the FP8 variant of the kernel.
 * ``attention_rows`` -- the unsharded softmax(q K^T scale) V of one head,
   two-pass exact softmax in fp64; the sequence-parallel result must equal it
   for every degree (LTX-2 "Multi-GPU Inference" README, Capabilities table:
@@ -61,6 +63,12 @@ def _bind(path: str):
         vp, vp, vp, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp,
         ctypes.c_int]
     lib.sp_oracle_attention_rows.restype = ctypes.c_int
+    lib.sp_oracle_attention_rows_e4m3.argtypes = [
+        vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp,
+        ctypes.c_int]
+    lib.sp_oracle_attention_rows_e4m3.restype = ctypes.c_int
+    lib.sp_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.sp_oracle_e4m3_value.restype = ctypes.c_double
     return lib
 
 
@@ -167,6 +175,37 @@ def attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     rc = (lib or _load()).sp_oracle_attention_rows(
         q.ctypes.data, k.ctypes.data, v.ctypes.data, B, N, H, D, float(scale),
         R, rows.ctypes.data, o.ctypes.data, lse.ctypes.data, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle attention failed ({rc})")
+    return o, lse
+
+
+def e4m3_value(byte: int, lib=None) -> float:
+    """Exact value of one OCP E4M3 byte."""
+    return float((lib or _load()).sp_oracle_e4m3_value(int(byte)))
+
+
+def attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows, scale: float = 0.0,
+                        threads: Optional[int] = None, lib=None):
+    """fp64 attention of e4m3 inputs: element values are the exact e4m3 values
+    (uint8 arrays, logical [B][N][H][D]) times per-(b, h) factors dq, dk, dv
+    ([B][H] float64).  Returns (O [R][D], LSE [R])."""
+    for a in (q8, k8, v8):
+        assert a.dtype == np.uint8 and a.shape == q8.shape and a.ndim == 4
+    B, N, H, D = q8.shape
+    q8, k8, v8 = (np.ascontiguousarray(a) for a in (q8, k8, v8))
+    dq, dk, dv = (np.ascontiguousarray(np.broadcast_to(np.asarray(d, dtype=np.float64), (B, H)))
+                  for d in (dq, dk, dv))
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    R = rows.shape[0]
+    o = np.empty((R, D), dtype=np.float64)
+    lse = np.empty(R, dtype=np.float64)
+    if threads is None:
+        threads = max(1, len(os.sched_getaffinity(0)))
+    rc = (lib or _load()).sp_oracle_attention_rows_e4m3(
+        q8.ctypes.data, k8.ctypes.data, v8.ctypes.data, dq.ctypes.data, dk.ctypes.data,
+        dv.ctypes.data, B, N, H, D, float(scale), R, rows.ctypes.data, o.ctypes.data,
+        lse.ctypes.data, int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle attention failed ({rc})")
     return o, lse

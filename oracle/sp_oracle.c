@@ -45,6 +45,20 @@ static double bf16_to_f64(uint16_t x) {
     return (double)f;
 }
 
+/* OCP 8-bit floating point E4M3 (sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; exponent 0 is subnormal, S.1111.111 is NaN, no infinity),
+ * decoded exactly. */
+static double e4m3_to_f64(uint8_t x) {
+    int s = x >> 7, e = (x >> 3) & 15, m = x & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+double sp_oracle_e4m3_value(uint8_t x) { return e4m3_to_f64(x); }
+
 /*
  * Pack (sequence-sharded -> head-sharded): the send-buffer reorder plus the
  * all-to-all of the page section "Splitting one generation across four GPUs".
@@ -155,6 +169,8 @@ int sp_oracle_exchange_unpack(const uint16_t *recv, uint16_t *os_r, int64_t B, i
  */
 typedef struct {
     const uint16_t *q, *k, *v;
+    const uint8_t *q8, *k8, *v8;       /* e4m3 inputs instead of bf16, or NULL */
+    const double *dq, *dk, *dv;        /* per-(b, h) scale factors of q8/k8/v8 */
     int64_t B, N, H, D;
     double scale;
     int64_t nrows;
@@ -165,15 +181,24 @@ typedef struct {
     int failed;
 } attn_job_t;
 
+/* Element e of a logical [B][N][H][D] input: bf16 words, or e4m3 bytes
+ * times the per-(b, h) scale. */
+static double elem(const uint16_t *x16, const uint8_t *x8, const double *scale, int64_t bh,
+                   int64_t e) {
+    if (x8) return e4m3_to_f64(x8[e]) * scale[bh];
+    return bf16_to_f64(x16[e]);
+}
+
 static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
     int64_t b = J->rows[3 * r], h = J->rows[3 * r + 1], i = J->rows[3 * r + 2];
-    int64_t N = J->N, H = J->H, D = J->D;
-    const uint16_t *qi = J->q + ((b * N + i) * H + h) * D;
+    int64_t N = J->N, H = J->H, D = J->D, bh = b * H + h;
+    int64_t qi = ((b * N + i) * H + h) * D;
     double m = -INFINITY;
     for (int64_t kk = 0; kk < N; ++kk) {
-        const uint16_t *kr = J->k + ((b * N + kk) * H + h) * D;
+        int64_t kr = ((b * N + kk) * H + h) * D;
         double dot = 0.0;
-        for (int64_t c = 0; c < D; ++c) dot += bf16_to_f64(qi[c]) * bf16_to_f64(kr[c]);
+        for (int64_t c = 0; c < D; ++c)
+            dot += elem(J->q, J->q8, J->dq, bh, qi + c) * elem(J->k, J->k8, J->dk, bh, kr + c);
         s[kk] = J->scale * dot;
         if (s[kk] > m) m = s[kk];
     }
@@ -183,8 +208,8 @@ static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
     for (int64_t kk = 0; kk < N; ++kk) {
         double w = exp(s[kk] - m);
         l += w;
-        const uint16_t *vr = J->v + ((b * N + kk) * H + h) * D;
-        for (int64_t c = 0; c < D; ++c) o[c] += w * bf16_to_f64(vr[c]);
+        int64_t vr = ((b * N + kk) * H + h) * D;
+        for (int64_t c = 0; c < D; ++c) o[c] += w * elem(J->v, J->v8, J->dv, bh, vr + c);
     }
     for (int64_t c = 0; c < D; ++c) o[c] /= l;
     if (J->out_lse) J->out_lse[r] = m + log(l);
@@ -213,10 +238,45 @@ static void *attention_worker(void *arg) {
 /* Returns 0 on success, -1 on bad arguments, -2 when out of host memory.
  * Rows are handed to up to nthreads threads in list order; callers that sort
  * the list by (b, h) let the threads share each head's K/V in cache. */
+static int attention_rows_impl(attn_job_t *J, int nthreads);
+
 int sp_oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                              int64_t B, int64_t N, int64_t H, int64_t D, double scale,
                              int64_t nrows, const int64_t *rows, double *out_o,
                              double *out_lse, int nthreads) {
+    attn_job_t J;
+    memset(&J, 0, sizeof(J));
+    J.q = q; J.k = k; J.v = v;
+    J.B = B; J.N = N; J.H = H; J.D = D;
+    J.scale = scale;
+    J.nrows = nrows; J.rows = rows;
+    J.out_o = out_o; J.out_lse = out_lse;
+    return attention_rows_impl(&J, nthreads);
+}
+
+/* The same attention on e4m3 inputs: element values are the exact e4m3
+ * values times per-(b, h) scale factors dq/dk/dv ([B][H] each). */
+int sp_oracle_attention_rows_e4m3(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
+                                  const double *dq, const double *dk, const double *dv,
+                                  int64_t B, int64_t N, int64_t H, int64_t D, double scale,
+                                  int64_t nrows, const int64_t *rows, double *out_o,
+                                  double *out_lse, int nthreads) {
+    attn_job_t J;
+    memset(&J, 0, sizeof(J));
+    J.q8 = q8; J.k8 = k8; J.v8 = v8;
+    J.dq = dq; J.dk = dk; J.dv = dv;
+    J.B = B; J.N = N; J.H = H; J.D = D;
+    J.scale = scale;
+    J.nrows = nrows; J.rows = rows;
+    J.out_o = out_o; J.out_lse = out_lse;
+    return attention_rows_impl(&J, nthreads);
+}
+
+static int attention_rows_impl(attn_job_t *JP, int nthreads) {
+    attn_job_t J = *JP;
+    int64_t B = J.B, N = J.N, H = J.H, D = J.D, nrows = J.nrows;
+    const int64_t *rows = J.rows;
+    double scale = J.scale;
     if (B < 1 || N < 1 || H < 1 || D < 1 || nrows < 0) return -1;
     for (int64_t r = 0; r < nrows; ++r) {
         if (rows[3 * r] < 0 || rows[3 * r] >= B || rows[3 * r + 1] < 0 ||
@@ -224,12 +284,7 @@ int sp_oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_
             return -1;
     }
     if (!(scale > 0.0)) scale = 1.0 / sqrt((double)D);
-    attn_job_t J;
-    J.q = q; J.k = k; J.v = v;
-    J.B = B; J.N = N; J.H = H; J.D = D;
     J.scale = scale;
-    J.nrows = nrows; J.rows = rows;
-    J.out_o = out_o; J.out_lse = out_lse;
     J.next = 0;
     J.failed = 0;
     pthread_mutex_init(&J.lock, NULL);

@@ -244,3 +244,29 @@ def f32_to_bf16(f: np.ndarray) -> np.ndarray:
     u = np.ascontiguousarray(f, dtype=np.float32).view(np.uint32)
     u = u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
     return (u >> np.uint32(16)).astype(np.uint16)
+
+
+E4M3_MAX = 448.0
+
+
+def to_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even narrowing of fp32 values (|x| <= 448) to OCP
+    E4M3 bytes (torch's float8_e4m3fn conversion)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def fp8_qkv(cfg: Config, threads: Optional[int] = None):
+    """8-bit inputs for the FP8 variant: the config's bf16 Q, K, V, each
+    scaled per (batch, head) so its largest magnitude maps to 448, then
+    rounded to E4M3.  Returns (q8, k8, v8) as logical [B][N][H][D] uint8 and
+    the descale factors d [3][B][H] float32 (value = e4m3 value * d)."""
+    out, scales = [], []
+    for x in qkv_logical(cfg, threads):
+        f = bf16_to_f32(x)                                    # [B][N][H][D]
+        amax = np.abs(f).max(axis=(1, 3)).astype(np.float32)  # [B][H]
+        d = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        out.append(to_e4m3(f / d[:, None, :, None]))
+        scales.append(d)
+    return out[0], out[1], out[2], np.stack(scales)

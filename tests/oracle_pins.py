@@ -293,11 +293,54 @@ def check_rows_api(lib=None):
         assert np.array_equal(o[r], O[b, i, h]) and l[r] == L[b, h, i]
 
 
+def check_e4m3_decode_matches_torch(lib=None):
+    """All 256 E4M3 bytes decode as torch's float8_e4m3fn does."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_value(int(c), lib=lib) for c in codes])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+
+
+def _e4m3_from_float(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def check_fp8_attention_reduces_to_bf16(lib=None):
+    """Small integers are exact in both formats: with unit scales the e4m3
+    path equals the (pinned) bf16 path; scale factors act as their closed
+    forms (dv scales O, dq*dk scales the logits)."""
+    rng = np.random.default_rng(RNG_SEED + 16)
+    B, N, H, D = 2, 33, 2, 16
+    fq, fk, fv = (rng.integers(-3, 4, size=(B, N, H, D)).astype(np.float32) for _ in range(3))
+    q8, k8, v8 = (_e4m3_from_float(x) for x in (fq, fk, fv))
+    qb, kb, vb = (synth.f32_to_bf16(x) for x in (fq, fk, fv))
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(N)], np.int64)
+    scale = 0.125
+    o8, l8 = oracle.attention_rows_e4m3(q8, k8, v8, 1.0, 1.0, 1.0, rows, scale, 2, lib=lib)
+    ob, lb = oracle.attention_rows(qb, kb, vb, rows, scale, 2, lib=lib)
+    assert np.max(np.abs(o8 - ob)) < 1e-13 and np.max(np.abs(l8 - lb)) < 1e-13
+    dq = rng.uniform(0.5, 2.0, size=(B, H))
+    dk = rng.uniform(0.5, 2.0, size=(B, H))
+    dv = rng.uniform(0.5, 2.0, size=(B, H))
+    o8s, _ = oracle.attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows, scale, 2, lib=lib)
+    for r, (b, h, i) in enumerate(rows):
+        # logits scale by dq*dk: the same as the unit-scale problem at scale*dq*dk
+        want, _ = oracle.attention_rows_e4m3(q8, k8, v8, 1.0, 1.0, 1.0, rows[r:r + 1],
+                                             scale * dq[b, h] * dk[b, h], 1, lib=lib)
+        assert np.max(np.abs(o8s[r] - dv[b, h] * want[0])) < 1e-12
+
+
 PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
                check_unpack_returns_shards, check_pack_degree_one_is_copy,
                check_exchange_chunks_hold_head_groups,
                check_exchange_matches_numpy_and_single_gpu_pack]
 ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one,
                     check_closed_forms, check_dominant_key, check_invariances,
-                    check_two_token_example, check_rows_api]
+                    check_two_token_example, check_rows_api,
+                    check_e4m3_decode_matches_torch, check_fp8_attention_reduces_to_bf16]
 ALL_CHECKS = PACK_CHECKS + ATTENTION_CHECKS

@@ -307,6 +307,77 @@ def test_explicit_scale(scale):
     assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]), f"scale={scale}")
 
 
+# ------------------------------------------------------------------ FP8 variant
+
+# The FP8 kernel rounds every probability to E4M3 before the PV product:
+# relative rounding error at most 2^-4 per weight (3 mantissa bits), errors
+# of different keys independent with zero mean.  Its bars, against the fp64
+# attention of the same E4M3 inputs, scale with the output: relative L2 per
+# head <= 2^-4, and every element within 2^-3 of the largest output
+# magnitude (twice the per-weight bound, for the tail of the distribution).
+FP8_REL_L2 = 2.0 ** -4
+FP8_MAX_REL = 2.0 ** -3
+
+
+def _fp8_inputs(B, N, H, D, seed):
+    cfg = synth.Config("f8", synth.Shape(B, N, H, D, 1), seed=seed)
+    return synth.fp8_qkv(cfg)
+
+
+def _run_fp8(q8, k8, v8, d, P, lse=False):
+    B, N, H, D = q8.shape
+    shape = sp.Shape(B, N, H, D, P)
+
+    def dev8(x):
+        return torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, P))).cuda()
+
+    os_ = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    l = torch.full(shape.lse_shape, float("nan"), dtype=torch.float32, device="cuda") if lse else None
+    sp.attention_fp8_seqsharded(dev8(q8), dev8(k8), dev8(v8), torch.from_numpy(d).cuda(), os_,
+                                shape, lse=l)
+    _status_ok()
+    return to_host(os_), (l.cpu().numpy() if lse else None)
+
+
+def _check_fp8(out, q8, k8, v8, d, rows, P, where):
+    B, N, H, D = q8.shape
+    O = synth.from_seq_shards(out.reshape(P, B, -1, H, D), N)
+    ref, _ = oracle.attention_rows_e4m3(q8, k8, v8, d[0], d[1], d[2], rows)
+    m = compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1])
+    assert m["finite"], where
+    assert m["rel_l2"] <= FP8_REL_L2, (where, m)
+    assert m["max_abs"] <= FP8_MAX_REL * np.max(np.abs(ref)), (where, m)
+    return m
+
+
+@pytest.mark.parametrize("B,N,H,P", [(1, 1024, 4, 2), (1, 3000, 8, 4), (2, 1000, 8, 4),
+                                     (1, 257, 2, 1)])
+def test_fp8_attention_against_oracle(B, N, H, P):
+    q8, k8, v8, d = _fp8_inputs(B, N, H, 128, seed=40 + N)
+    out, lse = _run_fp8(q8, k8, v8, d, P, lse=True)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H)
+                     for i in sorted({0, N - 1, *range(0, N, max(1, N // 48))})], dtype=np.int64)
+    m = _check_fp8(out, q8, k8, v8, d, rows, P, f"fp8 B={B} N={N} P={P}")
+    print(f"fp8 B={B} N={N} P={P}: {m}")
+    one, lse1 = _run_fp8(q8, k8, v8, d, 1, lse=True)
+    assert np.array_equal(synth.from_seq_shards(out.reshape(P, B, -1, H, 128), N),
+                          synth.from_seq_shards(one.reshape(1, B, -1, H, 128), N))
+    _, lse_ref = oracle.attention_rows_e4m3(q8, k8, v8, d[0], d[1], d[2], rows)
+    got = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert np.max(np.abs(got - lse_ref)) < 2e-2
+
+
+def test_fp8_720p_sampled_rows():
+    cfg = synth.CONFIGS["720p"]
+    s = cfg.shape
+    q8, k8, v8, d = synth.fp8_qkv(cfg)
+    out, _ = _run_fp8(q8, k8, v8, d, s.P)
+    rows_t = synth.sampled_rows(cfg, 8)
+    rows = np.array([(0, h, i) for h in range(s.H) for i in rows_t], dtype=np.int64)
+    m = _check_fp8(out, q8, k8, v8, d, rows, s.P, "fp8 720p")
+    print(f"fp8 720p: {m}")
+
+
 def test_closed_forms_on_gpu():
     B, N, H, D, P = 1, 700, 4, 128, 2
     q, k, v = _random_logical(B, N, H, D, seed=5)

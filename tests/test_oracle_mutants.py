@@ -29,19 +29,24 @@ MUTANTS = [
     ("no-normalisation", "o[c] /= l;", "o[c] /= 1.0;"),
     ("exp-sign", "exp(s[kk] - m)", "exp(m - s[kk])"),
     ("sum-of-squares", "l += w;", "l += w * w;"),
-    ("v-uses-query-token", "J->v + ((b * N + kk) * H + h) * D",
-     "J->v + ((b * N + i) * H + h) * D"),
-    ("k-wrong-head", "J->k + ((b * N + kk) * H + h) * D",
-     "J->k + ((b * N + kk) * H + (H - 1 - h)) * D"),
-    ("q-head-zero", "J->q + ((b * N + i) * H + h) * D",
-     "J->q + ((b * N + i) * H + 0) * D"),
-    ("dot-drops-last-channel", "for (int64_t c = 0; c < D; ++c) dot +=",
-     "for (int64_t c = 0; c + 1 < D; ++c) dot +="),
+    ("v-uses-query-token", "int64_t vr = ((b * N + kk) * H + h) * D;",
+     "int64_t vr = ((b * N + i) * H + h) * D;"),
+    ("k-wrong-head", "int64_t kr = ((b * N + kk) * H + h) * D;",
+     "int64_t kr = ((b * N + kk) * H + (H - 1 - h)) * D;"),
+    ("q-head-zero", "int64_t qi = ((b * N + i) * H + h) * D;",
+     "int64_t qi = ((b * N + i) * H + 0) * D;"),
+    ("dot-drops-last-channel", "for (int64_t c = 0; c < D; ++c)\n            dot +=",
+     "for (int64_t c = 0; c + 1 < D; ++c)\n            dot +="),
     ("second-pass-drops-last-key",
      "for (int64_t kk = 0; kk < N; ++kk) {\n        double w",
      "for (int64_t kk = 0; kk + 1 < N; ++kk) {\n        double w"),
-    ("k-transposed-with-q", "dot += bf16_to_f64(qi[c]) * bf16_to_f64(kr[c]);",
-     "dot += bf16_to_f64(qi[c]) * bf16_to_f64(qi[c]);"),
+    ("k-transposed-with-q",
+     "elem(J->k, J->k8, J->dk, bh, kr + c);",
+     "elem(J->q, J->q8, J->dq, bh, qi + c);"),
+    ("e4m3-exponent-bias", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("e4m3-subnormal-scale", "if (e == 0) v = ldexp((double)m / 8.0, -6);",
+     "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
 ]
 
 

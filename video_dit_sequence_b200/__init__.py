@@ -41,7 +41,7 @@ SP_ERR_TIMEOUT = 7
 EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_attention", "sp_attention_seqsharded", "sp_device_status",
             "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout",
-            "sp_exchange_pack", "sp_exchange_unpack")
+            "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded")
 
 
 class sp_shape(ctypes.Structure):
@@ -80,6 +80,8 @@ def load(path: str = LIB_PATH):
         f = getattr(lib, name)
         f.argtypes = [vp, vp, vp, vp, vp, sp_p, vp]
         f.restype = ctypes.c_int
+    lib.sp_attention_fp8_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, sp_p, vp]
+    lib.sp_attention_fp8_seqsharded.restype = ctypes.c_int
     lib.sp_device_status.argtypes = [vp]
     lib.sp_device_status.restype = ctypes.c_int
     lib.sp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
@@ -259,6 +261,23 @@ def attention_seqsharded(qs, ks, vs, os_, shape: Shape, lse=None, stream=None):
             _ptr(qs, ss, "qs"), _ptr(ks, ss, "ks"), _ptr(vs, ss, "vs"), _ptr(os_, ss, "os"),
             _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
             _stream(stream, qs.device)), "sp_attention_seqsharded")
+
+
+def attention_fp8_seqsharded(qs8, ks8, vs8, descale, os_, shape: Shape, lse=None,
+                             stream=None):
+    """FP8 (E4M3) variant of attention_seqsharded: qs8/ks8/vs8 are uint8
+    [P][B][Nl][H][D] E4M3 bytes, descale float32 [3][B][H] (q, k, v factors),
+    os_ bf16 [P][B][Nl][H][D]."""
+    torch = _torch()
+    s = shape.c()
+    ss = shape.seq_sharded
+    with _same_device(qs8, ks8, vs8, descale, os_, lse):
+        _check(load().sp_attention_fp8_seqsharded(
+            _ptr(qs8, ss, "qs8", torch.uint8), _ptr(ks8, ss, "ks8", torch.uint8),
+            _ptr(vs8, ss, "vs8", torch.uint8),
+            _ptr(descale, (3, shape.B, shape.H), "descale", torch.float32),
+            _ptr(os_, ss, "os"), _ptr(lse, shape.lse_shape, "lse", torch.float32),
+            ctypes.byref(s), _stream(stream, qs8.device)), "sp_attention_fp8_seqsharded")
 
 
 def exchange_pack(xs_r, send, shape: Shape, stream=None):

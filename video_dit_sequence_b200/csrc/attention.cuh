@@ -55,21 +55,40 @@ struct AttnParams {
   // nl_split = Nl (else 0); token t lives in rank t / Nl at local row t % Nl.
   int32_t nl_split;
   int64_t o_rank;       // elements between rank slabs (B * Nl * H * D)
-  const __nv_bfloat16 *q, *k, *v;  // bases, for tiles that cross a shard boundary
+  const uint8_t *q, *k, *v;  // bases, for tiles that cross a shard boundary
+  // E4M3 variant: per-(batch, head) descale factors [3][B][H] (q, k, v);
+  // element value = byte value * factor.  Null for bf16.
+  const float *descale;
   float *lse;           // [B][H][Np] or null
   int32_t *status;      // device status word
 };
 
 constexpr int32_t kStatusTimeout = 7;
 
-template <int D>
+// kF8: operands in E4M3 (one byte) instead of bf16 (two bytes).
+template <int D, bool kF8 = false>
 struct AttnCfg {
   static_assert(D == 64 || D == 128, "head dim");
+  static_assert(!kF8 || D == 128, "the E4M3 variant has D = 128");
   static constexpr int kBM = 128;                   // query rows per tile
   static constexpr int kBN = 128;                   // keys per tile
-  static constexpr int kHalves = D / 64;            // 128-byte column blocks per row
-  static constexpr int kBlockBytes = 128 * 128;     // 128 rows x 64 bf16 (one swizzle block)
+  static constexpr int kElemBytes = kF8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElemBytes;  // one token row of one head
+  static constexpr int kHalves = kRowBytes / 128;   // 128-byte column blocks per row
+  static constexpr int kBoxInner = 128 / kElemBytes;  // elements per 128-byte block row
+  static constexpr int kBlockBytes = 128 * 128;     // 128 rows x 128 bytes (one swizzle block)
   static constexpr int kTileBytes = kHalves * kBlockBytes;
+  static constexpr int kQkSteps = kRowBytes / 32;   // MMA K steps of 32 bytes over D
+  static constexpr int kPvKeys = 32 / kElemBytes;   // keys per PV MMA (K = 16 or 32)
+  static constexpr int kPvSteps = kBN / kPvKeys;
+  static constexpr int kPCols = kBN * kElemBytes / 4;  // TMEM columns of one P row
+  // Probabilities are 2^(s*scale*log2e - m + kShift) and the reference m
+  // moves when a tile maximum exceeds it by more than kThresh, so they stay
+  // below 2^(kThresh + kShift): 2^8 for both.  E4M3 keeps 3 mantissa bits
+  // above 2^-6 only; the shift of 6 lifts the typical weights of a long
+  // sequence (about 2^-6 of the row maximum) out of its subnormal range.
+  static constexpr float kShift = kF8 ? 6.0f : 0.0f;
+  static constexpr float kThresh = kF8 ? 2.0f : 8.0f;
   static constexpr int kStages = 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
@@ -87,12 +106,12 @@ struct AttnCfg {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 
-template <int D>
+template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(320, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using C = AttnCfg<D>;
+  using C = AttnCfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -165,24 +184,25 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     auto tma_tile = [&](const CUtensorMap *m, uint32_t dst, uint32_t bar, int t0, uint64_t pol) {
       if (nl == 0) {
         for (int h = 0; h < C::kHalves; ++h)
-          tma_load_4d(dst + h * C::kBlockBytes, m, bar, h * 64, map_head, t0, map_batch, pol);
+          tma_load_4d(dst + h * C::kBlockBytes, m, bar, h * C::kBoxInner, map_head, t0, map_batch,
+                      pol);
       } else {
         const int r0 = t0 / nl;
         for (int h = 0; h < C::kHalves; ++h)
-          tma_load_5d(dst + h * C::kBlockBytes, m, bar, h * 64, map_head, t0 - r0 * nl, b, r0,
-                      pol);
+          tma_load_5d(dst + h * C::kBlockBytes, m, bar, h * C::kBoxInner, map_head, t0 - r0 * nl,
+                      b, r0, pol);
       }
     };
-    auto copy_tile = [&](const __nv_bfloat16 *base, uint32_t dst, int t0) {
-      constexpr int kChunks = D / 8;  // 16-byte chunks per token row
+    auto copy_tile = [&](const uint8_t *base, uint32_t dst, int t0) {
+      constexpr int kChunks = C::kRowBytes / 16;  // 16-byte chunks per token row
       for (int idx = lane; idx < C::kBM * kChunks; idx += 32) {
         const int r = idx / kChunks, cc = idx % kChunks;
         const int tok = t0 + r;
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
         if (tok < p.N) {
           const int rk = tok / nl, n = tok - rk * nl;
-          const int64_t off = ((static_cast<int64_t>(rk) * p.B + b) * nl + n) * p.H * D +
-                              static_cast<int64_t>(map_head) * D + cc * 8;
+          const int64_t off = ((static_cast<int64_t>(rk) * p.B + b) * nl + n) * p.H * C::kRowBytes +
+                              static_cast<int64_t>(map_head) * C::kRowBytes + cc * 16;
           val = ld_global_nc_v4(base + off);
         }
         st_shared_v4(dst + (cc >> 3) * C::kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4), val);
@@ -231,8 +251,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, 0, 1);
+      constexpr uint32_t idesc_qk = kF8 ? make_idesc_e4m3(128, 128, 0, 0)
+                                        : make_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = kF8 ? make_idesc_e4m3(128, D, 0, 1)
+                                        : make_idesc_bf16(128, D, 0, 1);
       // Shared-memory descriptors are built once; an operand's start address
       // lives in the low 14 bits (address >> 4), so moving to another tile,
       // slot or K step is one integer add (all addresses stay below 256 KB).
@@ -247,9 +269,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint64_t b0 = dK + static_cast<uint32_t>((slot * C::kTileBytes) >> 4);
         const uint32_t d = tmem + (t ? C::kColS1 : 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::kQkSteps; ++kk) {
           const uint32_t off = ((kk >> 2) * C::kBlockBytes + (kk & 3) * 32) >> 4;
-          umma_ss(d, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss<kF8>(d, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t[:, 64h .. 64h+63] V_j[64h .. 64h+63, :] for key half h.
@@ -258,10 +280,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t a0 = tmem + (t ? C::kColS1 : 0u);
         const uint32_t d = tmem + (t ? C::kColO1 : C::kColO0);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int kk = 4 * h + k;
-          umma_ts(d, a0 + kk * 8, b0 + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc_pv,
-                  (first && kk == 0) ? 0u : 1u);
+        for (int k = 0; k < C::kPvSteps / 2; ++k) {
+          const int kk = (C::kPvSteps / 2) * h + k;
+          umma_ts<kF8>(d, a0 + kk * 8, b0 + static_cast<uint32_t>((kk * C::kPvKeys * 128) >> 4),
+                       idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
       };
       // Waits for each half of P_t, then issues that half's PV MMAs.
@@ -325,7 +347,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_bits + (t ? C::kColS1 : 0u);
     const uint32_t tO = tmem + lane_bits + (t ? C::kColO1 : C::kColO0);
-    const float sl2 = p.scale_log2e;
+    // E4M3: the logits carry the q and k descale factors of this (b, h).
+    const float sl2 = kF8 ? p.scale_log2e * p.descale[b * p.H + hg] *
+                                p.descale[(p.B + b) * p.H + hg]
+                          : p.scale_log2e;
     const int tail = p.N - (T - 1) * C::kBN;   // valid keys in the last tile, 1..128
     float m_ref = -INFINITY;                   // reference maximum, log2 units
     float l = 0.f;
@@ -362,7 +387,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
                              fmaxf(mc[6], mc[7])) * sl2;
-      const bool need = mx > m_ref + 8.0f;
+      const bool need = mx > m_ref + C::kThresh;
       const bool warp_rescale = __any_sync(0xffffffffu, need);
       const float alpha = need ? ex2(m_ref - mx) : 1.0f;
       if (need) {
@@ -374,7 +399,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       // (bf16, over the first 64 columns of S_t) and signalled on its own, so
       // the PV MMAs of keys 0..63 can start while keys 64..127 are computed.
       const uint64_t k_sl2 = f2_pack(sl2, sl2);
-      const uint64_t k_negm = f2_pack(-m_ref, -m_ref);
+      const uint64_t k_negm = f2_pack(C::kShift - m_ref, C::kShift - m_ref);
       uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -388,7 +413,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
           p0 = ex2(p0);
           p1 = ex2(p1);
           acc[i & 1] = f2_add(acc[i & 1], f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
+          if (kF8) {
+            // four E4M3 probabilities per 32-bit column, key order in bytes
+            const uint32_t two = pack_e4m3x2(p0, p1);
+            pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (two << 16)) : two;
+          } else {
+            pk[i] = pack_bf16x2(p0, p1);
+          }
         }
         if (h == 0 && warp_rescale && j > 0) {
           // Rescale O_t by alpha before any PV MMA of this tile (warp-uniform
@@ -405,7 +436,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
             tmem_st8(tO + c, o);
           }
         }
-        tmem_st32(tS + 32 * h, pk);
+        if (kF8)
+          tmem_st16(tS + (C::kPCols / 2) * h, pk);
+        else
+          tmem_st32(tS + (C::kPCols / 2) * h, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar_p + 16 * t + 8 * h);
@@ -424,7 +458,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       const int token = q0 + t * C::kBM + row;
       const bool valid = token < p.N;
       const bool exists = token < p.Np;
-      const float inv_l = valid ? 1.0f / l : 0.0f;
+      const float inv_l = valid ? (kF8 ? p.descale[(2 * p.B + b) * p.H + hg] : 1.0f) / l : 0.0f;
       int64_t row_off;
       if (p.nl_split) {
         const int rk = token / p.nl_split, n = token - rk * p.nl_split;
@@ -453,7 +487,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
       }
       if (p.lse != nullptr && exists) {
-        const float v = valid ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const float v = valid ? (m_ref - C::kShift + __log2f(l)) * 0.69314718055994531f
+                              : -INFINITY;
         p.lse[(static_cast<int64_t>(b) * p.H + hg) * p.Np + token] = v;
       }
     } else {

@@ -122,17 +122,20 @@ sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, i
 
 // Tensor map over one of Q/K/V, viewed as [Bx][N rows][Hx heads][D] with
 // the given row and batch strides (elements).  Rows >= N read as zero.
+// es: element size in bytes (2: bf16, 1: E4M3 moved as bytes).  The box is
+// 128 bytes wide: 64 bf16 or 128 E4M3 elements.
 bool make_map(CUtensorMap *m, const void *base, int D, int Hx, int N, int Bx, int64_t row_el,
-              int64_t batch_el) {
+              int64_t batch_el, int es = 2) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hx),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(Bx)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(row_el) * 2,
-                           static_cast<cuuint64_t>(batch_el) * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(row_el) * es,
+                           static_cast<cuuint64_t>(batch_el) * es};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, 128, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+  CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
+                   const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -142,27 +145,30 @@ bool make_map(CUtensorMap *m, const void *base, int D, int Hx, int N, int Bx, in
 // P > 1), dims inner to outer (D, H, Nl, B, P).  Used only for token tiles
 // that lie inside one shard; the box is 128 rows (or Nl when smaller, in
 // which case no tile uses the map).
-bool make_map5(CUtensorMap *m, const void *base, int D, int H, int Nl, int B, int P) {
+bool make_map5(CUtensorMap *m, const void *base, int D, int H, int Nl, int B, int P,
+               int es = 2) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
-  const cuuint64_t row = static_cast<cuuint64_t>(H) * D * 2;
+  const cuuint64_t row = static_cast<cuuint64_t>(H) * D * es;
   cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(Nl), static_cast<cuuint64_t>(B),
                         static_cast<cuuint64_t>(P)};
-  cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * 2, row, row * Nl,
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * es, row, row * Nl,
                            row * Nl * static_cast<cuuint64_t>(B)};
-  cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(Nl < 128 ? Nl : 128), 1, 1};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / es), 1,
+                       static_cast<cuuint32_t>(Nl < 128 ? Nl : 128), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
+  CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 5,
+                   const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const sp::AttnParams &p, int B, cudaStream_t cs) {
-  using C = sp::AttnCfg<D>;
+  using C = sp::AttnCfg<D, kF8>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -171,14 +177,14 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
   {
     std::lock_guard<std::mutex> g(g_mu);
     if (!attr_set[dev]) {
-      e = cudaFuncSetAttribute(sp::attention_kernel<D>,
+      e = cudaFuncSetAttribute(sp::attention_kernel<D, kF8>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
       if (e != cudaSuccess) return e;
       attr_set[dev] = true;
     }
   }
   dim3 grid((p.N + 2 * C::kBM - 1) / (2 * C::kBM), p.H, B);
-  sp::attention_kernel<D><<<grid, C::kThreads, C::kSmemBytes, cs>>>(q, k, v, p);
+  sp::attention_kernel<D, kF8><<<grid, C::kThreads, C::kSmemBytes, cs>>>(q, k, v, p);
   return cudaGetLastError();
 }
 
@@ -187,15 +193,20 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
 // finds (slot, head-in-slot) of global head h as (h / hsplit * B + b,
 // h % hsplit).
 sp_status attention(const void *q, const void *k, const void *v, void *o, float *lse,
-                    const sp_shape *s, void *stream, bool seqsharded) {
+                    const sp_shape *s, void *stream, bool seqsharded,
+                    const float *descale = nullptr) {
+  const bool f8 = descale != nullptr;
+  const int es = f8 ? 1 : 2;
   // The fused call shards tokens only; heads are never split, so it takes
   // any P (the per-rank call of the multi-GPU form has Hl heads and P shards).
   sp_status st = check_common(s, !seqsharded);
   if (st != SP_OK) return st;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SP_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) ||
+      (f8 && (reinterpret_cast<uintptr_t>(descale) & 3u) != 0))
     return SP_ERR_ALIGN;
+  if (f8 && s->D != 128) return SP_ERR_UNSUPPORTED_D;
   const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
   const int Hl = H / P;
   const int Nl = (N + P - 1) / P;
@@ -220,12 +231,12 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   if (status == nullptr) return SP_ERR_CUDA;
   CUtensorMap mq, mk, mv;
   if (rank_major) {
-    if (!make_map5(&mq, q, D, H, Nl, B, P) || !make_map5(&mk, k, D, H, Nl, B, P) ||
-        !make_map5(&mv, v, D, H, Nl, B, P))
+    if (!make_map5(&mq, q, D, H, Nl, B, P, es) || !make_map5(&mk, k, D, H, Nl, B, P, es) ||
+        !make_map5(&mv, v, D, H, Nl, B, P, es))
       return SP_ERR_CUDA;
-  } else if (!make_map(&mq, q, D, Hx, N, Bx, row_el, batch_el) ||
-             !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el) ||
-             !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el)) {
+  } else if (!make_map(&mq, q, D, Hx, N, Bx, row_el, batch_el, es) ||
+             !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el, es) ||
+             !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el, es)) {
     return SP_ERR_CUDA;
   }
   sp::AttnParams p;
@@ -244,12 +255,14 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   p.status = status;
   p.nl_split = rank_major ? Nl : 0;
   p.o_rank = static_cast<int64_t>(B) * Nl * H * D;
-  p.q = static_cast<const __nv_bfloat16 *>(q);
-  p.k = static_cast<const __nv_bfloat16 *>(k);
-  p.v = static_cast<const __nv_bfloat16 *>(v);
+  p.q = static_cast<const uint8_t *>(q);
+  p.k = static_cast<const uint8_t *>(k);
+  p.v = static_cast<const uint8_t *>(v);
+  p.descale = descale;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  cudaError_t e = D == 64 ? launch_attention<64>(mq, mk, mv, p, B, cs)
-                          : launch_attention<128>(mq, mk, mv, p, B, cs);
+  cudaError_t e = f8        ? launch_attention<128, true>(mq, mk, mv, p, B, cs)
+                  : D == 64 ? launch_attention<64>(mq, mk, mv, p, B, cs)
+                            : launch_attention<128>(mq, mk, mv, p, B, cs);
   return launch_status(e);
 }
 
@@ -312,6 +325,13 @@ sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh,
 sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs, void *os,
                                   float *lse, const sp_shape *shape, void *stream) {
   return attention(qs, ks, vs, os, lse, shape, stream, true);
+}
+
+sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void *vs,
+                                      const float *descale, void *os, float *lse,
+                                      const sp_shape *shape, void *stream) {
+  if (descale == nullptr) return SP_ERR_NULL;
+  return attention(qs, ks, vs, os, lse, shape, stream, true, descale);
 }
 
 sp_status sp_device_status(void *stream) {
