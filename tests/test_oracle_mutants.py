@@ -47,6 +47,12 @@ MUTANTS = [
      "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     ("e4m3-subnormal-scale", "if (e == 0) v = ldexp((double)m / 8.0, -6);",
      "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
+    ("descale-dropped", "return e4m3_to_f64(x8[e]) * scale[bh];",
+     "return e4m3_to_f64(x8[e]);"),
+    ("descale-first-head-only", "return e4m3_to_f64(x8[e]) * scale[bh];",
+     "return e4m3_to_f64(x8[e]) * scale[0];"),
+    ("v-takes-q-descale", "elem(J->v, J->v8, J->dv, bh, vr + c)",
+     "elem(J->v, J->v8, J->dq, bh, vr + c)"),
 ]
 
 
