@@ -15,7 +15,8 @@ What it computes, and the passages it follows:
   generation across four GPUs" (each GPU sees the full sequence for its share
   of the heads, then the shards return).  Index formulas in ``sp_oracle.c``.
 * ``attention_rows_e4m3`` -- the same attention on 8-bit (E4M3) inputs with
-  per-(batch, head) scale factors, for the FP8 variant of the kernel.
+  scale factors per block of tokens for Q and K and per channel for V, for
+  the FP8 variant of the kernel.
 * ``attention_rows`` -- the unsharded softmax(q K^T scale) V of one head,
   two-pass exact softmax in fp64; the sequence-parallel result must equal it
   for every degree (LTX-2 "Multi-GPU Inference" README, Capabilities table:
@@ -64,7 +65,7 @@ def _bind(path: str):
         ctypes.c_int]
     lib.sp_oracle_attention_rows.restype = ctypes.c_int
     lib.sp_oracle_attention_rows_e4m3.argtypes = [
-        vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp,
+        vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp,
         ctypes.c_int]
     lib.sp_oracle_attention_rows_e4m3.restype = ctypes.c_int
     lib.sp_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
@@ -186,16 +187,26 @@ def e4m3_value(byte: int, lib=None) -> float:
 
 
 def attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows, scale: float = 0.0,
-                        threads: Optional[int] = None, lib=None):
-    """fp64 attention of e4m3 inputs: element values are the exact e4m3 values
-    (uint8 arrays, logical [B][N][H][D]) times per-(b, h) factors dq, dk, dv
-    ([B][H] float64).  Returns (O [R][D], LSE [R])."""
+                        threads: Optional[int] = None, block: int = 128, lib=None):
+    """fp64 attention of e4m3 inputs (uint8 arrays, logical [B][N][H][D]).
+    Element values are the exact e4m3 values times scale factors: Q and K
+    element (b, t, h, c) take dq[b][h][t // block] and dk[b][h][t // block],
+    V element (b, t, h, c) takes dv[b][h][c].  dq and dk broadcast to
+    [B][H][ceil(N / block)] and dv to [B][H][D]; a [B][H] array gives one
+    factor per (b, h).  Returns (O [R][D], LSE [R])."""
     for a in (q8, k8, v8):
         assert a.dtype == np.uint8 and a.shape == q8.shape and a.ndim == 4
     B, N, H, D = q8.shape
+    nblk = -(-N // block)
     q8, k8, v8 = (np.ascontiguousarray(a) for a in (q8, k8, v8))
-    dq, dk, dv = (np.ascontiguousarray(np.broadcast_to(np.asarray(d, dtype=np.float64), (B, H)))
-                  for d in (dq, dk, dv))
+
+    def factors(d, last):
+        d = np.asarray(d, dtype=np.float64)
+        if d.ndim == 2:
+            d = d[:, :, None]
+        return np.ascontiguousarray(np.broadcast_to(d, (B, H, last)))
+
+    dq, dk, dv = factors(dq, nblk), factors(dk, nblk), factors(dv, D)
     rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
     R = rows.shape[0]
     o = np.empty((R, D), dtype=np.float64)
@@ -204,8 +215,8 @@ def attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows, scale: float = 0.0,
         threads = max(1, len(os.sched_getaffinity(0)))
     rc = (lib or _load()).sp_oracle_attention_rows_e4m3(
         q8.ctypes.data, k8.ctypes.data, v8.ctypes.data, dq.ctypes.data, dk.ctypes.data,
-        dv.ctypes.data, B, N, H, D, float(scale), R, rows.ctypes.data, o.ctypes.data,
-        lse.ctypes.data, int(threads))
+        dv.ctypes.data, int(block), B, N, H, D, float(scale), R, rows.ctypes.data,
+        o.ctypes.data, lse.ctypes.data, int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle attention failed ({rc})")
     return o, lse

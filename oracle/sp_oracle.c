@@ -29,8 +29,15 @@
  *  - attention is non-causal softmax(q k^T * scale) v over all N tokens with
  *    scale = 1/sqrt(D) unless given; no mask except the padding slots.
  *
- * Element type: bf16, given as its 16-bit pattern.  The oracle widens each
- * bf16 value exactly to double.
+ *  - FP8 attention (named for the FastVideo stack on "Pair two NVIDIA DGX
+ *    Sparks" without a definition): the same attention on inputs stored as
+ *    E4M3 bytes, each element scaled by a factor; Q and K carry one factor per
+ *    block of consecutive tokens, V one per channel (the contraction of q.k
+ *    runs over channels and that of p.v over tokens, so these factors come
+ *    out of the sums).
+ *
+ * Element type: bf16, given as its 16-bit pattern, or E4M3 bytes with their
+ * factors.  The oracle widens each value exactly to double.
  */
 #include <math.h>
 #include <pthread.h>
@@ -170,7 +177,10 @@ int sp_oracle_exchange_unpack(const uint16_t *recv, uint16_t *os_r, int64_t B, i
 typedef struct {
     const uint16_t *q, *k, *v;
     const uint8_t *q8, *k8, *v8;       /* e4m3 inputs instead of bf16, or NULL */
-    const double *dq, *dk, *dv;        /* per-(b, h) scale factors of q8/k8/v8 */
+    /* Scale factors of the e4m3 inputs: dq and dk [B][H][nblk], one per block
+     * of blk consecutive tokens; dv [B][H][D], one per channel. */
+    const double *dq, *dk, *dv;
+    int64_t blk, nblk;
     int64_t B, N, H, D;
     double scale;
     int64_t nrows;
@@ -182,10 +192,9 @@ typedef struct {
 } attn_job_t;
 
 /* Element e of a logical [B][N][H][D] input: bf16 words, or e4m3 bytes
- * times the per-(b, h) scale. */
-static double elem(const uint16_t *x16, const uint8_t *x8, const double *scale, int64_t bh,
-                   int64_t e) {
-    if (x8) return e4m3_to_f64(x8[e]) * scale[bh];
+ * times the scale factor that applies to that element. */
+static double elem(const uint16_t *x16, const uint8_t *x8, double scale, int64_t e) {
+    if (x8) return e4m3_to_f64(x8[e]) * scale;
     return bf16_to_f64(x16[e]);
 }
 
@@ -193,12 +202,14 @@ static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
     int64_t b = J->rows[3 * r], h = J->rows[3 * r + 1], i = J->rows[3 * r + 2];
     int64_t N = J->N, H = J->H, D = J->D, bh = b * H + h;
     int64_t qi = ((b * N + i) * H + h) * D;
+    double sq = J->q8 ? J->dq[bh * J->nblk + i / J->blk] : 1.0;
     double m = -INFINITY;
     for (int64_t kk = 0; kk < N; ++kk) {
         int64_t kr = ((b * N + kk) * H + h) * D;
+        double sk = J->k8 ? J->dk[bh * J->nblk + kk / J->blk] : 1.0;
         double dot = 0.0;
         for (int64_t c = 0; c < D; ++c)
-            dot += elem(J->q, J->q8, J->dq, bh, qi + c) * elem(J->k, J->k8, J->dk, bh, kr + c);
+            dot += elem(J->q, J->q8, sq, qi + c) * elem(J->k, J->k8, sk, kr + c);
         s[kk] = J->scale * dot;
         if (s[kk] > m) m = s[kk];
     }
@@ -209,7 +220,8 @@ static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
         double w = exp(s[kk] - m);
         l += w;
         int64_t vr = ((b * N + kk) * H + h) * D;
-        for (int64_t c = 0; c < D; ++c) o[c] += w * elem(J->v, J->v8, J->dv, bh, vr + c);
+        for (int64_t c = 0; c < D; ++c)
+            o[c] += w * elem(J->v, J->v8, J->v8 ? J->dv[bh * D + c] : 1.0, vr + c);
     }
     for (int64_t c = 0; c < D; ++c) o[c] /= l;
     if (J->out_lse) J->out_lse[r] = m + log(l);
@@ -254,17 +266,22 @@ int sp_oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_
     return attention_rows_impl(&J, nthreads);
 }
 
-/* The same attention on e4m3 inputs: element values are the exact e4m3
- * values times per-(b, h) scale factors dq/dk/dv ([B][H] each). */
+/* The same attention on e4m3 inputs.  Element values are the exact e4m3
+ * values times scale factors: q[b][t][h][c] and k[b][t][h][c] take
+ * dq[b][h][t / blk] and dk[b][h][t / blk] (one factor per block of blk
+ * tokens, nblk = ceil(N / blk) blocks), v[b][t][h][c] takes dv[b][h][c]. */
 int sp_oracle_attention_rows_e4m3(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8,
                                   const double *dq, const double *dk, const double *dv,
+                                  int64_t blk,
                                   int64_t B, int64_t N, int64_t H, int64_t D, double scale,
                                   int64_t nrows, const int64_t *rows, double *out_o,
                                   double *out_lse, int nthreads) {
     attn_job_t J;
     memset(&J, 0, sizeof(J));
+    if (blk < 1) return -1;
     J.q8 = q8; J.k8 = k8; J.v8 = v8;
     J.dq = dq; J.dk = dk; J.dv = dv;
+    J.blk = blk; J.nblk = (N + blk - 1) / blk;
     J.B = B; J.N = N; J.H = H; J.D = D;
     J.scale = scale;
     J.nrows = nrows; J.rows = rows;

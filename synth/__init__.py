@@ -257,16 +257,33 @@ def to_e4m3(x: np.ndarray) -> np.ndarray:
         torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
-def fp8_qkv(cfg: Config, threads: Optional[int] = None):
-    """8-bit inputs for the FP8 variant: the config's bf16 Q, K, V, each
-    scaled per (batch, head) so its largest magnitude maps to 448, then
-    rounded to E4M3.  Returns (q8, k8, v8) as logical [B][N][H][D] uint8 and
-    the descale factors d [3][B][H] float32 (value = e4m3 value * d)."""
-    out, scales = [], []
-    for x in qkv_logical(cfg, threads):
-        f = bf16_to_f32(x)                                    # [B][N][H][D]
-        amax = np.abs(f).max(axis=(1, 3)).astype(np.float32)  # [B][H]
-        d = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-        out.append(to_e4m3(f / d[:, None, :, None]))
-        scales.append(d)
-    return out[0], out[1], out[2], np.stack(scales)
+FP8_BLOCK = 128   # tokens per Q/K scale block of the 8-bit inputs
+
+
+def fp8_qkv(cfg: Config, threads: Optional[int] = None, block: int = FP8_BLOCK):
+    """8-bit inputs for the FP8 variant: the config's bf16 Q, K, V scaled so
+    that each scale group's largest magnitude maps to 448, then rounded to
+    E4M3.  Q and K have one factor per (batch, head, block of `block`
+    tokens), V one per (batch, head, channel).  Returns q8, k8, v8 (logical
+    [B][N][H][D] uint8) and the factors dq, dk [B][H][ceil(N / block)] and
+    dv [B][H][D] (float32; element value = e4m3 value * factor)."""
+    q, k, v = (bf16_to_f32(x) for x in qkv_logical(cfg, threads))
+    B, N, H, D = q.shape
+    nblk = -(-N // block)
+
+    def factor(amax):
+        return np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+
+    def per_block(x):
+        pad = np.zeros((B, nblk * block, H, D), dtype=np.float32)
+        pad[:, :N] = np.abs(x)
+        amax = pad.reshape(B, nblk, block, H, D).max(axis=(2, 4))    # [B][nblk][H]
+        d = factor(amax.transpose(0, 2, 1))                           # [B][H][nblk]
+        tok = np.arange(N) // block
+        return to_e4m3(x / d.transpose(0, 2, 1)[:, tok, :, None]), np.ascontiguousarray(d)
+
+    q8, dq = per_block(q)
+    k8, dk = per_block(k)
+    dv = factor(np.abs(v).max(axis=1))                                # [B][H][D]
+    v8 = to_e4m3(v / dv[:, None, :, :])
+    return q8, k8, v8, dq, dk, np.ascontiguousarray(dv)

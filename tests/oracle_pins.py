@@ -335,6 +335,35 @@ def check_fp8_attention_reduces_to_bf16(lib=None):
         assert np.max(np.abs(o8s[r] - dv[b, h] * want[0])) < 1e-12
 
 
+def check_fp8_block_factors_match_dequantized_bf16(lib=None):
+    """Q and K factors per block of tokens and V factors per channel, all
+    powers of two, times small integers give values exact in bf16: the e4m3
+    attention must equal the (pinned) bf16 attention of the dequantized
+    tensors.  Block size 8 over N = 33 leaves a ragged last block."""
+    rng = np.random.default_rng(RNG_SEED + 17)
+    B, N, H, D, blk = 2, 33, 3, 16, 8
+    nblk = -(-N // blk)
+    fq, fk, fv = (rng.integers(-3, 4, size=(B, N, H, D)).astype(np.float32) for _ in range(3))
+    q8, k8, v8 = (_e4m3_from_float(x) for x in (fq, fk, fv))
+    dq = 2.0 ** rng.integers(-2, 3, size=(B, H, nblk))
+    dk = 2.0 ** rng.integers(-2, 3, size=(B, H, nblk))
+    dv = 2.0 ** rng.integers(-2, 3, size=(B, H, D))
+    tok_blk = np.arange(N) // blk
+    deq_q = fq * dq.transpose(0, 2, 1)[:, tok_blk, :, None]
+    deq_k = fk * dk.transpose(0, 2, 1)[:, tok_blk, :, None]
+    deq_v = fv * dv[:, None, :, :]
+    qb, kb, vb = (synth.f32_to_bf16(x.astype(np.float32)) for x in (deq_q, deq_k, deq_v))
+    for x, xb in ((deq_q, qb), (deq_k, kb), (deq_v, vb)):
+        assert np.array_equal(synth.bf16_to_f32(xb), x.astype(np.float32))  # exact in bf16
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(N)], np.int64)
+    scale = 0.05
+    o8, l8 = oracle.attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows, scale, 2, block=blk,
+                                        lib=lib)
+    ob, lb = oracle.attention_rows(qb, kb, vb, rows, scale, 2, lib=lib)
+    assert np.max(np.abs(o8 - ob)) < 1e-12 * max(1.0, np.max(np.abs(ob)))
+    assert np.max(np.abs(l8 - lb)) < 1e-12 * max(1.0, np.max(np.abs(lb)))
+
+
 PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
                check_unpack_returns_shards, check_pack_degree_one_is_copy,
                check_exchange_chunks_hold_head_groups,
@@ -342,5 +371,6 @@ PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_tran
 ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one,
                     check_closed_forms, check_dominant_key, check_invariances,
                     check_two_token_example, check_rows_api,
-                    check_e4m3_decode_matches_torch, check_fp8_attention_reduces_to_bf16]
+                    check_e4m3_decode_matches_torch, check_fp8_attention_reduces_to_bf16,
+                    check_fp8_block_factors_match_dequantized_bf16]
 ALL_CHECKS = PACK_CHECKS + ATTENTION_CHECKS

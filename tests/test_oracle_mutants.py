@@ -41,18 +41,22 @@ MUTANTS = [
      "for (int64_t kk = 0; kk < N; ++kk) {\n        double w",
      "for (int64_t kk = 0; kk + 1 < N; ++kk) {\n        double w"),
     ("k-transposed-with-q",
-     "elem(J->k, J->k8, J->dk, bh, kr + c);",
-     "elem(J->q, J->q8, J->dq, bh, qi + c);"),
+     "elem(J->k, J->k8, sk, kr + c);",
+     "elem(J->q, J->q8, sq, qi + c);"),
     ("e4m3-exponent-bias", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
      "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     ("e4m3-subnormal-scale", "if (e == 0) v = ldexp((double)m / 8.0, -6);",
      "if (e == 0) v = ldexp((double)m / 8.0, -7);"),
-    ("descale-dropped", "return e4m3_to_f64(x8[e]) * scale[bh];",
+    ("descale-dropped", "return e4m3_to_f64(x8[e]) * scale;",
      "return e4m3_to_f64(x8[e]);"),
-    ("descale-first-head-only", "return e4m3_to_f64(x8[e]) * scale[bh];",
-     "return e4m3_to_f64(x8[e]) * scale[0];"),
-    ("v-takes-q-descale", "elem(J->v, J->v8, J->dv, bh, vr + c)",
-     "elem(J->v, J->v8, J->dq, bh, vr + c)"),
+    ("q-factor-first-head-only", "J->dq[bh * J->nblk + i / J->blk]",
+     "J->dq[i / J->blk]"),
+    ("q-factor-next-block", "J->dq[bh * J->nblk + i / J->blk]",
+     "J->dq[bh * J->nblk + (i + 1) / J->blk - ((i + 1) / J->blk == J->nblk)]"),
+    ("k-factor-of-query-block", "J->dk[bh * J->nblk + kk / J->blk]",
+     "J->dk[bh * J->nblk + i / J->blk]"),
+    ("v-factor-of-channel-0", "J->dv[bh * D + c]", "J->dv[bh * D]"),
+    ("v-takes-q-factor", "J->v8 ? J->dv[bh * D + c] : 1.0", "J->v8 ? sq : 1.0"),
 ]
 
 

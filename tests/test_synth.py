@@ -86,3 +86,30 @@ def test_sampled_rows_cover_boundaries():
     assert len(rows) == 256 and len(set(rows.tolist())) == 256
     for t in (0, s.N - 1, 18900 - 1, 18900, 37800, 56700, 9450, 9450 - 1):
         assert t in rows
+
+
+def test_fp8_quantisation_groups():
+    """Q/K factors per (batch, head, 128-token block), V factors per (batch,
+    head, channel): each group's largest magnitude becomes 448 exactly, and
+    every dequantized value is within E4M3's rounding of the bf16 value."""
+    import torch
+    cfg = synth.Config("f8", synth.Shape(2, 300, 3, 16, 1), seed=11)
+    q, k, v = (synth.bf16_to_f32(x) for x in synth.qkv_logical(cfg))
+    q8, k8, v8, dq, dk, dv = synth.fp8_qkv(cfg)
+    assert dq.shape == dk.shape == (2, 3, 3) and dv.shape == (2, 3, 16)
+
+    def val(x8):
+        return torch.from_numpy(x8).view(torch.float8_e4m3fn).float().numpy()
+
+    tok = np.arange(300) // 128
+    for x, x8, d in ((q, q8, dq), (k, k8, dk)):
+        deq = val(x8) * d.transpose(0, 2, 1)[:, tok, :, None]
+        groups = np.abs(val(x8)).max(axis=3)                      # [B][N][H]
+        for blk in range(3):
+            sel = tok == blk
+            assert np.all(groups[:, sel].max(axis=1) == 448.0)
+        bound = 2.0 ** -4 * np.abs(x) + 2.0 ** -10 * d.transpose(0, 2, 1)[:, tok, :, None]
+        assert np.all(np.abs(deq - x) <= bound)
+    deq_v = val(v8) * dv[:, None]
+    assert np.all(np.abs(val(v8)).max(axis=1) == 448.0)
+    assert np.all(np.abs(deq_v - v) <= 2.0 ** -4 * np.abs(v) + 2.0 ** -10 * dv[:, None])
