@@ -137,22 +137,34 @@ sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs
                                   void *os, float *lse, const sp_shape *shape,
                                   void *stream);
 
-/* FP8 variant of sp_attention_seqsharded: Q, K and V in OCP E4M3 (one byte
- * per element; value = byte value * per-(batch, head) descale factor), the
- * output O in bf16 as for the bf16 call.  QK^T and PV run on the tensor
- * cores' 8-bit path with fp32 accumulation; the probabilities are rounded to
- * E4M3 (relative rounding error at most 2^-4) before the PV product, scaled
- * by 2^6 relative to the running row maximum so that the typical weights of
- * long sequences keep E4M3's 3 mantissa bits.  The pages name FP8 and FP4
- * attention (FastVideo, "Pair two NVIDIA DGX Sparks", the NVFP4 stacks)
- * without defining it; this is the plainest reading: the same attention on
- * dequantized 8-bit inputs.
+/* Tokens per scale block of the FP8 call's Q and K factors. */
+#define SP_FP8_BLOCK 128
+
+/* FP8 variant of sp_attention_seqsharded: Q, K and V in OCP E4M3, one byte
+ * per element, each element scaled by a factor: Q and K element (b, t, h, c)
+ * by q_scale / k_scale [b][h][t / SP_FP8_BLOCK], V element (b, t, h, c) by
+ * v_scale[b][h][c].  The output O is bf16 as for the bf16 call.  QK^T and PV
+ * run on the tensor cores' 8-bit path with fp32 accumulation; the
+ * probabilities are rounded to E4M3 (relative rounding error at most 2^-4)
+ * before the PV product, scaled by 2^6 relative to the running row maximum
+ * so that the typical weights of long sequences keep E4M3's 3 mantissa bits.
+ * The pages name FP8 and FP4 attention (FastVideo, "Pair two NVIDIA DGX
+ * Sparks", the NVFP4 stacks) without defining it; this is the plainest
+ * reading: the same attention on dequantized 8-bit inputs, with factors at
+ * the granularity the two products allow (q.k sums over channels, so Q and K
+ * factors may change from token block to token block; p.v sums over tokens,
+ * so V factors may change from channel to channel).
  * qs, ks, vs: device [P][B][Nl][H][D] uint8 (E4M3), read only, 16-byte
- * aligned; D must be 128.  descale: device fp32 [3][B][H] (q, k, v factors),
- * read only.  os: device [P][B][Nl][H][D] bf16, written.  lse: device fp32
- * [B][H][Np] or NULL.  Results do not depend on P (bit-identical). */
+ * aligned; D must be 128.  q_scale, k_scale: device fp32
+ * [B][H][ceil(N / SP_FP8_BLOCK)]; v_scale: device fp32 [B][H][D]; all read
+ * only, 4-byte aligned, finite and positive.  os: device [P][B][Nl][H][D]
+ * bf16, written.  lse: device fp32 [B][H][Np] or NULL (natural log of the
+ * row sum of exp(scaled logits)).  Results do not depend on P
+ * (bit-identical).  Errors: SP_ERR_NULL for a NULL scale pointer, otherwise
+ * as for sp_attention_seqsharded. */
 sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void *vs,
-                                      const float *descale, void *os, float *lse,
+                                      const float *q_scale, const float *k_scale,
+                                      const float *v_scale, void *os, float *lse,
                                       const sp_shape *shape, void *stream);
 
 /* Synchronises `stream`, then returns and clears the device status word:

@@ -100,6 +100,17 @@ def test_argument_errors_return_before_launch(lib):
         sp.SP_ERR_HEADS_NOT_DIVISIBLE
     assert lib.sp_check_shape(ctypes.byref(sp.Shape(1, 1024, 4, 64, 3).c())) == \
         sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    f8 = lambda q, k, v, dq, dk, dv, o, lse=None, shp=sp.Shape(1, 1024, 4, 128, 2): \
+        lib.sp_attention_fp8_seqsharded(
+            *[ctypes.c_void_p(x) if x else None for x in (q, k, v, dq, dk, dv, o, lse)],
+            ctypes.byref(shp.c()), None)
+    C = 0x40000
+    assert f8(A, A, A, C, C, 0, B_) == sp.SP_ERR_NULL          # each factor array required
+    assert f8(A, A, A, 0, C, C, B_) == sp.SP_ERR_NULL
+    assert f8(A, A, A, C, 0, C, B_) == sp.SP_ERR_NULL
+    assert f8(A, A, A, C, C + 2, C, B_) == sp.SP_ERR_ALIGN      # fp32 factors, 4-byte aligned
+    assert f8(A, A, A + 8, C, C, C, B_) == sp.SP_ERR_ALIGN
+    assert f8(A, A, A, C, C, C, B_, shp=sp.Shape(1, 1024, 4, 64, 2)) == sp.SP_ERR_UNSUPPORTED_D
     for fn in (lib.sp_exchange_pack, lib.sp_exchange_unpack):
         assert _call(fn, 0, B_, shape=shape) == sp.SP_ERR_NULL
         assert _call(fn, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN

@@ -320,11 +320,14 @@ FP8_MAX_REL = 2.0 ** -3
 
 
 def _fp8_inputs(B, N, H, D, seed):
+    """E4M3 bytes of the seeded bf16 inputs, factors per 128-token block (Q,
+    K) and per channel (V): returns q8, k8, v8 and f = (dq, dk, dv)."""
     cfg = synth.Config("f8", synth.Shape(B, N, H, D, 1), seed=seed)
-    return synth.fp8_qkv(cfg)
+    q8, k8, v8, dq, dk, dv = synth.fp8_qkv(cfg)
+    return q8, k8, v8, (dq, dk, dv)
 
 
-def _run_fp8(q8, k8, v8, d, P, lse=False):
+def _run_fp8(q8, k8, v8, f, P, lse=False):
     B, N, H, D = q8.shape
     shape = sp.Shape(B, N, H, D, P)
 
@@ -333,16 +336,16 @@ def _run_fp8(q8, k8, v8, d, P, lse=False):
 
     os_ = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
     l = torch.full(shape.lse_shape, float("nan"), dtype=torch.float32, device="cuda") if lse else None
-    sp.attention_fp8_seqsharded(dev8(q8), dev8(k8), dev8(v8), torch.from_numpy(d).cuda(), os_,
-                                shape, lse=l)
+    dq, dk, dv = (torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda() for x in f)
+    sp.attention_fp8_seqsharded(dev8(q8), dev8(k8), dev8(v8), dq, dk, dv, os_, shape, lse=l)
     _status_ok()
     return to_host(os_), (l.cpu().numpy() if lse else None)
 
 
-def _check_fp8(out, q8, k8, v8, d, rows, P, where):
+def _check_fp8(out, q8, k8, v8, f, rows, P, where):
     B, N, H, D = q8.shape
     O = synth.from_seq_shards(out.reshape(P, B, -1, H, D), N)
-    ref, _ = oracle.attention_rows_e4m3(q8, k8, v8, d[0], d[1], d[2], rows)
+    ref, _ = oracle.attention_rows_e4m3(q8, k8, v8, f[0], f[1], f[2], rows)
     m = compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1])
     assert m["finite"], where
     assert m["rel_l2"] <= FP8_REL_L2, (where, m)
@@ -367,10 +370,37 @@ def test_fp8_attention_against_oracle(B, N, H, P):
     assert np.max(np.abs(got - lse_ref)) < 2e-2
 
 
+def test_fp8_block_and_channel_factors():
+    """Factors that change by powers of two from one 128-token block to the
+    next (Q, K) and from channel to channel (V), over a ragged N: the kernel
+    must apply block j's factor to key tile j, the query tile's own factor,
+    and channel c's factor to output column c."""
+    B, N, H, D, P = 2, 1000, 4, 128, 4
+    q8, k8, v8, _ = _fp8_inputs(B, N, H, D, seed=77)
+    rng = np.random.default_rng(77)
+    nblk = -(-N // 128)
+    dq = (2.0 ** rng.integers(-2, 3, size=(B, H, nblk)) / 256).astype(np.float32)
+    dk = (2.0 ** rng.integers(-2, 3, size=(B, H, nblk)) / 256).astype(np.float32)
+    dv = (2.0 ** rng.integers(-3, 4, size=(B, H, D)) / 256).astype(np.float32)
+    f = (dq, dk, dv)
+    out, lse = _run_fp8(q8, k8, v8, f, P, lse=True)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H)
+                     for i in sorted({0, 127, 128, 500, 895, 896, N - 1,
+                                      *range(3, N, 37)})], dtype=np.int64)
+    m = _check_fp8(out, q8, k8, v8, f, rows, P, "fp8 block factors")
+    print(f"fp8 block factors: {m}")
+    _, lse_ref = oracle.attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows)
+    assert np.max(np.abs(lse[rows[:, 0], rows[:, 1], rows[:, 2]] - lse_ref)) < 2e-2
+    one, _ = _run_fp8(q8, k8, v8, f, 1)
+    assert np.array_equal(synth.from_seq_shards(out.reshape(P, B, -1, H, D), N),
+                          synth.from_seq_shards(one.reshape(1, B, -1, H, D), N))
+
+
 def test_fp8_720p_sampled_rows():
     cfg = synth.CONFIGS["720p"]
     s = cfg.shape
-    q8, k8, v8, d = synth.fp8_qkv(cfg)
+    q8, k8, v8, dq, dk, dv = synth.fp8_qkv(cfg)
+    d = (dq, dk, dv)
     out, _ = _run_fp8(q8, k8, v8, d, s.P)
     rows_t = synth.sampled_rows(cfg, 8)
     rows = np.array([(0, h, i) for h in range(s.H) for i in rows_t], dtype=np.int64)

@@ -80,7 +80,7 @@ def load(path: str = LIB_PATH):
         f = getattr(lib, name)
         f.argtypes = [vp, vp, vp, vp, vp, sp_p, vp]
         f.restype = ctypes.c_int
-    lib.sp_attention_fp8_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, sp_p, vp]
+    lib.sp_attention_fp8_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sp_p, vp]
     lib.sp_attention_fp8_seqsharded.restype = ctypes.c_int
     lib.sp_device_status.argtypes = [vp]
     lib.sp_device_status.restype = ctypes.c_int
@@ -96,6 +96,9 @@ def load(path: str = LIB_PATH):
 
 def status_str(status: int) -> str:
     return load().sp_status_str(int(status)).decode()
+
+
+FP8_BLOCK = 128  # tokens per Q/K scale block of the FP8 call (SP_FP8_BLOCK)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -146,6 +149,11 @@ class Shape:
     @property
     def lse_shape(self):
         return (self.B, self.H, self.Np)
+
+    @property
+    def fp8_blocks(self) -> int:
+        """Q/K scale blocks of the FP8 call: ceil(N / FP8_BLOCK)."""
+        return -(-self.N // FP8_BLOCK)
 
     def c(self) -> sp_shape:
         return sp_shape(self.B, self.N, self.H, self.D, self.P, float(self.scale))
@@ -263,19 +271,24 @@ def attention_seqsharded(qs, ks, vs, os_, shape: Shape, lse=None, stream=None):
             _stream(stream, qs.device)), "sp_attention_seqsharded")
 
 
-def attention_fp8_seqsharded(qs8, ks8, vs8, descale, os_, shape: Shape, lse=None,
-                             stream=None):
+def attention_fp8_seqsharded(qs8, ks8, vs8, q_scale, k_scale, v_scale, os_, shape: Shape,
+                             lse=None, stream=None):
     """FP8 (E4M3) variant of attention_seqsharded: qs8/ks8/vs8 are uint8
-    [P][B][Nl][H][D] E4M3 bytes, descale float32 [3][B][H] (q, k, v factors),
-    os_ bf16 [P][B][Nl][H][D]."""
+    [P][B][Nl][H][D] E4M3 bytes; q_scale and k_scale float32
+    [B][H][shape.fp8_blocks] (one factor per block of FP8_BLOCK tokens),
+    v_scale float32 [B][H][D] (one factor per channel); os_ bf16
+    [P][B][Nl][H][D]."""
     torch = _torch()
     s = shape.c()
     ss = shape.seq_sharded
-    with _same_device(qs8, ks8, vs8, descale, os_, lse):
+    blk = (shape.B, shape.H, shape.fp8_blocks)
+    with _same_device(qs8, ks8, vs8, q_scale, k_scale, v_scale, os_, lse):
         _check(load().sp_attention_fp8_seqsharded(
             _ptr(qs8, ss, "qs8", torch.uint8), _ptr(ks8, ss, "ks8", torch.uint8),
             _ptr(vs8, ss, "vs8", torch.uint8),
-            _ptr(descale, (3, shape.B, shape.H), "descale", torch.float32),
+            _ptr(q_scale, blk, "q_scale", torch.float32),
+            _ptr(k_scale, blk, "k_scale", torch.float32),
+            _ptr(v_scale, (shape.B, shape.H, shape.D), "v_scale", torch.float32),
             _ptr(os_, ss, "os"), _ptr(lse, shape.lse_shape, "lse", torch.float32),
             ctypes.byref(s), _stream(stream, qs8.device)), "sp_attention_fp8_seqsharded")
 

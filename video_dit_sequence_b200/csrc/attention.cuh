@@ -56,9 +56,11 @@ struct AttnParams {
   int32_t nl_split;
   int64_t o_rank;       // elements between rank slabs (B * Nl * H * D)
   const uint8_t *q, *k, *v;  // bases, for tiles that cross a shard boundary
-  // E4M3 variant: per-(batch, head) descale factors [3][B][H] (q, k, v);
-  // element value = byte value * factor.  Null for bf16.
-  const float *descale;
+  // E4M3 variant: scale factors, element value = byte value * factor.
+  // dq, dk: [B][H][nblk], one per block of 128 tokens (= one query or key
+  // tile); dv: [B][H][D], one per channel.  Null for bf16.
+  const float *dq, *dk, *dv;
+  int32_t nblk;
   float *lse;           // [B][H][Np] or null
   int32_t *status;      // device status word
 };
@@ -308,11 +310,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         it = 1;
       }
       for (int j = 0; j < T && ok; ++j) {
+        // Both K/V waits come first: the loads landed long ago, and no
+        // barrier wait sits between a tile's PV and its next S.
         const int sv = it % C::kStages;
         ok = mbar_wait(bar_kv_full + 8 * sv, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
         ++it;
-        if (!ok) break;
-        ok = issue_pv(0, sv, j == 0, j);
         if (!ok) break;
         int sk = 0;
         if (j + 1 < T) {
@@ -320,7 +322,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
           ok = mbar_wait(bar_kv_full + 8 * sk, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
           ++it;
           if (!ok) break;
-          tc_fence_after();
+        }
+        ok = issue_pv(0, sv, j == 0, j);
+        if (!ok) break;
+        if (j + 1 < T) {
           issue_s(0, sk);
           umma_commit(bar_s);
         } else {
@@ -328,13 +333,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         ok = issue_pv(1, sv, j == 0, j);
         if (!ok) break;
-        umma_commit(bar_kv_empty + 8 * sv);
         if (j + 1 < T) {
           issue_s(1, sk);
           umma_commit(bar_s + 8);
+          umma_commit(bar_kv_empty + 8 * sv);
           umma_commit(bar_kv_empty + 8 * sk);
         } else {
           umma_commit(bar_o + 8);
+          umma_commit(bar_kv_empty + 8 * sv);
         }
       }
     }
@@ -347,10 +353,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_bits + (t ? C::kColS1 : 0u);
     const uint32_t tO = tmem + lane_bits + (t ? C::kColO1 : C::kColO0);
-    // E4M3: the logits carry the q and k descale factors of this (b, h).
-    const float sl2 = kF8 ? p.scale_log2e * p.descale[b * p.H + hg] *
-                                p.descale[(p.B + b) * p.H + hg]
-                          : p.scale_log2e;
+    // E4M3: the logits carry the factor of this query tile's token block
+    // and, per key tile j, the factor of key block j (read one step ahead).
+    const int bh = b * p.H + hg;
+    const int qblk = blockIdx.x * 2 + t;
+    const float sl2q = kF8 && qblk < p.nblk ? p.scale_log2e * p.dq[bh * p.nblk + qblk]
+                                            : p.scale_log2e;
+    const float *dk_row = kF8 ? p.dk + static_cast<int64_t>(bh) * p.nblk : nullptr;
+    float dk_next = kF8 ? __ldg(dk_row) : 1.0f;
     const int tail = p.N - (T - 1) * C::kBN;   // valid keys in the last tile, 1..128
     float m_ref = -INFINITY;                   // reference maximum, log2 units
     float l = 0.f;
@@ -362,6 +372,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         break;
       }
       tc_fence_after();
+      const float sl2 = kF8 ? sl2q * dk_next : sl2q;
+      if (kF8 && j + 1 < T) dk_next = __ldg(dk_row + j + 1);
       uint32_t s[128];
       tmem_ld32(tS + 0, &s[0]);
       tmem_ld32(tS + 32, &s[32]);
@@ -427,13 +439,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
           // reference multiply by exactly 1).  O_t is complete: the commit
           // that signalled S_t also covered the previous PV.
 #pragma unroll 1
-          for (int c = 0; c < D; c += 8) {
-            uint32_t o[8];
-            tmem_ld8(tO + c, o);
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st8(tO + c, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + c, o);
           }
         }
         if (kF8)
@@ -458,7 +470,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       const int token = q0 + t * C::kBM + row;
       const bool valid = token < p.N;
       const bool exists = token < p.Np;
-      const float inv_l = valid ? (kF8 ? p.descale[(2 * p.B + b) * p.H + hg] : 1.0f) / l : 0.0f;
+      const float inv_l = valid ? 1.0f / l : 0.0f;
+      const float *dv_row = kF8 ? p.dv + static_cast<int64_t>(bh) * D : nullptr;
       int64_t row_off;
       if (p.nl_split) {
         const int rk = token / p.nl_split, n = token - rk * p.nl_split;
@@ -473,6 +486,12 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         uint32_t o[32];
         tmem_ld32(tO + c, o);
         tmem_wait_ld();
+        if (kF8) {
+          // E4M3: channel c of O carries V's factor of channel c.
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            o[i] = __float_as_uint(__uint_as_float(o[i]) * __ldg(dv_row + c + i));
+        }
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)

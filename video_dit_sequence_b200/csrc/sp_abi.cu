@@ -194,8 +194,10 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
 // h % hsplit).
 sp_status attention(const void *q, const void *k, const void *v, void *o, float *lse,
                     const sp_shape *s, void *stream, bool seqsharded,
-                    const float *descale = nullptr) {
-  const bool f8 = descale != nullptr;
+                    const float *dq = nullptr, const float *dk = nullptr,
+                    const float *dv = nullptr) {
+  const bool f8 = dq != nullptr;
+  if (f8 && (dk == nullptr || dv == nullptr)) return SP_ERR_NULL;
   const int es = f8 ? 1 : 2;
   // The fused call shards tokens only; heads are never split, so it takes
   // any P (the per-rank call of the multi-GPU form has Hl heads and P shards).
@@ -204,7 +206,8 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SP_ERR_NULL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) ||
-      (f8 && (reinterpret_cast<uintptr_t>(descale) & 3u) != 0))
+      (f8 && ((reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
+               reinterpret_cast<uintptr_t>(dv)) & 3u) != 0))
     return SP_ERR_ALIGN;
   if (f8 && s->D != 128) return SP_ERR_UNSUPPORTED_D;
   const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
@@ -258,7 +261,10 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   p.q = static_cast<const uint8_t *>(q);
   p.k = static_cast<const uint8_t *>(k);
   p.v = static_cast<const uint8_t *>(v);
-  p.descale = descale;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.nblk = p.num_kv_tiles;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   cudaError_t e = f8        ? launch_attention<128, true>(mq, mk, mv, p, B, cs)
                   : D == 64 ? launch_attention<64>(mq, mk, mv, p, B, cs)
@@ -328,10 +334,11 @@ sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs
 }
 
 sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void *vs,
-                                      const float *descale, void *os, float *lse,
+                                      const float *q_scale, const float *k_scale,
+                                      const float *v_scale, void *os, float *lse,
                                       const sp_shape *shape, void *stream) {
-  if (descale == nullptr) return SP_ERR_NULL;
-  return attention(qs, ks, vs, os, lse, shape, stream, true, descale);
+  if (q_scale == nullptr || k_scale == nullptr || v_scale == nullptr) return SP_ERR_NULL;
+  return attention(qs, ks, vs, os, lse, shape, stream, true, q_scale, k_scale, v_scale);
 }
 
 sp_status sp_device_status(void *stream) {
