@@ -20,7 +20,10 @@ the same single-GPU problem on its own GPU: independent problems, no
 data-path collective, weak scaling.  --mode ulysses instead splits the one
 problem across the N GPUs the way the method does (P = N ranks, NCCL
 all-to-all of the sequence shards, each GPU attends H/N heads over the whole
-sequence, all-to-all back): strong scaling.
+sequence, all-to-all back): strong scaling.  --mode ulysses-peer exchanges
+only K and V that way; the attention kernel reads Q tiles from the ranks
+that hold them and stores O rows into the ranks that own them over peer
+memory (CUDA IPC).
 
 --impl reference times the fp64 CPU oracle on the host cores instead, each
 step a bounded sample (query rows) of the same workload.
@@ -217,7 +220,11 @@ def run_reference(args):
 
 
 def run_ulysses(args):
-    """--mode ulysses with N > 1: the multi-GPU form, one rank per GPU."""
+    """--mode ulysses / ulysses-peer: the multi-GPU form, one rank per GPU.
+    ulysses: Q, K and V exchanged by NCCL all-to-alls around the fused
+    attention of the head group, O exchanged back the same way.
+    ulysses-peer: K and V exchanged by NCCL, Q read and O written by the
+    attention kernel itself over peer memory (UlyssesPeerRank)."""
     import datetime
 
     import numpy as np
@@ -258,9 +265,19 @@ def run_ulysses(args):
     stream = torch.cuda.current_stream(dev)
     a2a = sp.nccl_all_to_all()
     out = [None]
+    peer = args.mode == "ulysses-peer"
+    if peer:
+        pr = sp.UlyssesPeerRank(shape, device=dev)
+        pr.q_shard.copy_(dq)                 # Q lives in the exported shard buffer
+        q_in = pr.q_shard
 
-    def step():
-        out[0] = sp.ulysses_attention_distributed(dq, dk, dv, shape, a2a)
+        def step():
+            out[0] = pr.step(dk, dv)
+    else:
+        q_in = dq
+
+        def step():
+            out[0] = sp.ulysses_attention_distributed(dq, dk, dv, shape, a2a)
 
     def timed(fn):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -291,7 +308,7 @@ def run_ulysses(args):
     t_max = max_over_ranks(t_ms, world, dev)
 
     def e2e_step():
-        dq.copy_(hq, non_blocking=True)
+        q_in.copy_(hq, non_blocking=True)
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         step()
@@ -309,7 +326,9 @@ def run_ulysses(args):
                 "ms_per_step": t_max / args.steps, "higher_is_better": True,
                 "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": dict(workload_desc(cfg), P=world, parallelism=f"ulysses{world}",
-                               exchange="NCCL all_to_all_single"),
+                               exchange=("K/V: NCCL all_to_all_single; Q/O: inside the "
+                                         "attention kernel over peer memory (CUDA IPC)")
+                               if peer else "NCCL all_to_all_single"),
                 "e2e": {"value": args.steps * flops / (te * 1e-3) / 1e12, "unit": UNIT,
                         "h2d_bytes_per_step": int(3 * shard_bytes),
                         "d2h_bytes_per_step": int(shard_bytes)},
@@ -320,6 +339,8 @@ def run_ulysses(args):
                              "peak_kind": f"{pkq} bf16 dense (burst)", "traffic": None},
                 "cpu_baseline": None}
         print(json.dumps(line), flush=True)
+    if peer:
+        pr.close()
     dist.barrier()
     dist.destroy_process_group()
     return 0
@@ -532,7 +553,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--mode", choices=["replicas", "ulysses"], default="replicas",
+    ap.add_argument("--mode", choices=["replicas", "ulysses", "ulysses-peer"], default="replicas",
                     help="N > 1 only: independent problems per GPU (default) or one problem "
                          "split across the GPUs with the Ulysses all-to-all")
     ap.add_argument("--config", default="720p")
@@ -548,7 +569,7 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
-    if args.mode == "ulysses":
+    if args.mode in ("ulysses", "ulysses-peer"):
         return run_ulysses(args)
     return run_ours(args)
 

@@ -167,6 +167,63 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
                                       const float *v_scale, void *os, float *lse,
                                       const sp_shape *shape, void *stream);
 
+/* ---------------------------------------------------------------------
+ * Multi-GPU form with the Q and O exchanges fused into the attention kernel.
+ *
+ * "Splitting one generation across four GPUs" (fal.ai, "Generate video with
+ * WAN 2.2 across four GPUs") moves Q, K and V from token shards to head
+ * groups before attention and O back afterwards; the LTX-2 "Multi-GPU
+ * Inference" README (Requirements) names an all2all kernel over CUDA-IPC
+ * peer buffers for it.  In this form each Q tile crosses NVLink once, read by
+ * TMA straight from the rank that holds it, and each O row once, stored by
+ * the epilogue straight into the rank that owns it; only K and V, which every
+ * query tile of a head re-reads, are exchanged into local memory first
+ * (sp_exchange_pack + an all-to-all).
+ */
+
+/* Most ranks the peer step addresses. */
+#define SP_MAX_PEERS 8
+
+/* One rank's attention step: rank `rank` (= j) attends head group j (heads
+ * j*Hl .. j*Hl+Hl-1, Hl = H/P) over the full sequence.
+ * q_shards: HOST array of P device addresses valid in this process (this
+ *   rank's own buffer and the peers' buffers mapped with sp_ipc_open);
+ *   q_shards[r] is rank r's Q shard [B][Nl][H][D] bf16, read only, 16-byte
+ *   aligned.  Token t of the sequence is row t % Nl of rank t / Nl.
+ * k_group, v_group: this rank's received K and V head group
+ *   [P][B][Nl][Hl][D] bf16 (chunk r from rank r), local, read only.
+ * o_shards: HOST array of P device addresses; o_shards[r] is rank r's output
+ *   shard [B][Nl][H][D] bf16; the kernel writes the columns of heads
+ *   j*Hl .. j*Hl+Hl-1 of every row (padding rows as +0.0) and nothing else.
+ * lse: device fp32 [B][Hl][Np] of this head group, or NULL.
+ * shape: the whole problem {B, N, H, D, P}; D must be 128, P <= SP_MAX_PEERS,
+ *   H % P == 0, 0 <= rank < P (else SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE /
+ *   SP_ERR_HEADS_NOT_DIVISIBLE).
+ * Ordering is the caller's: every rank's Q must be complete before the
+ * launch, and rank r may read its O only after every rank's step has
+ * finished (an all-to-all that follows the Q writes, and a collective after
+ * the step, order both).  The kernel ends with a system-scope fence.
+ * Results equal sp_attention_seqsharded's bit for bit. */
+sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_group,
+                                    const void *v_group, void *const *o_shards, float *lse,
+                                    int32_t rank, const sp_shape *shape, void *stream);
+
+/* Bytes of a CUDA IPC memory handle. */
+#define SP_IPC_HANDLE_BYTES 64
+
+/* Exports the device allocation that contains dev_ptr to other processes on
+ * this node: writes its SP_IPC_HANDLE_BYTES-byte handle to handle_out (host)
+ * and the offset of dev_ptr from the allocation's base to *offset_out. */
+sp_status sp_ipc_export(const void *dev_ptr, void *handle_out, int64_t *offset_out);
+
+/* Maps an allocation exported by another process (peer access enabled on
+ * first use); *base_out receives its base address in this process.  Add the
+ * exporter's offset to reach its buffer.  Unmap with sp_ipc_close. */
+sp_status sp_ipc_open(const void *handle, void **base_out);
+
+/* Unmaps an allocation mapped by sp_ipc_open. */
+sp_status sp_ipc_close(void *base);
+
 /* Synchronises `stream`, then returns and clears the device status word:
  * SP_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
  * SP_ERR_CUDA if the stream reports an error, else SP_OK. */

@@ -111,6 +111,33 @@ def test_argument_errors_return_before_launch(lib):
     assert f8(A, A, A, C, C + 2, C, B_) == sp.SP_ERR_ALIGN      # fp32 factors, 4-byte aligned
     assert f8(A, A, A + 8, C, C, C, B_) == sp.SP_ERR_ALIGN
     assert f8(A, A, A, C, C, C, B_, shp=sp.Shape(1, 1024, 4, 64, 2)) == sp.SP_ERR_UNSUPPORTED_D
+    # the peer step: host arrays of P device addresses, D = 128, P <= 8
+    def peer(qs, k, v, os_, rank, shp):
+        arr = lambda xs: None if xs is None else (ctypes.c_void_p * len(xs))(*xs)
+        return lib.sp_attention_ulysses_peer(arr(qs), ctypes.c_void_p(k) if k else None,
+                                             ctypes.c_void_p(v) if v else None, arr(os_), None,
+                                             rank, ctypes.byref(shp.c()), None)
+    s4 = sp.Shape(1, 1000, 8, 128, 4)
+    ok_q, ok_o = [A + 0x1000 * r for r in range(4)], [B_ + 0x1000 * r for r in range(4)]
+    assert peer(None, A, A, ok_o, 0, s4) == sp.SP_ERR_NULL
+    assert peer(ok_q, A, 0, ok_o, 0, s4) == sp.SP_ERR_NULL
+    assert peer(ok_q[:3] + [0], A, A, ok_o, 0, s4) == sp.SP_ERR_NULL
+    assert peer(ok_q, A, A, ok_o[:3] + [B_ + 8], 0, s4) == sp.SP_ERR_ALIGN
+    assert peer(ok_q, A, A + 2, ok_o, 0, s4) == sp.SP_ERR_ALIGN
+    assert peer(ok_q, A, A, ok_o, 4, s4) == sp.SP_ERR_SHAPE
+    assert peer(ok_q, A, A, ok_o, -1, s4) == sp.SP_ERR_SHAPE
+    assert peer(ok_q, A, A, ok_o, 0, sp.Shape(1, 1000, 8, 64, 4)) == sp.SP_ERR_UNSUPPORTED_D
+    assert peer(ok_q, A, A, ok_o, 0, sp.Shape(1, 1000, 6, 128, 4)) == \
+        sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    assert peer(ok_q * 4, A, A, ok_o * 4, 0, sp.Shape(1, 1000, 16, 128, 16)) == sp.SP_ERR_SHAPE
+    h = (ctypes.c_uint8 * sp.IPC_HANDLE_BYTES)()
+    off = ctypes.c_int64()
+    base = ctypes.c_void_p()
+    assert lib.sp_ipc_export(None, h, ctypes.byref(off)) == sp.SP_ERR_NULL
+    assert lib.sp_ipc_export(ctypes.c_void_p(A), None, ctypes.byref(off)) == sp.SP_ERR_NULL
+    assert lib.sp_ipc_open(None, ctypes.byref(base)) == sp.SP_ERR_NULL
+    assert lib.sp_ipc_open(h, None) == sp.SP_ERR_NULL
+    assert lib.sp_ipc_close(None) == sp.SP_ERR_NULL
     for fn in (lib.sp_exchange_pack, lib.sp_exchange_unpack):
         assert _call(fn, 0, B_, shape=shape) == sp.SP_ERR_NULL
         assert _call(fn, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN

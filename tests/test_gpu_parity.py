@@ -192,6 +192,123 @@ def test_multi_gpu_form_on_virtual_ranks(B, N, H, D, P):
     _check_rows(got, q, k, v, rows, P, f"virtual ranks B={B} N={N} P={P}")
 
 
+def _peer_steps_on_virtual_ranks(q, k, v, P, ranks=None, lse=False):
+    """The fused multi-GPU form with P virtual ranks on one GPU: every rank's
+    Q shard and O shard is its own allocation (standing in for a peer's
+    memory), K and V go through exchange pack + an all-to-all done as copies,
+    and each rank's peer step reads every Q shard and writes every O shard.
+    The launches run one after another; none waits on another."""
+    B, N, H, D = q.shape
+    shape = sp.Shape(B, N, H, D, P)
+    shards = [to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v)]
+    q_list = [shards[0][r].clone() for r in range(P)]
+    o_list = [torch.full(shape.rank_shard, float("nan"), dtype=torch.bfloat16, device="cuda")
+              for _ in range(P)]
+    groups = []
+    for t in (1, 2):
+        sends = []
+        for r in range(P):
+            send = torch.empty(shape.send_chunks, dtype=torch.bfloat16, device="cuda")
+            sp.exchange_pack(shards[t][r], send, shape)
+            sends.append(send)
+        groups.append([torch.stack([sends[r][j] for r in range(P)]).contiguous()
+                       for j in range(P)])
+    lses = {}
+    for j in (range(P) if ranks is None else ranks):
+        l = (torch.full((B, shape.Hl, shape.Np), float("nan"), dtype=torch.float32,
+                        device="cuda") if lse else None)
+        sp.attention_ulysses_peer(q_list, groups[0][j], groups[1][j], o_list, shape, j, lse=l)
+        if lse:
+            lses[j] = l.cpu().numpy()
+    _status_ok()
+    return to_host(torch.stack(o_list)), lses
+
+
+@pytest.mark.parametrize("B,N,H,P", [(1, 1000, 8, 4), (1, 4096, 8, 2), (2, 777, 6, 3),
+                                     (1, 512, 6, 3), (3, 300, 16, 8), (1, 2048, 40, 8)])
+def test_fused_peer_exchange_on_virtual_ranks(B, N, H, P):
+    """Q tiles read from the rank that holds them (TMA inside a shard, a row
+    gather across shards), O rows stored into the rank that owns them: the
+    result equals the one-GPU fused call bit for bit, padding rows included,
+    and so does the LSE of every head group."""
+    D = 128
+    q, k, v = _random_logical(B, N, H, D, seed=11 * N + P)
+    got, lses = _peer_steps_on_virtual_ranks(q, k, v, P, lse=True)
+    one, lse1 = _run_fused(q, k, v, P, lse=True)
+    assert np.array_equal(got.reshape(one.shape), one)
+    Hl = H // P
+    for j, l in lses.items():
+        assert np.array_equal(l, lse1[:, j * Hl:(j + 1) * Hl], equal_nan=True)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H)
+                     for i in sorted({0, N - 1, *range(0, N, max(1, N // 16))})], dtype=np.int64)
+    _check_rows(got, q, k, v, rows, P, f"peer step B={B} N={N} P={P}")
+
+
+def test_peer_step_writes_only_its_head_group():
+    B, N, H, D, P = 1, 1000, 8, 128, 4
+    q, k, v = _random_logical(B, N, H, D, seed=21)
+    got, _ = _peer_steps_on_virtual_ranks(q, k, v, P, ranks=[1])
+    Hl = H // P
+    g = synth.bf16_to_f32(got)                       # [P][B][Nl][H][D]
+    assert np.all(np.isfinite(g[:, :, :, Hl:2 * Hl]))
+    rest = np.concatenate([g[:, :, :, :Hl], g[:, :, :, 2 * Hl:]], axis=3)
+    assert np.all(np.isnan(rest))
+
+
+def _ipc_child(handle, offset, n, q):
+    """Maps the parent's allocation through CUDA IPC and copies the exported
+    buffer out with a degree-1 pack (a plain copy through the C ABI)."""
+    import ctypes
+
+    import torch
+
+    import video_dit_sequence_b200 as sp
+    torch.cuda.set_device(0)
+    base = sp.ipc_open(handle)
+    shape = sp.Shape(1, n, 8, 128, 1)
+    dst = torch.empty(shape.head_sharded, dtype=torch.bfloat16, device="cuda")
+    s = shape.c()
+    st = sp.load().sp_pack(ctypes.c_void_p(base + offset), ctypes.c_void_p(dst.data_ptr()),
+                           ctypes.byref(s), None)
+    torch.cuda.synchronize()
+    q.put((st, dst.view(torch.int16).cpu().numpy()))
+    sp.ipc_close(base)
+
+
+def test_ipc_export_open_across_processes():
+    """A buffer inside a larger allocation (non-zero offset) is exported,
+    mapped by a second process on the same GPU and read back exactly."""
+    import torch.multiprocessing as mp
+    n = 1000
+    big = torch.randn(3 * n * 8 * 128 + 64, device="cuda").to(torch.bfloat16)
+    x = big[64:64 + n * 8 * 128]
+    handle, offset = sp.ipc_export(x)
+    assert len(handle) == sp.IPC_HANDLE_BYTES and offset >= 128
+    torch.cuda.synchronize()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    proc = ctx.Process(target=_ipc_child, args=(handle, offset, n, q))
+    proc.start()
+    st, got = q.get(timeout=120)
+    proc.join(60)
+    assert proc.exitcode == 0 and st == sp.SP_OK
+    assert np.array_equal(got.reshape(-1), x.view(torch.int16).cpu().numpy())
+
+
+def test_padding_rows_past_the_last_full_tile_pair():
+    """N = 512, P = 3: Np = 513, so the one padding row lies past the last
+    256-row CTA tile of the true tokens; both attention calls must still
+    write it as +0.0."""
+    B, N, H, D, P = 1, 512, 6, 128, 3
+    q, k, v = _random_logical(B, N, H, D, seed=23)
+    fused, _ = _run_fused(q, k, v, P)
+    unfused, _ = _run_unfused(q, k, v, P)
+    for out in (fused, unfused):
+        pad = out.reshape(P, B, -1, H, D)[P - 1, :, -1]
+        assert np.all(pad == 0)
+    assert np.array_equal(fused, unfused)
+
+
 # ------------------------------------------------------------------ attention, small
 
 def test_tiny_config_every_row():

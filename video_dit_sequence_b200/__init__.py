@@ -41,7 +41,8 @@ SP_ERR_TIMEOUT = 7
 EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_attention", "sp_attention_seqsharded", "sp_device_status",
             "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout",
-            "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded")
+            "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded",
+            "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close")
 
 
 class sp_shape(ctypes.Structure):
@@ -82,6 +83,15 @@ def load(path: str = LIB_PATH):
         f.restype = ctypes.c_int
     lib.sp_attention_fp8_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sp_p, vp]
     lib.sp_attention_fp8_seqsharded.restype = ctypes.c_int
+    lib.sp_attention_ulysses_peer.argtypes = [
+        ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), vp, ctypes.c_int32, sp_p, vp]
+    lib.sp_attention_ulysses_peer.restype = ctypes.c_int
+    lib.sp_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int64)]
+    lib.sp_ipc_export.restype = ctypes.c_int
+    lib.sp_ipc_open.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.sp_ipc_open.restype = ctypes.c_int
+    lib.sp_ipc_close.argtypes = [vp]
+    lib.sp_ipc_close.restype = ctypes.c_int
     lib.sp_device_status.argtypes = [vp]
     lib.sp_device_status.restype = ctypes.c_int
     lib.sp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
@@ -352,6 +362,172 @@ class UlyssesRank:
         out = torch.empty(self.shape.rank_shard, dtype=back.dtype, device=back.device)
         exchange_unpack(back, out, self.shape, stream)
         return out
+
+
+MAX_PEERS = 8            # SP_MAX_PEERS
+IPC_HANDLE_BYTES = 64    # SP_IPC_HANDLE_BYTES
+
+
+def attention_ulysses_peer(q_shards, k_group, v_group, o_shards, shape: Shape, rank: int,
+                           lse=None, stream=None):
+    """One rank's step of the multi-GPU form with the Q and O exchanges fused
+    into the kernel (sp_attention_ulysses_peer).  q_shards / o_shards: P
+    entries in rank order, each a CUDA tensor [B][Nl][H][D] bf16 or an int
+    device address valid in this process (a peer buffer from ipc_open).
+    k_group / v_group: this rank's received head group [P][B][Nl][Hl][D];
+    lse: [B][Hl][Np] float32 or None."""
+    torch = _torch()
+    P = shape.P
+    if len(q_shards) != P or len(o_shards) != P:
+        raise ValueError(f"need {P} Q and {P} O shard addresses")
+    local = [x for x in (*q_shards, *o_shards) if not isinstance(x, int)]
+
+    def addr(x, name):
+        return x if isinstance(x, int) else _ptr(x, shape.rank_shard, name).value
+
+    qa = (ctypes.c_void_p * P)(*[addr(x, f"q_shards[{r}]") for r, x in enumerate(q_shards)])
+    oa = (ctypes.c_void_p * P)(*[addr(x, f"o_shards[{r}]") for r, x in enumerate(o_shards)])
+    s = shape.c()
+    group = shape.send_chunks
+    with _same_device(k_group, v_group, lse, *local):
+        _check(load().sp_attention_ulysses_peer(
+            qa, _ptr(k_group, group, "k_group"), _ptr(v_group, group, "v_group"), oa,
+            _ptr(lse, (shape.B, shape.Hl, shape.Np), "lse", torch.float32), int(rank),
+            ctypes.byref(s), _stream(stream, k_group.device)), "sp_attention_ulysses_peer")
+
+
+def ipc_export(t):
+    """(handle, offset): the CUDA IPC handle (bytes) of the allocation that
+    holds CUDA tensor t, and t's byte offset from that allocation's base."""
+    torch = _torch()
+    h = (ctypes.c_uint8 * IPC_HANDLE_BYTES)()
+    off = ctypes.c_int64()
+    with torch.cuda.device(t.device):
+        _check(load().sp_ipc_export(ctypes.c_void_p(t.data_ptr()), h, ctypes.byref(off)),
+               "sp_ipc_export")
+    return bytes(h), off.value
+
+
+def ipc_open(handle: bytes) -> int:
+    """Maps another process's exported allocation on the current device;
+    returns its base address in this process (unmap with ipc_close)."""
+    buf = (ctypes.c_uint8 * IPC_HANDLE_BYTES).from_buffer_copy(handle)
+    base = ctypes.c_void_p()
+    _check(load().sp_ipc_open(buf, ctypes.byref(base)), "sp_ipc_open")
+    return int(base.value)
+
+
+def ipc_close(base: int):
+    _check(load().sp_ipc_close(ctypes.c_void_p(base)), "sp_ipc_close")
+
+
+class CudaPeerBackend:
+    """Memory and kernels of UlyssesPeerRank on a GPU: buffers from torch's
+    allocator, peers' buffers mapped through CUDA IPC (each allocation once),
+    the exchange reorder and the peer step of this library."""
+
+    def __init__(self, device):
+        torch = _torch()
+        self.device = torch.device(device)
+        self._opened = {}
+
+    def empty(self, shape, dtype=None):
+        torch = _torch()
+        return torch.empty(shape, dtype=dtype or torch.bfloat16, device=self.device)
+
+    def export(self, t):
+        return ipc_export(t)
+
+    def open(self, handle: bytes, offset: int):
+        torch = _torch()
+        if handle not in self._opened:
+            with torch.cuda.device(self.device):
+                self._opened[handle] = ipc_open(handle)
+        return self._opened[handle] + offset
+
+    def exchange_pack(self, x, send, shape: Shape):
+        exchange_pack(x, send, shape)
+
+    def peer_step(self, q_addrs, k_group, v_group, o_addrs, rank: int, shape: Shape):
+        attention_ulysses_peer(q_addrs, k_group, v_group, o_addrs, shape, rank)
+
+    def close(self):
+        torch = _torch()
+        with torch.cuda.device(self.device):
+            for base in self._opened.values():
+                ipc_close(base)
+        self._opened.clear()
+
+
+class UlyssesPeerRank:
+    """One rank of the multi-GPU form with the Q and O exchanges fused into
+    the attention kernel.
+
+    Construction allocates this rank's Q shard and output shard
+    ([B][Nl][H][D] each), exports both, gathers every rank's exports over the
+    process group and maps the peers' buffers, so that every rank holds the
+    P Q-shard and P O-shard addresses in rank order.  step(k, v, q) then
+      writes q into the Q shard (or the caller wrote it),
+      reorders k and v into send chunks (sp_exchange_pack) and exchanges
+        them (all-to-all: chunk j of every rank to rank j),
+      runs the peer step (Q tiles read from the ranks that hold them, O rows
+        stored into the ranks that own them),
+      and ends with a one-element all-reduce.
+    The all-to-all follows every rank's Q write in that rank's stream order,
+    so when it completes here every Q shard is complete; the closing
+    all-reduce follows every rank's kernel, so when it completes here every
+    row of this rank's output shard has been written.  The returned output
+    shard stays valid until the next step."""
+
+    def __init__(self, shape: Shape, group=None, backend=None, device=None):
+        import torch.distributed as dist
+        torch = _torch()
+        self.shape, self.group = shape, group
+        self.rank = dist.get_rank(group)
+        if dist.get_world_size(group) != shape.P:
+            raise ValueError(f"group of {dist.get_world_size(group)} ranks, shape has P = {shape.P}")
+        if shape.P > MAX_PEERS:
+            raise ValueError(f"P = {shape.P} > {MAX_PEERS}")
+        if backend is None:
+            backend = CudaPeerBackend(device if device is not None else torch.cuda.current_device())
+        self.backend = be = backend
+        self.q_shard = be.empty(shape.rank_shard)
+        self.o_shard = be.empty(shape.rank_shard)
+        self._k_send, self._v_send, self._k_recv, self._v_recv = (
+            be.empty(shape.send_chunks) for _ in range(4))
+        self._flag = be.empty((1,), torch.float32)
+        table = [None] * shape.P
+        dist.all_gather_object(table, (be.export(self.q_shard), be.export(self.o_shard)),
+                               group=group)
+        self.q_addrs, self.o_addrs = [], []
+        for r, (qx, ox) in enumerate(table):
+            if r == self.rank:
+                self.q_addrs.append(self.q_shard)
+                self.o_addrs.append(self.o_shard)
+            else:
+                self.q_addrs.append(be.open(*qx))
+                self.o_addrs.append(be.open(*ox))
+
+    def step(self, k, v, q=None):
+        import torch.distributed as dist
+        be, s = self.backend, self.shape
+        if q is not None:
+            self.q_shard.copy_(q)
+        be.exchange_pack(k, self._k_send, s)
+        be.exchange_pack(v, self._v_send, s)
+        dist.all_to_all_single(self._k_recv, self._k_send, group=self.group)
+        dist.all_to_all_single(self._v_recv, self._v_send, group=self.group)
+        be.peer_step(self.q_addrs, self._k_recv, self._v_recv, self.o_addrs, self.rank, s)
+        self._flag.zero_()
+        dist.all_reduce(self._flag, group=self.group)
+        return self.o_shard
+
+    def close(self):
+        """Unmaps the peers' buffers; returns once every rank has done so, so
+        that no rank frees a buffer another rank still maps."""
+        import torch.distributed as dist
+        self.backend.close()
+        dist.barrier(group=self.group)
 
 
 def nccl_all_to_all(group=None):

@@ -67,6 +67,22 @@ struct AttnParams {
 
 constexpr int32_t kStatusTimeout = 7;
 
+// One rank's step of the multi-GPU form with the Q and O exchanges fused
+// into the kernel: rank r's sequence shard of Q and its output shard O are
+// [B][Nl][H][D] bf16 on GPU r, reached through peer addresses.  Query token
+// t of the head group lives in rank t / nl at local row t % nl; this rank
+// attends heads head0 .. head0 + Hl - 1 of the H global heads.
+constexpr int kMaxPeers = 8;
+struct PeerArgs {
+  CUtensorMap q[kMaxPeers];            // 4-D maps (D, H, Nl, B) over each rank's Q shard
+  const uint8_t *q_ptr[kMaxPeers];     // the same shards, for tiles that cross ranks
+  __nv_bfloat16 *o_ptr[kMaxPeers];     // each rank's output shard
+  int32_t nranks;                      // P
+  int32_t nl;                          // tokens per rank
+  int32_t heads;                       // H, global heads of a shard row
+  int32_t head0;                       // first global head of this rank's group
+};
+
 // kF8: operands in E4M3 (one byte) instead of bf16 (two bytes).
 template <int D, bool kF8 = false>
 struct AttnCfg {
@@ -108,11 +124,13 @@ struct AttnCfg {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 
-template <int D, bool kF8 = false>
-__global__ void __launch_bounds__(320, 1)
-attention_kernel(const __grid_constant__ CUtensorMap tmQ,
-                 const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+// The kernel body.  kPeer: Q tiles come from the ranks' shards through
+// `peer` (tmQ unused) and O rows go to the ranks' output shards; K and V are
+// this rank's received head group, addressed as for the fused call.
+template <int D, bool kF8, bool kPeer>
+__device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUtensorMap *tmK,
+                                               const CUtensorMap *tmV, const AttnParams &p,
+                                               const PeerArgs *peer) {
   using C = AttnCfg<D, kF8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -173,9 +191,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint64_t pol_q = policy_evict_first();
     const uint64_t pol_kv = policy_evict_last();
     if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
+      if (!kPeer) prefetch_tmap(tmQ);
+      prefetch_tmap(tmK);
+      prefetch_tmap(tmV);
     }
     const int nl = p.nl_split;
     auto tma_ok = [&](int t0) {
@@ -211,19 +229,58 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
       fence_proxy_async_smem();
     };
+    // Peer Q: a tile inside one rank's shard is one TMA box per column block
+    // from that rank's map; a tile that crosses ranks is gathered row by row.
+    auto peer_q_ok = [&](int t0) {
+      const int r0 = t0 / peer->nl;
+      return r0 < peer->nranks && t0 - r0 * peer->nl + C::kBM <= peer->nl;
+    };
+    auto copy_q_peer = [&](uint32_t dst, int t0) {
+      constexpr int kChunks = C::kRowBytes / 16;
+      const int pnl = peer->nl;
+      for (int idx = lane; idx < C::kBM * kChunks; idx += 32) {
+        const int r = idx / kChunks, cc = idx % kChunks;
+        const int tok = t0 + r;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (tok < p.N) {
+          const int rk = tok / pnl, n = tok - rk * pnl;
+          const int64_t off = ((static_cast<int64_t>(b) * pnl + n) * peer->heads +
+                               peer->head0 + hg) * C::kRowBytes + cc * 16;
+          val = ld_global_v4(peer->q_ptr[rk] + off);
+        }
+        st_shared_v4(dst + (cc >> 3) * C::kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4), val);
+      }
+      fence_proxy_async_smem();
+    };
     // Q: both tiles complete one barrier.
     uint32_t q_tx = 0;
     for (int t = 0; t < 2; ++t) {
       const uint32_t dst = sbase + C::kOffQ + t * C::kTileBytes;
-      if (tma_ok(q0 + t * C::kBM)) q_tx += C::kTileBytes;
-      else copy_tile(p.q, dst, q0 + t * C::kBM);
+      if (kPeer) {
+        if (peer_q_ok(q0 + t * C::kBM)) q_tx += C::kTileBytes;
+        else copy_q_peer(dst, q0 + t * C::kBM);
+      } else {
+        if (tma_ok(q0 + t * C::kBM)) q_tx += C::kTileBytes;
+        else copy_tile(p.q, dst, q0 + t * C::kBM);
+      }
     }
     __syncwarp();
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, q_tx);
-      for (int t = 0; t < 2; ++t)
-        if (tma_ok(q0 + t * C::kBM))
-          tma_tile(&tmQ, sbase + C::kOffQ + t * C::kTileBytes, bar_q, q0 + t * C::kBM, pol_q);
+      for (int t = 0; t < 2; ++t) {
+        const int t0 = q0 + t * C::kBM;
+        const uint32_t dst = sbase + C::kOffQ + t * C::kTileBytes;
+        if (kPeer) {
+          if (peer_q_ok(t0)) {
+            const int r0 = t0 / peer->nl;
+            for (int h = 0; h < C::kHalves; ++h)
+              tma_load_4d(dst + h * C::kBlockBytes, &peer->q[r0], bar_q, h * C::kBoxInner,
+                          peer->head0 + hg, t0 - r0 * peer->nl, b, pol_q);
+          }
+        } else if (tma_ok(t0)) {
+          tma_tile(tmQ, dst, bar_q, t0, pol_q);
+        }
+      }
     }
     int it = 0;
     for (int j = 0; j < T && ok; ++j) {
@@ -240,7 +297,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (tma_ok(j * C::kBN)) {
           if (lane == 0) {
             mbar_arrive_expect_tx(bar, C::kTileBytes);
-            tma_tile(kv == 0 ? &tmK : &tmV, dst, bar, j * C::kBN, pol_kv);
+            tma_tile(kv == 0 ? tmK : tmV, dst, bar, j * C::kBN, pol_kv);
           }
         } else {
           copy_tile(kv == 0 ? p.k : p.v, dst, j * C::kBN);
@@ -473,14 +530,22 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
       const float inv_l = valid ? 1.0f / l : 0.0f;
       const float *dv_row = kF8 ? p.dv + static_cast<int64_t>(bh) * D : nullptr;
       int64_t row_off;
-      if (p.nl_split) {
+      __nv_bfloat16 *obase = p.o;
+      int ohead = map_head;
+      if (kPeer) {
+        // this row belongs to rank token / nl; O goes straight to its shard
+        const int rk = token / peer->nl, n = token - rk * peer->nl;
+        obase = peer->o_ptr[rk < peer->nranks ? rk : 0];  // rows past Np are not stored
+        row_off = (static_cast<int64_t>(b) * peer->nl + n) * peer->heads * D;
+        ohead = peer->head0 + hg;
+      } else if (p.nl_split) {
         const int rk = token / p.nl_split, n = token - rk * p.nl_split;
         row_off = static_cast<int64_t>(rk) * p.o_rank + static_cast<int64_t>(b) * p.o_batch +
                   static_cast<int64_t>(n) * p.o_row;
       } else {
         row_off = static_cast<int64_t>(map_batch) * p.o_batch + static_cast<int64_t>(token) * p.o_row;
       }
-      __nv_bfloat16 *dst = p.o + row_off + static_cast<int64_t>(map_head) * D;
+      __nv_bfloat16 *dst = obase + row_off + static_cast<int64_t>(ohead) * D;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
@@ -516,6 +581,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
   }
 
   // ------------------------------------------------------------------ teardown
+  // Peer stores are ordered before whatever the host sequences after the
+  // kernel (the end-of-step collective that lets the owners read O).
+  if (kPeer) __threadfence_system();
   if (!ok) {
     *abort_flag = 1;
     atomicExch(p.status, kStatusTimeout);
@@ -533,6 +601,24 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+template <int D, bool kF8 = false>
+__global__ void __launch_bounds__(320, 1)
+attention_kernel(const __grid_constant__ CUtensorMap tmQ,
+                 const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
+  attention_body<D, kF8, false>(&tmQ, &tmK, &tmV, p, nullptr);
+}
+
+// One rank's step of the multi-GPU form (bf16, D = 128): Q read from every
+// rank's shard and O written to every rank's output shard over peer
+// addresses; K and V from this rank's received head group.
+__global__ void __launch_bounds__(320, 1)
+attention_peer_kernel(const __grid_constant__ PeerArgs peer,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
+  attention_body<128, false, true>(nullptr, &tmK, &tmV, p, &peer);
 }
 
 }  // namespace sp

@@ -121,6 +121,15 @@ __device__ __forceinline__ uint4 ld_global_nc_v4(const void *p) {
   return v;
 }
 
+// Coherent 16-byte load (peer memory of another GPU included).
+__device__ __forceinline__ uint4 ld_global_v4(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4 &v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
                ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)

@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "attention.cuh"
@@ -165,6 +166,23 @@ bool make_map5(CUtensorMap *m, const void *base, int D, int H, int Nl, int B, in
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over one rank's sequence shard [B][Nl][H][D] bf16, dims inner
+// to outer (D, H, Nl, B): the Q source of the peer step.
+bool make_map_shard(CUtensorMap *m, const void *base, int D, int H, int Nl, int B) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(H) * D * 2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(Nl), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, row, row * Nl};
+  cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(Nl < 128 ? Nl : 128), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, bool kF8 = false>
 cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
                              const sp::AttnParams &p, int B, cudaStream_t cs) {
@@ -183,9 +201,26 @@ cudaError_t launch_attention(const CUtensorMap &q, const CUtensorMap &k, const C
       attr_set[dev] = true;
     }
   }
-  dim3 grid((p.N + 2 * C::kBM - 1) / (2 * C::kBM), p.H, B);
+  // every output row up to Np, padding rows included, belongs to some CTA
+  dim3 grid((p.Np + 2 * C::kBM - 1) / (2 * C::kBM), p.H, B);
   sp::attention_kernel<D, kF8><<<grid, C::kThreads, C::kSmemBytes, cs>>>(q, k, v, p);
   return cudaGetLastError();
+}
+
+// Sets the kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel kernel, int bytes, bool (&done)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> g(g_mu);
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
 }
 
 // Shared launch path.  The head-sharded and the sequence-sharded layouts are
@@ -272,6 +307,97 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   return launch_status(e);
 }
 
+// One rank's step of the multi-GPU form with the Q and O exchanges fused
+// into the attention kernel (see sp_attention_ulysses_peer in sp.h).
+sp_status attention_peer(const void *const *q_shards, const void *k_group, const void *v_group,
+                         void *const *o_shards, float *lse, int32_t rank, const sp_shape *s,
+                         void *stream) {
+  sp_status st = check_common(s, true);
+  if (st != SP_OK) return st;
+  if (s->D != 128) return SP_ERR_UNSUPPORTED_D;
+  if (s->P > sp::kMaxPeers || rank < 0 || rank >= s->P) return SP_ERR_SHAPE;
+  if (q_shards == nullptr || o_shards == nullptr || k_group == nullptr || v_group == nullptr)
+    return SP_ERR_NULL;
+  const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
+  for (int r = 0; r < P; ++r) {
+    if (q_shards[r] == nullptr || o_shards[r] == nullptr) return SP_ERR_NULL;
+    if (!aligned16(q_shards[r]) || !aligned16(o_shards[r])) return SP_ERR_ALIGN;
+  }
+  if (!aligned16(k_group) || !aligned16(v_group) ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
+    return SP_ERR_ALIGN;
+  const int Hl = H / P;
+  const int Nl = (N + P - 1) / P;
+  const int Np = Nl * P;
+  int32_t *status = status_ptr();
+  if (status == nullptr) return SP_ERR_CUDA;
+  sp::PeerArgs pa;
+  std::memset(&pa, 0, sizeof(pa));
+  for (int r = 0; r < P; ++r) {
+    if (!make_map_shard(&pa.q[r], q_shards[r], D, H, Nl, B)) return SP_ERR_CUDA;
+    pa.q_ptr[r] = static_cast<const uint8_t *>(q_shards[r]);
+    pa.o_ptr[r] = static_cast<__nv_bfloat16 *>(o_shards[r]);
+  }
+  pa.nranks = P;
+  pa.nl = Nl;
+  pa.heads = H;
+  pa.head0 = rank * Hl;
+  // K and V: this rank's received head group [P][B][Nl][Hl][D], addressed
+  // as the fused call addresses a sequence-sharded tensor with Hl heads.
+  const bool rank_major = B > 1 && P > 1;
+  CUtensorMap mk, mv;
+  if (rank_major) {
+    if (!make_map5(&mk, k_group, D, Hl, Nl, B, P) || !make_map5(&mv, v_group, D, Hl, Nl, B, P))
+      return SP_ERR_CUDA;
+  } else {
+    const int64_t row_el = static_cast<int64_t>(Hl) * D;
+    const int64_t batch_el = static_cast<int64_t>(Nl) * Hl * D;
+    if (!make_map(&mk, k_group, D, Hl, N, B, row_el, batch_el) ||
+        !make_map(&mv, v_group, D, Hl, N, B, row_el, batch_el))
+      return SP_ERR_CUDA;
+  }
+  sp::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.N = N;
+  p.Np = Np;
+  p.H = Hl;
+  p.B = B;
+  p.hsplit = Hl;
+  p.num_kv_tiles = (N + 127) / 128;
+  const float scale = s->scale > 0.f ? s->scale : 1.0f / std::sqrt(static_cast<float>(D));
+  p.scale_log2e = scale * 1.4426950408889634f;
+  p.lse = lse;
+  p.status = status;
+  p.nl_split = rank_major ? Nl : 0;
+  p.k = static_cast<const uint8_t *>(k_group);
+  p.v = static_cast<const uint8_t *>(v_group);
+  p.nblk = p.num_kv_tiles;
+  using C = sp::AttnCfg<128>;
+  static bool attr_set[kMaxDevices] = {};
+  cudaError_t e = set_smem_once(sp::attention_peer_kernel, C::kSmemBytes, attr_set);
+  if (e != cudaSuccess) return SP_ERR_CUDA;
+  dim3 grid((Np + 2 * C::kBM - 1) / (2 * C::kBM), Hl, B);
+  sp::attention_peer_kernel<<<grid, C::kThreads, C::kSmemBytes,
+                              static_cast<cudaStream_t>(stream)>>>(pa, mk, mv, p);
+  return launch_status(cudaGetLastError());
+}
+
+using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+AddressRangeFn address_range_fn() {
+  static AddressRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(p);
+  });
+  return fn;
+}
+
 __global__ void wait_timeout_kernel(uint64_t limit_ns, int32_t *status) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
@@ -339,6 +465,42 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
                                       const sp_shape *shape, void *stream) {
   if (q_scale == nullptr || k_scale == nullptr || v_scale == nullptr) return SP_ERR_NULL;
   return attention(qs, ks, vs, os, lse, shape, stream, true, q_scale, k_scale, v_scale);
+}
+
+sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_group,
+                                    const void *v_group, void *const *o_shards, float *lse,
+                                    int32_t rank, const sp_shape *shape, void *stream) {
+  return attention_peer(q_shards, k_group, v_group, o_shards, lse, rank, shape, stream);
+}
+
+sp_status sp_ipc_export(const void *dev_ptr, void *handle_out, int64_t *offset_out) {
+  if (dev_ptr == nullptr || handle_out == nullptr || offset_out == nullptr) return SP_ERR_NULL;
+  AddressRangeFn range = address_range_fn();
+  if (range == nullptr) return SP_ERR_CUDA;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return SP_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) return SP_ERR_CUDA;
+  static_assert(sizeof(h) == SP_IPC_HANDLE_BYTES, "CUDA IPC handle size");
+  std::memcpy(handle_out, &h, sizeof(h));
+  *offset_out = static_cast<int64_t>(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return SP_OK;
+}
+
+sp_status sp_ipc_open(const void *handle, void **base_out) {
+  if (handle == nullptr || base_out == nullptr) return SP_ERR_NULL;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  if (cudaIpcOpenMemHandle(base_out, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+    return SP_ERR_CUDA;
+  return SP_OK;
+}
+
+sp_status sp_ipc_close(void *base) {
+  if (base == nullptr) return SP_ERR_NULL;
+  return cudaIpcCloseMemHandle(base) == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
 
 sp_status sp_device_status(void *stream) {
