@@ -11,7 +11,10 @@
  * numerically the single-GPU result (LTX-2 "Multi-GPU Inference" README,
  * Capabilities table).  On one GPU the exchange is a permutation in HBM
  * (sp_pack / sp_unpack) or disappears into the attention kernel's addressing
- * (sp_attention_seqsharded).
+ * (sp_attention_seqsharded).  With one GPU per rank, sp_exchange_pack /
+ * sp_exchange_unpack reorder a rank's shard around an all-to-all, and
+ * sp_attention_ulysses_peer moves the Q and O exchanges into the attention
+ * kernel over peer memory.
  *
  * Notation: B batch, N true token count, H heads, D head dim, P degree,
  * Hl = H/P, Nl = ceil(N/P), Np = P*Nl.  Elements are bf16 (16-bit words).

@@ -31,6 +31,11 @@
 // a row depends only on its own scores and the fixed key-tile order, never on
 // P, the layout, or the CTA it runs in: outputs are bit-identical across
 // degrees and between the fused and the three-call path.
+//
+// One body serves three kernels: bf16 (D = 64 or 128), E4M3 operands with
+// per-block / per-channel scale factors (kF8), and one rank's step of the
+// multi-GPU form (kPeer), which reads Q tiles from, and stores O rows into,
+// the shards of the ranks that hold those tokens.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
