@@ -60,7 +60,7 @@ def peaks():
 
 
 KERNEL_SOURCES = ("video_dit_sequence_b200/csrc/attention.cuh", "video_dit_sequence_b200/csrc/sm100.cuh")
-TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "attention_kernel_dram_traffic.md")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "attention_kernel_dram_traffic.txt")
 
 
 def kernel_source_sha() -> str:
@@ -96,7 +96,7 @@ def recorded_traffic(cfg):
 
 def max_over_ranks(value: float, world: int, device=None) -> float:
     """The slowest rank's time: an all-reduce MAX over the default process
-    group (NCCL on the GPU machine, gloo in the CPU tests)."""
+    group (NCCL on GPUs, gloo in the CPU tests)."""
     if world <= 1:
         return value
     import torch
