@@ -65,6 +65,11 @@ def test_shape_errors(lib):
     assert sp.check_shape(sp.Shape(1, 10, 40, 96, 4)) == sp.SP_ERR_UNSUPPORTED_D
     assert sp.check_shape(sp.Shape(1, 10, 40, 64, 3)) == sp.SP_ERR_HEADS_NOT_DIVISIBLE
     assert lib.sp_check_shape(None) == sp.SP_ERR_NULL
+    # largest problem: a tensor's 16-byte vectors are indexed below 2^31
+    assert sp.check_shape(sp.Shape(1, 2 ** 21 - 1, 64, 128, 1)) == sp.SP_OK
+    assert sp.check_shape(sp.Shape(1, 2 ** 21, 64, 128, 1)) == sp.SP_ERR_SHAPE
+    assert sp.check_shape(sp.Shape(1, 2 ** 21 - 7, 64, 128, 8)) == sp.SP_ERR_SHAPE  # padded
+    assert sp.check_shape(sp.Shape(65536, 16, 8, 64, 1)) == sp.SP_ERR_SHAPE
     for code in range(8):
         assert isinstance(sp.status_str(code), str) and sp.status_str(code)
 

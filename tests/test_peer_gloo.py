@@ -65,15 +65,19 @@ def _peer_rank_main(rank, world, port, q, shape_args):
             return t
 
         def export(self, t):
-            return self.own[t.data_ptr()].name, 0
+            return self.own[t.data_ptr()].name, 0   # the whole block
 
         def open(self, name, offset):
             assert offset == 0
             shm = shared_memory.SharedMemory(name=name)
             resource_tracker.unregister(shm._name, "shared_memory")  # the owner unlinks it
             self.maps.append(shm)
-            return torch.frombuffer(shm.buf, dtype=torch.bfloat16,
-                                    count=math.prod(self.shape.rank_shard)).view(self.shape.rank_shard)
+            shp = (2,) + tuple(self.shape.rank_shard)
+            return torch.frombuffer(shm.buf, dtype=torch.bfloat16, count=math.prod(shp)).view(shp)
+
+        @staticmethod
+        def part(x, i, shape):
+            return x[i]
 
         def exchange_pack(self, x, send, shape):
             send.copy_(bf16(oracle.exchange_pack(words(x), shape.N, shape.P)))

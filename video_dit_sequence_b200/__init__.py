@@ -445,6 +445,14 @@ class CudaPeerBackend:
                 self._opened[handle] = ipc_open(handle)
         return self._opened[handle] + offset
 
+    @staticmethod
+    def part(x, i: int, shape: Shape):
+        """Sub-buffer i of an exported [2][B][Nl][H][D] buffer: a tensor index
+        for this rank's own buffer, a byte offset for a mapped peer's."""
+        if isinstance(x, int):
+            return x + i * 2 * math.prod(shape.rank_shard)
+        return x[i]
+
     def exchange_pack(self, x, send, shape: Shape):
         exchange_pack(x, send, shape)
 
@@ -464,9 +472,9 @@ class UlyssesPeerRank:
     the attention kernel.
 
     Construction allocates this rank's Q shard and output shard
-    ([B][Nl][H][D] each), exports both, gathers every rank's exports over the
-    process group and maps the peers' buffers, so that every rank holds the
-    P Q-shard and P O-shard addresses in rank order.  step(k, v, q) then
+    ([B][Nl][H][D] each, one buffer), exports it, gathers every rank's export
+    over the process group and maps the peers' buffers (each once), so that
+    every rank holds the P Q-shard and P O-shard addresses in rank order.  step(k, v, q) then
       writes q into the Q shard (or the caller wrote it),
       reorders k and v into send chunks (sp_exchange_pack) and exchanges
         them (all-to-all: chunk j of every rank to rank j),
@@ -491,22 +499,18 @@ class UlyssesPeerRank:
         if backend is None:
             backend = CudaPeerBackend(device if device is not None else torch.cuda.current_device())
         self.backend = be = backend
-        self.q_shard = be.empty(shape.rank_shard)
-        self.o_shard = be.empty(shape.rank_shard)
+        self._qo = be.empty((2,) + tuple(shape.rank_shard))     # [Q shard, O shard]
+        self.q_shard, self.o_shard = self._qo[0], self._qo[1]
         self._k_send, self._v_send, self._k_recv, self._v_recv = (
             be.empty(shape.send_chunks) for _ in range(4))
         self._flag = be.empty((1,), torch.float32)
         table = [None] * shape.P
-        dist.all_gather_object(table, (be.export(self.q_shard), be.export(self.o_shard)),
-                               group=group)
+        dist.all_gather_object(table, be.export(self._qo), group=group)
         self.q_addrs, self.o_addrs = [], []
-        for r, (qx, ox) in enumerate(table):
-            if r == self.rank:
-                self.q_addrs.append(self.q_shard)
-                self.o_addrs.append(self.o_shard)
-            else:
-                self.q_addrs.append(be.open(*qx))
-                self.o_addrs.append(be.open(*ox))
+        for r, exported in enumerate(table):
+            x = self._qo if r == self.rank else be.open(*exported)
+            self.q_addrs.append(be.part(x, 0, shape))
+            self.o_addrs.append(be.part(x, 1, shape))
 
     def step(self, k, v, q=None):
         import torch.distributed as dist
