@@ -565,6 +565,37 @@ def test_dominant_key_selects_value_row():
     assert np.max(np.abs(O[0] - want[None])) < 1e-2
 
 
+@pytest.mark.parametrize("blocks", [("A",), ("A", "B"), ("B",)])
+def test_reference_moves_mid_row(blocks):
+    """A row's reference maximum moves mid-row, with O and the row sum
+    rescaled in TMEM.  Block A (keys 640..703, the first half of key tile 5)
+    and block B (keys 1216..1279, the second half of tile 9) carry logits
+    about 34 and 68 log2 units above the rest for even query rows (the later
+    block dominating the earlier), and far below for odd rows, so warps mix
+    rows that move their reference with rows that keep it.  Output against
+    the oracle, and bit for bit across degrees and between the fused and
+    three-call paths."""
+    B, N, H, D = 1, 1500, 2, 128
+    q, k, v = _random_logical(B, N, H, D, seed=17)
+    qf = np.abs(synth.bf16_to_f32(q)) + 0.5
+    qf[:, 1::2] *= -1.0
+    q = synth.f32_to_bf16(qf)
+    kf = np.clip(synth.bf16_to_f32(k), -1, 1)
+    if "A" in blocks:
+        kf[:, 640:704] = 1.6
+    if "B" in blocks:
+        kf[:, 1216:1280] = 3.2
+    k = synth.f32_to_bf16(kf)
+    outs = [_run_fused(q, k, v, P)[0] for P in (1, 2, 4)]
+    for P, out in zip((2, 4), outs[1:]):
+        assert np.array_equal(synth.from_seq_shards(out.reshape(P, B, -1, H, D), N),
+                              synth.from_seq_shards(outs[0].reshape(1, B, -1, H, D), N))
+    unf, _ = _run_unfused(q, k, v, 2)
+    assert np.array_equal(unf, outs[1])
+    rows = _rows_all(B, N, H)
+    _check_rows(outs[0], q, k, v, rows, 1, f"reference moves {blocks}")
+
+
 def test_wait_timeout_is_reported_not_hung():
     sp.selftest_wait_timeout(1_000_000)  # 1 ms
     assert sp.device_status() == sp.SP_ERR_TIMEOUT
