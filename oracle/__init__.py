@@ -17,6 +17,10 @@ What it computes, and the passages it follows:
 * ``attention_rows_e4m3`` -- the same attention on 8-bit (E4M3) inputs with
   scale factors per block of tokens for Q and K and per channel for V, for
   the FP8 variant of the kernel.
+* ``attention_rows_masked`` -- the same attention restricted by a block mask
+  over cubes of consecutive tokens (the sparse stage of video sparse
+  attention, which the FastVideo page names with 64-token tiles), for the
+  block-sparse kernel.
 * ``attention_rows`` -- the unsharded softmax(q K^T scale) V of one head,
   two-pass exact softmax in fp64; the sequence-parallel result must equal it
   for every degree (LTX-2 "Multi-GPU Inference" README, Capabilities table:
@@ -68,6 +72,9 @@ def _bind(path: str):
         vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp,
         ctypes.c_int]
     lib.sp_oracle_attention_rows_e4m3.restype = ctypes.c_int
+    lib.sp_oracle_attention_rows_masked.argtypes = [
+        vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp, ctypes.c_int]
+    lib.sp_oracle_attention_rows_masked.restype = ctypes.c_int
     lib.sp_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
     lib.sp_oracle_e4m3_value.restype = ctypes.c_double
     return lib
@@ -217,6 +224,33 @@ def attention_rows_e4m3(q8, k8, v8, dq, dk, dv, rows, scale: float = 0.0,
         q8.ctypes.data, k8.ctypes.data, v8.ctypes.data, dq.ctypes.data, dk.ctypes.data,
         dv.ctypes.data, int(block), B, N, H, D, float(scale), R, rows.ctypes.data,
         o.ctypes.data, lse.ctypes.data, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle attention failed ({rc})")
+    return o, lse
+
+
+def attention_rows_masked(q, k, v, mask, rows, scale: float = 0.0, cube: int = 64,
+                          threads: Optional[int] = None, lib=None):
+    """fp64 attention restricted by a block mask: query i of (b, h) attends
+    key t only when mask[b][h][i // cube][t // cube] is non-zero (mask: bool
+    or uint8 [B][H][ceil(N / cube)][ceil(N / cube)]).  A query that selects
+    no key gets O = 0 and LSE = -inf.  Returns (O [R][D], LSE [R])."""
+    for a in (q, k, v):
+        assert a.dtype == np.uint16 and a.shape == q.shape and a.ndim == 4
+    B, N, H, D = q.shape
+    nc = -(-N // cube)
+    mask = np.ascontiguousarray(np.asarray(mask).astype(np.uint8))
+    assert mask.shape == (B, H, nc, nc), mask.shape
+    q, k, v = (np.ascontiguousarray(a) for a in (q, k, v))
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    R = rows.shape[0]
+    o = np.empty((R, D), dtype=np.float64)
+    lse = np.empty(R, dtype=np.float64)
+    if threads is None:
+        threads = max(1, len(os.sched_getaffinity(0)))
+    rc = (lib or _load()).sp_oracle_attention_rows_masked(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, mask.ctypes.data, int(cube), B, N, H, D,
+        float(scale), R, rows.ctypes.data, o.ctypes.data, lse.ctypes.data, int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle attention failed ({rc})")
     return o, lse

@@ -35,6 +35,11 @@
  *    block of consecutive tokens, V one per channel (the contraction of q.k
  *    runs over channels and that of p.v over tokens, so these factors come
  *    out of the sums).
+ *  - block-sparse attention (the sparse stage of video sparse attention, named
+ *    on "Pair two NVIDIA DGX Sparks" with 64-token tiles and sparsity 0.8,
+ *    its block selection not defined there): a query attends only the keys
+ *    of the key cubes a block mask selects for its query cube; the mask is an
+ *    input.  A query whose cube selects nothing gets O = 0 and lse = -inf.
  *
  * Element type: bf16, given as its 16-bit pattern, or E4M3 bytes with their
  * factors.  The oracle widens each value exactly to double.
@@ -181,6 +186,11 @@ typedef struct {
      * of blk consecutive tokens; dv [B][H][D], one per channel. */
     const double *dq, *dk, *dv;
     int64_t blk, nblk;
+    /* Block mask, or NULL for every key: key kk is attended by query i of
+     * (b, h) iff mask[((b * H + h) * ncube + i / cube) * ncube + kk / cube]
+     * is non-zero (cubes of `cube` consecutive tokens, ncube of them). */
+    const uint8_t *mask;
+    int64_t cube, ncube;
     int64_t B, N, H, D;
     double scale;
     int64_t nrows;
@@ -203,8 +213,13 @@ static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
     int64_t N = J->N, H = J->H, D = J->D, bh = b * H + h;
     int64_t qi = ((b * N + i) * H + h) * D;
     double sq = J->q8 ? J->dq[bh * J->nblk + i / J->blk] : 1.0;
+    const uint8_t *sel = J->mask ? J->mask + (bh * J->ncube + i / J->cube) * J->ncube : NULL;
     double m = -INFINITY;
     for (int64_t kk = 0; kk < N; ++kk) {
+        if (sel && !sel[kk / J->cube]) {
+            s[kk] = -INFINITY;              /* key not in a selected cube */
+            continue;
+        }
         int64_t kr = ((b * N + kk) * H + h) * D;
         double sk = J->k8 ? J->dk[bh * J->nblk + kk / J->blk] : 1.0;
         double dot = 0.0;
@@ -215,8 +230,13 @@ static void attention_one_row(const attn_job_t *J, int64_t r, double *s) {
     }
     double *o = J->out_o + r * D;
     for (int64_t c = 0; c < D; ++c) o[c] = 0.0;
+    if (m == -INFINITY) {                   /* no key selected: O = 0, lse = -inf */
+        if (J->out_lse) J->out_lse[r] = -INFINITY;
+        return;
+    }
     double l = 0.0;
     for (int64_t kk = 0; kk < N; ++kk) {
+        if (s[kk] == -INFINITY) continue;
         double w = exp(s[kk] - m);
         l += w;
         int64_t vr = ((b * N + kk) * H + h) * D;
@@ -282,6 +302,28 @@ int sp_oracle_attention_rows_e4m3(const uint8_t *q8, const uint8_t *k8, const ui
     J.q8 = q8; J.k8 = k8; J.v8 = v8;
     J.dq = dq; J.dk = dk; J.dv = dv;
     J.blk = blk; J.nblk = (N + blk - 1) / blk;
+    J.B = B; J.N = N; J.H = H; J.D = D;
+    J.scale = scale;
+    J.nrows = nrows; J.rows = rows;
+    J.out_o = out_o; J.out_lse = out_lse;
+    return attention_rows_impl(&J, nthreads);
+}
+
+/* The same attention restricted by a block mask (the sparse stage of video
+ * sparse attention): query i of (b, h) attends key kk only when the mask
+ * selects kk's cube for i's cube, mask [B][H][ncube][ncube] bytes with
+ * ncube = ceil(N / cube).  A query whose cube selects no key gets O = 0 and
+ * lse = -inf. */
+int sp_oracle_attention_rows_masked(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                    const uint8_t *mask, int64_t cube,
+                                    int64_t B, int64_t N, int64_t H, int64_t D, double scale,
+                                    int64_t nrows, const int64_t *rows, double *out_o,
+                                    double *out_lse, int nthreads) {
+    attn_job_t J;
+    memset(&J, 0, sizeof(J));
+    if (mask == NULL || cube < 1) return -1;
+    J.q = q; J.k = k; J.v = v;
+    J.mask = mask; J.cube = cube; J.ncube = (N + cube - 1) / cube;
     J.B = B; J.N = N; J.H = H; J.D = D;
     J.scale = scale;
     J.nrows = nrows; J.rows = rows;

@@ -364,6 +364,65 @@ def check_fp8_block_factors_match_dequantized_bf16(lib=None):
     assert np.max(np.abs(l8 - lb)) < 1e-12 * max(1.0, np.max(np.abs(lb)))
 
 
+def _all_rows(B, N, H):
+    return np.array([(b, h, i) for b in range(B) for h in range(H) for i in range(N)],
+                    dtype=np.int64)
+
+
+def check_masked_attention(lib=None):
+    """Block-masked attention (the sparse stage of video sparse attention)
+    against what the mask means, on a ragged last cube (N = 45, cubes of 8):
+    * every cube selected -> the dense oracle, exactly;
+    * one key cube per query cube -> dense attention over that cube's keys
+      alone (the dense oracle on the sliced K and V);
+    * a random selection -> numpy's fp64 softmax with the unselected scores
+      set to -inf (scipy logsumexp for the LSE);
+    * a query cube that selects nothing -> O = 0 and LSE = -inf."""
+    rng = np.random.default_rng(RNG_SEED + 18)
+    B, N, H, D, cube = 2, 45, 2, 16, 8
+    nc = -(-N // cube)
+    q, k, v = (_bf16_normal((B, N, H, D), rng, m) for m in (1.0, 1.5, 1.0))
+    rows = _all_rows(B, N, H)
+    full = np.ones((B, H, nc, nc), np.uint8)
+    Om, Lm = oracle.attention_rows_masked(q, k, v, full, rows, cube=cube, threads=2, lib=lib)
+    Od, Ld = oracle.attention_rows(q, k, v, rows, threads=2, lib=lib)
+    assert np.array_equal(Om, Od) and np.array_equal(Lm, Ld)
+
+    pick = rng.integers(0, nc, size=(B, H, nc))
+    one = np.zeros((B, H, nc, nc), np.uint8)
+    for b in range(B):
+        for h in range(H):
+            one[b, h, np.arange(nc), pick[b, h]] = 1
+    O1, L1 = oracle.attention_rows_masked(q, k, v, one, rows, cube=cube, threads=2, lib=lib)
+    for r, (b, h, i) in enumerate(rows):
+        c = pick[b, h, i // cube]
+        ks = slice(c * cube, min(N, (c + 1) * cube))
+        kc = np.ascontiguousarray(k[b:b + 1, ks, h:h + 1])
+        vc = np.ascontiguousarray(v[b:b + 1, ks, h:h + 1])
+        qc = np.zeros_like(kc)
+        qc[0, 0, 0] = q[b, i, h]                     # the query as row 0 of a dense problem
+        want, wl = oracle.attention_rows(qc, kc, vc, np.zeros((1, 3), np.int64),
+                                         scale=1.0 / math.sqrt(D), threads=1, lib=lib)
+        assert np.max(np.abs(O1[r] - want[0])) < 1e-13 and abs(L1[r] - wl[0]) < 1e-13
+
+    sel = (rng.random((B, H, nc, nc)) < 0.3).astype(np.uint8)
+    sel[0, 1, 2] = 0                                 # query cube 2 of (0, 1) selects nothing
+    sel[1, 0, :, nc - 1] = 1                         # the ragged last cube is selected
+    Os, Ls = oracle.attention_rows_masked(q, k, v, sel, rows, cube=cube, threads=2, lib=lib)
+    qf, kf, vf = _f64(q), _f64(k), _f64(v)
+    tok = np.arange(N) // cube
+    for r, (b, h, i) in enumerate(rows):
+        keep = sel[b, h, i // cube][tok].astype(bool)
+        if not keep.any():
+            assert np.all(Os[r] == 0) and Ls[r] == -np.inf
+            continue
+        sc = np.where(keep, kf[b, :, h] @ qf[b, i, h] / math.sqrt(D), -np.inf)
+        lse = logsumexp(sc)
+        assert abs(Ls[r] - lse) < 1e-12
+        assert np.max(np.abs(Os[r] - np.exp(sc - lse) @ vf[b, :, h])) < 1e-12
+    assert np.any(~sel[0, 1, 2].astype(bool))
+
+
 PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
                check_unpack_returns_shards, check_pack_degree_one_is_copy,
                check_exchange_chunks_hold_head_groups,
@@ -372,5 +431,5 @@ ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one
                     check_closed_forms, check_dominant_key, check_invariances,
                     check_two_token_example, check_rows_api,
                     check_e4m3_decode_matches_torch, check_fp8_attention_reduces_to_bf16,
-                    check_fp8_block_factors_match_dequantized_bf16]
+                    check_fp8_block_factors_match_dequantized_bf16, check_masked_attention]
 ALL_CHECKS = PACK_CHECKS + ATTENTION_CHECKS

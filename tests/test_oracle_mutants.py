@@ -38,8 +38,8 @@ MUTANTS = [
     ("dot-drops-last-channel", "for (int64_t c = 0; c < D; ++c)\n            dot +=",
      "for (int64_t c = 0; c + 1 < D; ++c)\n            dot +="),
     ("second-pass-drops-last-key",
-     "for (int64_t kk = 0; kk < N; ++kk) {\n        double w",
-     "for (int64_t kk = 0; kk + 1 < N; ++kk) {\n        double w"),
+     "for (int64_t kk = 0; kk < N; ++kk) {\n        if (s[kk] == -INFINITY) continue;\n        double w",
+     "for (int64_t kk = 0; kk + 1 < N; ++kk) {\n        if (s[kk] == -INFINITY) continue;\n        double w"),
     ("k-transposed-with-q",
      "elem(J->k, J->k8, sk, kr + c);",
      "elem(J->q, J->q8, sq, qi + c);"),
@@ -57,6 +57,14 @@ MUTANTS = [
      "J->dk[bh * J->nblk + i / J->blk]"),
     ("v-factor-of-channel-0", "J->dv[bh * D + c]", "J->dv[bh * D]"),
     ("v-takes-q-factor", "J->v8 ? J->dv[bh * D + c] : 1.0", "J->v8 ? sq : 1.0"),
+    ("mask-query-cube-off-by-one", "(bh * J->ncube + i / J->cube) * J->ncube",
+     "(bh * J->ncube + (i + 1) / J->cube - ((i + 1) / J->cube == J->ncube)) * J->ncube"),
+    ("mask-key-cube-of-query", "if (sel && !sel[kk / J->cube]) {",
+     "if (sel && !sel[i / J->cube]) {"),
+    ("mask-head-ignored", "J->mask + (bh * J->ncube + i / J->cube) * J->ncube",
+     "J->mask + (b * H * J->ncube + i / J->cube) * J->ncube"),
+    ("mask-empty-row-not-zero", "        if (J->out_lse) J->out_lse[r] = -INFINITY;\n        return;",
+     "        if (J->out_lse) J->out_lse[r] = -INFINITY;\n        o[0] = 1.0;\n        return;"),
 ]
 
 
