@@ -463,6 +463,17 @@ def run_ours(args):
         o8 = torch.empty_like(os_)
         t_fp8 = timed(lambda: sp.attention_fp8_seqsharded(*dev8, *fac8, o8, shape, stream=stream))
         del dev8, fac8, o8
+    # block-sparse variant on the same problem: a synthetic cube mask of
+    # density 0.2 (the pages' sparsity 0.8), one selection per 256 query tokens
+    t_sparse = None
+    if not args.no_sparse and s.D == 128:
+        mask = synth.cube_mask(cfg, density=0.2, group=4)
+        words = torch.from_numpy(sp.sparse_mask_words(mask).view(np.int32)).to(dev)
+        o_sp = torch.empty_like(os_)
+        t_sparse = timed(lambda: sp.attention_sparse_seqsharded(qs, ks, vs, words, o_sp, shape,
+                                                                stream=stream))
+        sparse_flops = 4.0 * synth.attended_pairs(mask, s.N) * s.D
+        del words, o_sp
     if sp.device_status(stream) != sp.SP_OK:
         raise SystemExit("device status not ok after the unfused rows")
     pack_gbs = 2 * tensor_bytes / (t_pack * 1e-3) / 1e9
@@ -482,6 +493,10 @@ def run_ours(args):
             "peak_source": f"{pkq} bf16 burst x 2 (nominal fp8/bf16 ratio)",
             "inputs": "E4M3 Q/K/V; factors per 128-token block (Q, K) and per "
                       "channel (V); bf16 output"},
+        "sparse": None if t_sparse is None else {
+            "ms": t_sparse, "speedup_vs_dense": per_launch_ms / t_sparse,
+            "attended_TFLOP/s": sparse_flops / (t_sparse * 1e-3) / 1e12,
+            "mask": "64-token cubes, density 0.2, one selection per 4 query cubes (synthetic)"},
         "unfused_step_ms": 3 * t_pack + t_attn + t_unpack,
         "fused_step_ms": per_launch_ms,
     }
@@ -562,6 +577,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 row")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse row")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override N (same heads, head dim and degree); for profiling captures")
     ap.add_argument("--traffic-bytes", type=float, default=None,

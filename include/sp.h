@@ -170,6 +170,31 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
                                       const float *v_scale, void *os, float *lse,
                                       const sp_shape *shape, void *stream);
 
+/* Tokens per cube of the block-sparse call's mask. */
+#define SP_SPARSE_CUBE 64
+
+/* Block-sparse variant of sp_attention_seqsharded: the sparse stage of video
+ * sparse attention, which the FastVideo page ("Pair two NVIDIA DGX Sparks",
+ * the FastH3 release stacks) runs with 64-token tiles and sparsity 0.8 but
+ * whose block selection it does not define.  The selection is the caller's:
+ * query token i attends key token t only when the mask selects t's cube for
+ * i's cube (cubes of SP_SPARSE_CUBE consecutive tokens of the logical
+ * sequence).  A query whose cube selects no key gets a zero output row and
+ * lse = -inf.
+ * mask: device uint32 [B][H][ncube][nwords], ncube = ceil(N / 64),
+ *   nwords = ceil(ncube / 32); bit c of word w in query cube qc's row selects
+ *   key cube 32*w + c; bits for cubes >= ncube are ignored.  Read only,
+ *   4-byte aligned.
+ * qs, ks, vs, os, lse as for sp_attention_seqsharded; D must be 128 and
+ * ceil(N / 128) <= 16384 (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  The kernel
+ * visits, for each pair of 128-row query tiles, only the 128-key tiles that
+ * one of their four query cubes selects.  With every cube selected the
+ * result equals sp_attention_seqsharded's bit for bit; results do not depend
+ * on P. */
+sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const void *vs,
+                                         const uint32_t *mask, void *os, float *lse,
+                                         const sp_shape *shape, void *stream);
+
 /* ---------------------------------------------------------------------
  * Multi-GPU form with the Q and O exchanges fused into the attention kernel.
  *

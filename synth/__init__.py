@@ -257,6 +257,33 @@ def to_e4m3(x: np.ndarray) -> np.ndarray:
         torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
+SPARSE_CUBE = 64   # tokens per cube of a block-sparse mask
+
+
+def cube_mask(cfg: Config, density: float = 0.2, group: int = 4, seed: int = 0):
+    """A seeded block mask for the block-sparse call: over cubes of 64 tokens,
+    each query cube selects key cubes independently with probability
+    `density`, and each `group` consecutive query cubes share one selection
+    (a spatially coherent pattern, as neighbouring video cubes tend to pick
+    similar key cubes).  The pages give a sparsity (0.8) and the cube size but
+    no selection rule; this pattern is a synthetic stand-in.  Returns bool
+    [B][H][nc][nc]."""
+    s = cfg.shape
+    nc = -(-s.N // SPARSE_CUBE)
+    rng = np.random.default_rng([cfg.seed, seed, 64])
+    base = rng.random((s.B, s.H, -(-nc // group), nc)) < density
+    return np.ascontiguousarray(np.repeat(base, group, axis=2)[:, :, :nc])
+
+
+def attended_pairs(mask: np.ndarray, N: int) -> float:
+    """(query, key) pairs a cube mask selects over N tokens, summed over
+    batches and heads."""
+    nc = mask.shape[-1]
+    sizes = np.full(nc, SPARSE_CUBE, dtype=np.float64)
+    sizes[-1] = N - SPARSE_CUBE * (nc - 1)
+    return float(np.einsum("bhqk,q,k->", mask.astype(np.float64), sizes, sizes))
+
+
 FP8_BLOCK = 128   # tokens per Q/K scale block of the 8-bit inputs
 
 

@@ -135,6 +135,13 @@ def test_argument_errors_return_before_launch(lib):
     assert peer(ok_q, A, A, ok_o, 0, sp.Shape(1, 1000, 6, 128, 4)) == \
         sp.SP_ERR_HEADS_NOT_DIVISIBLE
     assert peer(ok_q * 4, A, A, ok_o * 4, 0, sp.Shape(1, 1000, 16, 128, 16)) == sp.SP_ERR_SHAPE
+    sparse = lambda m, shp=sp.Shape(1, 1000, 4, 128, 2): lib.sp_attention_sparse_seqsharded(
+        ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(A),
+        ctypes.c_void_p(m) if m else None, ctypes.c_void_p(B_), None, ctypes.byref(shp.c()), None)
+    assert sparse(0) == sp.SP_ERR_NULL
+    assert sparse(C + 2) == sp.SP_ERR_ALIGN
+    assert sparse(C, sp.Shape(1, 1000, 4, 64, 2)) == sp.SP_ERR_UNSUPPORTED_D
+    assert sparse(C, sp.Shape(1, 128 * 16384 + 1, 1, 128, 1)) == sp.SP_ERR_SHAPE
     h = (ctypes.c_uint8 * sp.IPC_HANDLE_BYTES)()
     off = ctypes.c_int64()
     base = ctypes.c_void_p()

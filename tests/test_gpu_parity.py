@@ -309,6 +309,91 @@ def test_padding_rows_past_the_last_full_tile_pair():
     assert np.array_equal(fused, unfused)
 
 
+# ------------------------------------------------------------------ block-sparse
+
+def _run_sparse(q, k, v, mask, P, lse=False):
+    B, N, H, D = q.shape
+    shape = sp.Shape(B, N, H, D, P)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    os_ = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    l = torch.full(shape.lse_shape, float("nan"), dtype=torch.float32, device="cuda") if lse else None
+    words = torch.from_numpy(sp.sparse_mask_words(mask).view(np.int32)).cuda()
+    sp.attention_sparse_seqsharded(qs, ks, vs, words, os_, shape, lse=l)
+    _status_ok()
+    return to_host(os_), (l.cpu().numpy() if lse else None)
+
+
+def _cube_mask(B, H, N, density, seed, group=1):
+    """Random selection over 64-token cubes; `group` consecutive query cubes
+    share one selection (a spatially coherent pattern)."""
+    nc = -(-N // 64)
+    rng = np.random.default_rng(seed)
+    base = rng.random((B, H, -(-nc // group), nc)) < density
+    return np.repeat(base, group, axis=2)[:, :, :nc]
+
+
+def test_sparse_full_mask_equals_dense_bit_for_bit():
+    B, N, H, D, P = 1, 1500, 4, 128, 2
+    q, k, v = _random_logical(B, N, H, D, seed=31)
+    full = np.ones((B, H, -(-N // 64), -(-N // 64)), bool)
+    got, lg = _run_sparse(q, k, v, full, P, lse=True)
+    want, lw = _run_fused(q, k, v, P, lse=True)
+    assert np.array_equal(got, want)
+    assert np.array_equal(lg, lw)
+
+
+@pytest.mark.parametrize("B,N,H,P,density,group", [(1, 1500, 4, 2, 0.2, 1), (2, 1000, 4, 4, 0.2, 4),
+                                                   (1, 3000, 2, 1, 0.5, 2), (3, 333, 2, 3, 0.3, 1),
+                                                   (1, 4096, 8, 8, 0.2, 4)])
+def test_sparse_against_oracle(B, N, H, P, density, group):
+    """Random cube masks on ragged lengths, batches and degrees: every row
+    against the masked fp64 oracle, bit for bit across degrees."""
+    D = 128
+    q, k, v = _random_logical(B, N, H, D, seed=N + P)
+    mask = _cube_mask(B, H, N, density, seed=N, group=group)
+    nc = mask.shape[-1]
+    mask[0, 0, 1] = False                            # a query cube that selects nothing
+    got, lse = _run_sparse(q, k, v, mask, P, lse=True)
+    rows = _rows_all(B, N, H)
+    O = synth.from_seq_shards(got.reshape(P, B, -1, H, D), N)
+    ref, lref = oracle.attention_rows_masked(q, k, v, mask, rows)
+    gotr = O[rows[:, 0], rows[:, 2], rows[:, 1]]
+    empty = ~mask[rows[:, 0], rows[:, 1], rows[:, 2] // 64].any(axis=1)
+    assert empty.any()
+    assert np.all(synth.bf16_to_f32(gotr[empty]) == 0.0)
+    assert np.all(lse[rows[empty, 0], rows[empty, 1], rows[empty, 2]] == -np.inf)
+    m = compare(gotr[~empty], ref[~empty], rows[~empty, 1])
+    assert_parity(m, f"sparse B={B} N={N} P={P}")
+    gl = lse[rows[~empty, 0], rows[~empty, 1], rows[~empty, 2]]
+    assert np.max(np.abs(gl - lref[~empty])) < 2e-2
+    if P > 1:
+        one, _ = _run_sparse(q, k, v, mask, 1)
+        assert np.array_equal(O, synth.from_seq_shards(one.reshape(1, B, -1, H, D), N))
+    print(f"sparse B={B} N={N} P={P} density={density}: {m}, nc={nc}")
+
+
+def test_sparse_cta_with_no_selected_tile():
+    """Query cubes 4..7 (one CTA's 256 rows) select nothing: that CTA visits
+    no key tile and writes zero rows; bits past the last cube are ignored."""
+    B, N, H, D, P = 1, 1000, 2, 128, 2
+    q, k, v = _random_logical(B, N, H, D, seed=37)
+    mask = _cube_mask(B, H, N, 0.3, seed=37)
+    mask[:, :, 4:8] = False
+    words = sp.sparse_mask_words(mask)
+    words[..., -1] |= np.uint32(0xFFFFFFFF) << np.uint32(mask.shape[-1] % 32)  # junk past ncube
+    shape = sp.Shape(B, N, H, D, P)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    os_ = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.attention_sparse_seqsharded(qs, ks, vs, torch.from_numpy(words.view(np.int32)).cuda(),
+                                   os_, shape)
+    _status_ok()
+    O = synth.from_seq_shards(to_host(os_).reshape(P, B, -1, H, D), N)
+    assert np.all(synth.bf16_to_f32(O[:, 256:512]) == 0.0)
+    rows = _rows_all(B, N, H)
+    ref, _ = oracle.attention_rows_masked(q, k, v, mask, rows)
+    assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]), "junk bits")
+
+
 # ------------------------------------------------------------------ attention, small
 
 def test_tiny_config_every_row():

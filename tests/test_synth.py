@@ -113,3 +113,19 @@ def test_fp8_quantisation_groups():
     deq_v = val(v8) * dv[:, None]
     assert np.all(np.abs(val(v8)).max(axis=1) == 448.0)
     assert np.all(np.abs(deq_v - v) <= 2.0 ** -4 * np.abs(v) + 2.0 ** -10 * dv[:, None])
+
+
+def test_cube_mask_and_attended_pairs():
+    cfg = synth.Config("m", synth.Shape(2, 1000, 3, 128, 1), seed=5)
+    m = synth.cube_mask(cfg, density=0.2, group=4)
+    nc = 16                                            # ceil(1000 / 64)
+    assert m.shape == (2, 3, nc, nc) and m.dtype == bool
+    assert np.array_equal(m[:, :, 0], m[:, :, 3]) and np.array_equal(m[:, :, 12], m[:, :, 15])
+    assert 0.1 < m.mean() < 0.3
+    assert np.array_equal(m, synth.cube_mask(cfg, density=0.2, group=4))
+    # brute force over tokens on a small case
+    small = synth.Config("s", synth.Shape(1, 150, 1, 16, 1), seed=6)
+    ms = synth.cube_mask(small, density=0.5, group=1)
+    tok = np.arange(150) // 64
+    brute = ms[0, 0][tok][:, tok].sum()
+    assert synth.attended_pairs(ms, 150) == brute

@@ -42,7 +42,8 @@ EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_attention", "sp_attention_seqsharded", "sp_device_status",
             "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout",
             "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded",
-            "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close")
+            "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close",
+            "sp_attention_sparse_seqsharded")
 
 
 class sp_shape(ctypes.Structure):
@@ -83,6 +84,8 @@ def load(path: str = LIB_PATH):
         f.restype = ctypes.c_int
     lib.sp_attention_fp8_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sp_p, vp]
     lib.sp_attention_fp8_seqsharded.restype = ctypes.c_int
+    lib.sp_attention_sparse_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, sp_p, vp]
+    lib.sp_attention_sparse_seqsharded.restype = ctypes.c_int
     lib.sp_attention_ulysses_peer.argtypes = [
         ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), vp, ctypes.c_int32, sp_p, vp]
     lib.sp_attention_ulysses_peer.restype = ctypes.c_int
@@ -362,6 +365,47 @@ class UlyssesRank:
         out = torch.empty(self.shape.rank_shard, dtype=back.dtype, device=back.device)
         exchange_unpack(back, out, self.shape, stream)
         return out
+
+
+SPARSE_CUBE = 64         # SP_SPARSE_CUBE
+
+
+def sparse_mask_words(mask):
+    """A block mask as the sparse call takes it: mask is bool (or 0/1)
+    [B][H][nc][nc] over cubes of SPARSE_CUBE tokens (mask[b][h][qc][kc]:
+    query cube qc attends key cube kc); returns uint32 [B][H][nc][nwords]
+    with bit kc % 32 of word kc // 32 set for a selected key cube."""
+    import numpy as np
+    m = np.asarray(mask).astype(bool)
+    B, H, nc, nc2 = m.shape
+    if nc != nc2:
+        raise ValueError(f"mask must be square over cubes, got {m.shape}")
+    nw = -(-nc // 32)
+    padded = np.zeros((B, H, nc, nw * 32), dtype=bool)
+    padded[..., :nc] = m
+    bits = np.packbits(padded.reshape(B, H, nc, nw, 32), axis=-1, bitorder="little")
+    return np.ascontiguousarray(bits.view(np.uint32).reshape(B, H, nc, nw))
+
+
+def attention_sparse_seqsharded(qs, ks, vs, mask_words, os_, shape: Shape, lse=None,
+                                stream=None):
+    """Block-sparse fused attention: sequence-sharded bf16 qs/ks/vs/os_ as for
+    attention_seqsharded, mask_words a CUDA int32/uint32 tensor
+    [B][H][ncube][nwords] (sparse_mask_words)."""
+    torch = _torch()
+    s = shape.c()
+    ss = shape.seq_sharded
+    nc = -(-shape.N // SPARSE_CUBE)
+    mshape = (shape.B, shape.H, nc, -(-nc // 32))
+    if not isinstance(mask_words, torch.Tensor) or mask_words.dtype not in (torch.int32,
+                                                                            torch.uint32):
+        raise TypeError("mask_words must be an int32 or uint32 CUDA tensor")
+    with _same_device(qs, ks, vs, mask_words, os_, lse):
+        _check(load().sp_attention_sparse_seqsharded(
+            _ptr(qs, ss, "qs"), _ptr(ks, ss, "ks"), _ptr(vs, ss, "vs"),
+            _ptr(mask_words, mshape, "mask_words", mask_words.dtype), _ptr(os_, ss, "os"),
+            _ptr(lse, shape.lse_shape, "lse", torch.float32), ctypes.byref(s),
+            _stream(stream, qs.device)), "sp_attention_sparse_seqsharded")
 
 
 MAX_PEERS = 8            # SP_MAX_PEERS

@@ -68,6 +68,10 @@ struct AttnParams {
   int32_t nblk;
   float *lse;           // [B][H][Np] or null
   int32_t *status;      // device status word
+  // Block-sparse variant: mask [B][H][ncube][nwords] bits over cubes of 64
+  // tokens; bit c of word w in query cube qc's row selects key cube 32w + c.
+  const uint32_t *mask;
+  int32_t ncube, nwords;
 };
 
 constexpr int32_t kStatusTimeout = 7;
@@ -118,7 +122,11 @@ struct AttnCfg {
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   static constexpr int kNumBar = 1 + 2 * kStages + 8;
   static constexpr int kOffMisc = kOffBar + kNumBar * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  // Block-sparse variant: one bit per key tile, set when any query cube of
+  // the CTA selects either key cube of the tile.
+  static constexpr int kMaxSelWords = 512;                  // 16,384 key tiles
+  static constexpr int kOffSel = kOffMisc + 16;
+  static constexpr int kSmemBytes = kOffSel + 4 * kMaxSelWords + 1024;  // + alignment slack
   static constexpr int kThreads = 320;
   static constexpr uint32_t kColS1 = 128;
   static constexpr uint32_t kColO0 = 256;
@@ -129,10 +137,22 @@ struct AttnCfg {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 
+// Bit i (i < 16) of the result: bit 2i or bit 2i+1 of x.
+__device__ __forceinline__ uint32_t pair_bits(uint32_t x) {
+  x = (x | (x >> 1)) & 0x55555555u;
+  x = (x | (x >> 1)) & 0x33333333u;
+  x = (x | (x >> 2)) & 0x0F0F0F0Fu;
+  x = (x | (x >> 4)) & 0x00FF00FFu;
+  return (x | (x >> 8)) & 0x0000FFFFu;
+}
+
 // The kernel body.  kPeer: Q tiles come from the ranks' shards through
 // `peer` (tmQ unused) and O rows go to the ranks' output shards; K and V are
 // this rank's received head group, addressed as for the fused call.
-template <int D, bool kF8, bool kPeer>
+// kSparse: a block mask over 64-token cubes restricts which keys each query
+// attends; the CTA walks only the key tiles that some of its query cubes
+// select, and each row masks the unselected halves of those tiles.
+template <int D, bool kF8, bool kPeer, bool kSparse = false>
 __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUtensorMap *tmK,
                                                const CUtensorMap *tmV, const AttnParams &p,
                                                const PeerArgs *peer) {
@@ -159,6 +179,42 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   const uint32_t bar_o = bar_p + 32;                      // [2]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sptr + C::kOffMisc + 4);
+  uint32_t *sel_bits = reinterpret_cast<uint32_t *>(sptr + C::kOffSel);
+  const int ntw = (T + 31) >> 5;
+  const int64_t mask_row0 = (static_cast<int64_t>(b) * p.H + hg) * p.ncube;
+  if constexpr (kSparse) {
+    // Key tiles this CTA visits: tile j when any of its four query cubes
+    // selects key cube 2j or 2j + 1.
+    const int qc0 = blockIdx.x * 4;
+    for (int w = threadIdx.x; w < ntw; w += blockDim.x) {
+      uint32_t lo = 0u, hi = 0u;
+      for (int qc = qc0; qc < qc0 + 4 && qc < p.ncube; ++qc) {
+        const uint32_t *m = p.mask + (mask_row0 + qc) * p.nwords;
+        if (2 * w < p.nwords) lo |= __ldg(m + 2 * w);
+        if (2 * w + 1 < p.nwords) hi |= __ldg(m + 2 * w + 1);
+      }
+      uint32_t bits = pair_bits(lo) | (pair_bits(hi) << 16);
+      if (w == ntw - 1 && (T & 31)) bits &= (1u << (T & 31)) - 1u;
+      sel_bits[w] = bits;
+    }
+  }
+  // The key tile visited after tile j (T when none); all roles walk the same
+  // sequence.
+  auto next_tile = [&](int j) -> int {
+    if constexpr (!kSparse) {
+      return j + 1;
+    } else {
+      const int n = j + 1;
+      int w = n >> 5;
+      if (w >= ntw) return T;
+      uint32_t x = sel_bits[w] & (0xffffffffu << (n & 31));
+      while (x == 0u) {
+        if (++w >= ntw) return T;
+        x = sel_bits[w];
+      }
+      return (w << 5) + __ffs(x) - 1;
+    }
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -288,7 +344,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       }
     }
     int it = 0;
-    for (int j = 0; j < T && ok; ++j) {
+    for (int j = next_tile(-1); j < T && ok; j = next_tile(j)) {
       for (int kv = 0; kv < 2; ++kv, ++it) {
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
@@ -360,9 +416,18 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         return true;
       };
       int it = 0;
-      ok = mbar_wait(bar_q, 0, abort_flag, kWaitLimitNs) &&
-           mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs);
-      if (ok) {
+      const int j0 = next_tile(-1);
+      // Q has landed before anything else happens (also when no key tile is
+      // selected, so that no copy into shared memory outlives the CTA).
+      ok = mbar_wait(bar_q, 0, abort_flag, kWaitLimitNs);
+      if (ok && j0 >= T) {
+        // no key tile selected for this CTA: O is never written (the rows
+        // come out as zeros), the epilogue only needs its barrier
+        umma_commit(bar_o);
+        umma_commit(bar_o + 8);
+      }
+      ok = ok && (j0 >= T || mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs));
+      if (ok && j0 < T) {
         tc_fence_after();
         issue_s(0, 0);
         umma_commit(bar_s);
@@ -371,7 +436,8 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         umma_commit(bar_kv_empty);
         it = 1;
       }
-      for (int j = 0; j < T && ok; ++j) {
+      for (int j = j0, jj = 0; j < T && ok; ++jj) {
+        const int jn = next_tile(j);
         // Both K/V waits come first: the loads landed long ago, and no
         // barrier wait sits between a tile's PV and its next S.
         const int sv = it % C::kStages;
@@ -379,23 +445,23 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         ++it;
         if (!ok) break;
         int sk = 0;
-        if (j + 1 < T) {
+        if (jn < T) {
           sk = it % C::kStages;
           ok = mbar_wait(bar_kv_full + 8 * sk, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
           ++it;
           if (!ok) break;
         }
-        ok = issue_pv(0, sv, j == 0, j);
+        ok = issue_pv(0, sv, jj == 0, jj);
         if (!ok) break;
-        if (j + 1 < T) {
+        if (jn < T) {
           issue_s(0, sk);
           umma_commit(bar_s);
         } else {
           umma_commit(bar_o);
         }
-        ok = issue_pv(1, sv, j == 0, j);
+        ok = issue_pv(1, sv, jj == 0, jj);
         if (!ok) break;
-        if (j + 1 < T) {
+        if (jn < T) {
           issue_s(1, sk);
           umma_commit(bar_s + 8);
           umma_commit(bar_kv_empty + 8 * sv);
@@ -404,6 +470,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
           umma_commit(bar_o + 8);
           umma_commit(bar_kv_empty + 8 * sv);
         }
+        j = jn;
       }
     }
     __syncwarp();
@@ -426,9 +493,14 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
     const int tail = p.N - (T - 1) * C::kBN;   // valid keys in the last tile, 1..128
     float m_ref = -INFINITY;                   // reference maximum, log2 units
     float l = 0.f;
-    for (int j = 0; j < T; ++j) {
+    // Block-sparse variant: this row's mask words (its 64-token query cube);
+    // rows past the last cube select nothing.
+    const int qcube = (q0 + t * C::kBM + row) >> 6;
+    const uint32_t *mrow = kSparse && qcube < p.ncube ? p.mask + (mask_row0 + qcube) * p.nwords
+                                                     : nullptr;
+    for (int j = next_tile(-1), jj = 0; j < T; j = next_tile(j), ++jj) {
       // Warp-uniform exit: the TMEM accesses below are warp-collective.
-      const bool got = mbar_wait(bar_s + 8 * t, j & 1, abort_flag, kWaitLimitNs);
+      const bool got = mbar_wait(bar_s + 8 * t, jj & 1, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -459,8 +531,23 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
           m = fmax3(m, __uint_as_float(e[c]), __uint_as_float(e[c + 1]));
         mc[q] = fmaxf(m, __uint_as_float(e[15]));
       }
-      const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
-                             fmaxf(mc[6], mc[7])) * sl2;
+      // Sparse: key cube 2j is the tile's first half, 2j + 1 its second; an
+      // unselected half counts for neither the maximum nor the sum.
+      bool sel0 = true, sel1 = true;
+      if constexpr (kSparse) {
+        const uint32_t word = mrow != nullptr ? __ldg(mrow + (j >> 4)) >> ((2 * j) & 31) : 0u;
+        sel0 = (word & 1u) != 0u;
+        sel1 = (word & 2u) != 0u;
+      }
+      float mx;
+      if constexpr (kSparse) {
+        const float h0 = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
+        const float h1 = fmaxf(fmax3(mc[4], mc[5], mc[6]), mc[7]);
+        mx = fmaxf(sel0 ? h0 : -INFINITY, sel1 ? h1 : -INFINITY) * sl2;
+      } else {
+        mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
+                   fmaxf(mc[6], mc[7])) * sl2;
+      }
       const bool need = mx > m_ref + C::kThresh;
       const bool warp_rescale = __any_sync(0xffffffffu, need);
       const float alpha = need ? ex2(m_ref - mx) : 1.0f;
@@ -474,14 +561,24 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       // the PV MMAs of keys 0..63 can start while keys 64..127 are computed.
       const uint64_t k_sl2 = f2_pack(sl2, sl2);
       const uint64_t k_negm = f2_pack(C::kShift - m_ref, C::kShift - m_ref);
+      // Sparse: an unselected half gets a bias of -inf (its probabilities are
+      // 0); a row that has not met a selected key yet keeps m = -inf and uses
+      // a bias of 0 for its (then all -inf) scores.
+      float bias_h[2] = {0.f, 0.f};
+      if constexpr (kSparse) {
+        const float bias = C::kShift - (m_ref > -INFINITY ? m_ref : 0.f);
+        bias_h[0] = sel0 ? bias : -INFINITY;
+        bias_h[1] = sel1 ? bias : -INFINITY;
+      }
       uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        const uint64_t k_bias = kSparse ? f2_pack(bias_h[h], bias_h[h]) : k_negm;
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int c = 64 * h + 2 * i;
-          const uint64_t x = f2_fma(f2_pack_bits(s[c], s[c + 1]), k_sl2, k_negm);
+          const uint64_t x = f2_fma(f2_pack_bits(s[c], s[c + 1]), k_sl2, k_bias);
           float p0, p1;
           f2_unpack(x, p0, p1);
           p0 = ex2(p0);
@@ -495,7 +592,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
             pk[i] = pack_bf16x2(p0, p1);
           }
         }
-        if (h == 0 && warp_rescale && j > 0) {
+        if (h == 0 && warp_rescale && jj > 0) {
           // Rescale O_t by alpha before any PV MMA of this tile (warp-uniform
           // because TMEM access is warp-collective; rows that keep their
           // reference multiply by exactly 1).  O_t is complete: the commit
@@ -530,7 +627,8 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const int token = q0 + t * C::kBM + row;
-      const bool valid = token < p.N;
+      // Sparse: a row that attended no key (l = 0) is written as zeros.
+      const bool valid = token < p.N && (!kSparse || l > 0.f);
       const bool exists = token < p.Np;
       const float inv_l = valid ? 1.0f / l : 0.0f;
       const float *dv_row = kF8 ? p.dv + static_cast<int64_t>(bh) * D : nullptr;
@@ -567,7 +665,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         for (int i = 0; i < 16; ++i)
           w[i] = valid ? pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
                                      __uint_as_float(o[2 * i + 1]) * inv_l)
-                       : 0u;  // padding rows: +0.0 words
+                       : 0u;  // padding rows (and sparse rows with no key): +0.0 words
         if (exists) {
           uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
 #pragma unroll
@@ -614,6 +712,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnParams p) {
   attention_body<D, kF8, false>(&tmQ, &tmK, &tmV, p, nullptr);
+}
+
+// Block-sparse attention (bf16, D = 128): the sequence-sharded fused call
+// with a mask of selected 64-token key cubes per 64-token query cube.
+__global__ void __launch_bounds__(320, 1)
+attention_sparse_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ AttnParams p) {
+  attention_body<128, false, false, true>(&tmQ, &tmK, &tmV, p, nullptr);
 }
 
 // One rank's step of the multi-GPU form (bf16, D = 128): Q read from every

@@ -230,7 +230,7 @@ cudaError_t set_smem_once(Kernel kernel, int bytes, bool (&done)[kMaxDevices]) {
 sp_status attention(const void *q, const void *k, const void *v, void *o, float *lse,
                     const sp_shape *s, void *stream, bool seqsharded,
                     const float *dq = nullptr, const float *dk = nullptr,
-                    const float *dv = nullptr) {
+                    const float *dv = nullptr, const uint32_t *mask = nullptr) {
   const bool f8 = dq != nullptr;
   if (f8 && (dk == nullptr || dv == nullptr)) return SP_ERR_NULL;
   const int es = f8 ? 1 : 2;
@@ -244,7 +244,11 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
       (f8 && ((reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
                reinterpret_cast<uintptr_t>(dv)) & 3u) != 0))
     return SP_ERR_ALIGN;
-  if (f8 && s->D != 128) return SP_ERR_UNSUPPORTED_D;
+  if ((f8 || mask != nullptr) && s->D != 128) return SP_ERR_UNSUPPORTED_D;
+  if (mask != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(mask) & 3u) != 0) return SP_ERR_ALIGN;
+    if ((s->N + 127) / 128 > 32 * sp::AttnCfg<128>::kMaxSelWords) return SP_ERR_SHAPE;
+  }
   const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
   const int Hl = H / P;
   const int Nl = (N + P - 1) / P;
@@ -300,7 +304,19 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   p.dk = dk;
   p.dv = dv;
   p.nblk = p.num_kv_tiles;
+  p.mask = mask;
+  p.ncube = (N + 63) / 64;
+  p.nwords = (p.ncube + 31) / 32;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (mask != nullptr) {
+    using C = sp::AttnCfg<128>;
+    static bool attr_set[kMaxDevices] = {};
+    cudaError_t e = set_smem_once(sp::attention_sparse_kernel, C::kSmemBytes, attr_set);
+    if (e != cudaSuccess) return SP_ERR_CUDA;
+    dim3 grid((Np + 2 * C::kBM - 1) / (2 * C::kBM), H, B);
+    sp::attention_sparse_kernel<<<grid, C::kThreads, C::kSmemBytes, cs>>>(mq, mk, mv, p);
+    return launch_status(cudaGetLastError());
+  }
   cudaError_t e = f8        ? launch_attention<128, true>(mq, mk, mv, p, B, cs)
                   : D == 64 ? launch_attention<64>(mq, mk, mv, p, B, cs)
                             : launch_attention<128>(mq, mk, mv, p, B, cs);
@@ -465,6 +481,13 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
                                       const sp_shape *shape, void *stream) {
   if (q_scale == nullptr || k_scale == nullptr || v_scale == nullptr) return SP_ERR_NULL;
   return attention(qs, ks, vs, os, lse, shape, stream, true, q_scale, k_scale, v_scale);
+}
+
+sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const void *vs,
+                                         const uint32_t *mask, void *os, float *lse,
+                                         const sp_shape *shape, void *stream) {
+  if (mask == nullptr) return SP_ERR_NULL;
+  return attention(qs, ks, vs, os, lse, shape, stream, true, nullptr, nullptr, nullptr, mask);
 }
 
 sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_group,
