@@ -394,6 +394,94 @@ def test_sparse_cta_with_no_selected_tile():
     assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]), "junk bits")
 
 
+# ------------------------------------------------------------------ guard bands
+
+GUARD = 4096  # elements of sentinel after every output buffer
+
+
+def _guarded(shape, dtype):
+    """An output view with GUARD sentinel elements behind it in the same
+    allocation; returns (view, check) where check() asserts the sentinel is
+    untouched."""
+    n = math.prod(shape)
+    full = torch.empty(n + GUARD, dtype=dtype, device="cuda")
+    raw = full.view(torch.int16) if full.element_size() == 2 else full.view(torch.int32)
+    raw[n:] = 0x5A5A if full.element_size() == 2 else 0x5A5A5A5A
+    snap = raw[n:].clone()
+
+    def check(where):
+        torch.cuda.synchronize()
+        assert torch.equal(raw[n:], snap), f"{where} wrote past its output"
+    return full[:n].view(shape), check
+
+
+def test_outputs_stay_inside_their_buffers():
+    """Every call that writes an output leaves the bytes after it untouched
+    (a stand-in for a memory checker, which this pool does not offer)."""
+    B, N, H, D, P = 2, 777, 6, 128, 3
+    shape = sp.Shape(B, N, H, D, P)
+    q, k, v = _random_logical(B, N, H, D, seed=41)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    checks = []
+
+    xh, c = _guarded(shape.head_sharded, torch.bfloat16); checks.append(c)
+    sp.pack(qs, xh, shape)
+    kh, vh = (torch.empty(shape.head_sharded, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    sp.pack(ks, kh, shape)
+    sp.pack(vs, vh, shape)
+    oh, c = _guarded(shape.head_sharded, torch.bfloat16); checks.append(c)
+    lh, c = _guarded(shape.lse_shape, torch.float32); checks.append(c)
+    sp.attention(xh, kh, vh, oh, shape, lse=lh)
+    os_, c = _guarded(shape.seq_sharded, torch.bfloat16); checks.append(c)
+    sp.unpack(oh, os_, shape)
+    of, c = _guarded(shape.seq_sharded, torch.bfloat16); checks.append(c)
+    lf, c = _guarded(shape.lse_shape, torch.float32); checks.append(c)
+    sp.attention_seqsharded(qs, ks, vs, of, shape, lse=lf)
+    send, c = _guarded(shape.send_chunks, torch.bfloat16); checks.append(c)
+    sp.exchange_pack(qs[0], send, shape)
+    back, c = _guarded(shape.rank_shard, torch.bfloat16); checks.append(c)
+    sp.exchange_unpack(send, back, shape)
+
+    mask = _cube_mask(B, H, N, 0.3, seed=41)
+    words = torch.from_numpy(sp.sparse_mask_words(mask).view(np.int32)).cuda()
+    osp, c = _guarded(shape.seq_sharded, torch.bfloat16); checks.append(c)
+    sp.attention_sparse_seqsharded(qs, ks, vs, words, osp, shape)
+
+    q8, k8, v8, f = _fp8_inputs(B, N, H, D, seed=41)
+    dev8 = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, P))).cuda()
+            for x in (q8, k8, v8)]
+    fac = [torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda() for x in f]
+    o8, c = _guarded(shape.seq_sharded, torch.bfloat16); checks.append(c)
+    sp.attention_fp8_seqsharded(*dev8, *fac, o8, shape)
+
+    peer = sp.Shape(B, N, H, D, P)
+    o_list = []
+    for _ in range(P):
+        o, c = _guarded(peer.rank_shard, torch.bfloat16)
+        o_list.append(o)
+        checks.append(c)
+    q_list = [qs[r].clone() for r in range(P)]
+    for j in range(P):
+        kg = torch.empty(peer.send_chunks, dtype=torch.bfloat16, device="cuda")
+        vg = torch.empty_like(kg)
+        sends = []
+        for x in (ks, vs):
+            sx = []
+            for r in range(P):
+                buf = torch.empty(peer.send_chunks, dtype=torch.bfloat16, device="cuda")
+                sp.exchange_pack(x[r], buf, peer)
+                sx.append(buf)
+            sends.append(sx)
+        kg.copy_(torch.stack([sends[0][r][j] for r in range(P)]))
+        vg.copy_(torch.stack([sends[1][r][j] for r in range(P)]))
+        lp, c = _guarded((B, peer.Hl, peer.Np), torch.float32)
+        checks.append(c)
+        sp.attention_ulysses_peer(q_list, kg, vg, o_list, peer, j, lse=lp)
+    _status_ok()
+    for i, c in enumerate(checks):
+        c(f"output {i}")
+
+
 # ------------------------------------------------------------------ attention, small
 
 def test_tiny_config_every_row():

@@ -11,11 +11,23 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "attention.cuh"
 #include "permute.cuh"
 #include "sp.h"
 
 namespace {
+
+// One NVTX range per ABI call that enqueues work, so that a profiler's
+// timeline shows the C-ABI entry points; with no profiler attached a
+// push/pop pair is a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 __device__ int32_t g_status = 0;
 
@@ -435,6 +447,7 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns, int32_t *status) {
 extern "C" {
 
 sp_status sp_selftest_wait_timeout(uint64_t limit_ns, void *stream) {
+  NvtxRange range("sp_selftest_wait_timeout");
   if (limit_ns > 1000000000ull) limit_ns = 1000000000ull;
   int32_t *status = status_ptr();
   if (status == nullptr) return SP_ERR_CUDA;
@@ -450,28 +463,34 @@ int64_t sp_padded_tokens(int32_t N, int32_t P) {
 sp_status sp_check_shape(const sp_shape *shape) { return check_common(shape); }
 
 sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_pack");
   return permute(xs, xh, shape, stream, sp::kModePack);
 }
 
 sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_unpack");
   return permute(oh, os, shape, stream, sp::kModeUnpack);
 }
 
 sp_status sp_exchange_pack(const void *xs_r, void *send, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_exchange_pack");
   return permute(xs_r, send, shape, stream, sp::kModeExchangePack);
 }
 
 sp_status sp_exchange_unpack(const void *recv, void *os_r, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_exchange_unpack");
   return permute(recv, os_r, shape, stream, sp::kModeExchangeUnpack);
 }
 
 sp_status sp_attention(const void *qh, const void *kh, const void *vh, void *oh, float *lse,
                        const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_attention");
   return attention(qh, kh, vh, oh, lse, shape, stream, false);
 }
 
 sp_status sp_attention_seqsharded(const void *qs, const void *ks, const void *vs, void *os,
                                   float *lse, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_attention_seqsharded");
   return attention(qs, ks, vs, os, lse, shape, stream, true);
 }
 
@@ -479,6 +498,7 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
                                       const float *q_scale, const float *k_scale,
                                       const float *v_scale, void *os, float *lse,
                                       const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_attention_fp8_seqsharded");
   if (q_scale == nullptr || k_scale == nullptr || v_scale == nullptr) return SP_ERR_NULL;
   return attention(qs, ks, vs, os, lse, shape, stream, true, q_scale, k_scale, v_scale);
 }
@@ -486,6 +506,7 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
 sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const void *vs,
                                          const uint32_t *mask, void *os, float *lse,
                                          const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_attention_sparse_seqsharded");
   if (mask == nullptr) return SP_ERR_NULL;
   return attention(qs, ks, vs, os, lse, shape, stream, true, nullptr, nullptr, nullptr, mask);
 }
@@ -493,6 +514,7 @@ sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const v
 sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_group,
                                     const void *v_group, void *const *o_shards, float *lse,
                                     int32_t rank, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_attention_ulysses_peer");
   return attention_peer(q_shards, k_group, v_group, o_shards, lse, rank, shape, stream);
 }
 
@@ -527,6 +549,7 @@ sp_status sp_ipc_close(void *base) {
 }
 
 sp_status sp_device_status(void *stream) {
+  NvtxRange range("sp_device_status");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(cs) != cudaSuccess) return SP_ERR_CUDA;
   int32_t *status = status_ptr();
