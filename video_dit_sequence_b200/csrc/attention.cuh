@@ -241,7 +241,13 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
+  // Block-sparse kernel: 12 warps, so that its per-row mask state fits.  The
+  // third warpgroup (TMA, MMA and two idle warps) gives registers to the two
+  // softmax warpgroups: 384 x 168 at launch = 2 x 128 x 208 + 128 x 88, and
+  // each sub-partition holds 208 + 208 + 88 registers per lane (<= 512).
+  constexpr bool kSplitRegs = kSparse;
   if (warp == 8) {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");
     // ---------------------------------------------------------------- producer
     // One elected lane issues the TMA loads.  In the rank-major layout a
     // 128-token tile that crosses a shard boundary is two strided blocks,
@@ -369,6 +375,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       }
     }
   } else if (warp == 9) {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
       constexpr uint32_t idesc_qk = kF8 ? make_idesc_e4m3(128, 128, 0, 0)
@@ -474,7 +481,10 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       }
     }
     __syncwarp();
+  } else if (kSplitRegs && warp >= 10) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");  // idle: registers to the softmax
   } else {
+    if constexpr (kSplitRegs) asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
     // ---------------------------------------------------------------- softmax
     const int t = warp >> 2;           // query tile
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
@@ -716,7 +726,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tmQ,
 
 // Block-sparse attention (bf16, D = 128): the sequence-sharded fused call
 // with a mask of selected 64-token key cubes per 64-token query cube.
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 attention_sparse_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,

@@ -326,7 +326,8 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
     cudaError_t e = set_smem_once(sp::attention_sparse_kernel, C::kSmemBytes, attr_set);
     if (e != cudaSuccess) return SP_ERR_CUDA;
     dim3 grid((Np + 2 * C::kBM - 1) / (2 * C::kBM), H, B);
-    sp::attention_sparse_kernel<<<grid, C::kThreads, C::kSmemBytes, cs>>>(mq, mk, mv, p);
+    // 12 warps: the block-sparse kernel splits registers between warpgroups
+    sp::attention_sparse_kernel<<<grid, 384, C::kSmemBytes, cs>>>(mq, mk, mv, p);
     return launch_status(cudaGetLastError());
   }
   cudaError_t e = f8        ? launch_attention<128, true>(mq, mk, mv, p, B, cs)
