@@ -172,3 +172,38 @@ def test_binding_refuses_mixed_devices(lib):
     b = torch.zeros(shape.head_sharded, dtype=torch.bfloat16, device="meta")
     with pytest.raises((ValueError, TypeError)):
         sp.pack(a, b, shape)
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/sp.h compiles as strict C99 and a C program links against
+    libsp.so and calls its host-only entry points: the boundary needs no C++,
+    Python or torch."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "sp.h"
+int main(void) {
+  sp_shape ok = {1, 75601, 40, 128, 8, 0.0f};
+  sp_shape bad = {1, 1000, 40, 128, 3, 0.0f};
+  printf("%lld %d %d %s\n", (long long)sp_padded_tokens(75601, 8), (int)sp_check_shape(&ok),
+         (int)sp_check_shape(&bad), sp_status_str(SP_ERR_HEADS_NOT_DIVISIBLE));
+  return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.join(ROOT, "video_dit_sequence_b200")
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src),
+                        "-L", libdir, "-lsp", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    padded, st_ok, st_bad, text = out.stdout.split(" ", 3)
+    assert int(padded) == 75608 and int(st_ok) == sp.SP_OK
+    assert int(st_bad) == sp.SP_ERR_HEADS_NOT_DIVISIBLE and text.strip()
