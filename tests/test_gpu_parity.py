@@ -582,6 +582,77 @@ def test_host_pipeline_matches_direct_calls():
         assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
 
 
+C_PROGRAM = r"""
+/* The fused call from a C program: device memory from the CUDA runtime, the
+ * computation through sp.h, no Python or torch on the path. */
+#include <stdio.h>
+#include <stdlib.h>
+#include <cuda_runtime.h>
+#include "sp.h"
+
+int main(int argc, char **argv) {
+  if (argc != 8) return 2;
+  sp_shape s = {atoi(argv[1]), atoi(argv[2]), atoi(argv[3]), atoi(argv[4]), atoi(argv[5]), 0.0f};
+  const long long n = (long long)s.P * s.B * ((s.N + s.P - 1) / s.P) * s.H * s.D;
+  const size_t bytes = (size_t)n * 2;
+  unsigned short *h = (unsigned short *)malloc(3 * bytes);
+  FILE *f = fopen(argv[6], "rb");
+  if (!h || !f || fread(h, 1, 3 * bytes, f) != 3 * bytes) return 3;
+  fclose(f);
+  void *q, *k, *v, *o;
+  if (cudaMalloc(&q, bytes) || cudaMalloc(&k, bytes) || cudaMalloc(&v, bytes) ||
+      cudaMalloc(&o, bytes))
+    return 4;
+  cudaMemcpy(q, h, bytes, cudaMemcpyHostToDevice);
+  cudaMemcpy(k, h + n, bytes, cudaMemcpyHostToDevice);
+  cudaMemcpy(v, h + 2 * n, bytes, cudaMemcpyHostToDevice);
+  sp_status st = sp_attention_seqsharded(q, k, v, o, NULL, &s, NULL);
+  if (st != SP_OK) { fprintf(stderr, "%s\n", sp_status_str(st)); return 5; }
+  st = sp_device_status(NULL);
+  if (st != SP_OK) { fprintf(stderr, "%s\n", sp_status_str(st)); return 6; }
+  cudaMemcpy(h, o, bytes, cudaMemcpyDeviceToHost);
+  f = fopen(argv[7], "wb");
+  if (!f || fwrite(h, 1, bytes, f) != bytes) return 7;
+  fclose(f);
+  cudaFree(q); cudaFree(k); cudaFree(v); cudaFree(o);
+  free(h);
+  return 0;
+}
+"""
+
+
+def test_c_program_runs_the_fused_call(tmp_path):
+    """A C program (CUDA runtime for memory, sp.h for the work) gives the same
+    bits as the call through the Python binding, and the oracle agrees."""
+    import os
+    import shutil
+    import subprocess
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.join(root, "video_dit_sequence_b200")
+    src = tmp_path / "fused.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "fused"
+    r = subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-x", "cu",
+                        "-I", os.path.join(root, "include"), "-o", str(exe),
+                        str(src), "-L", libdir, "-lsp", f"-Xlinker=-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    B, N, H, D, P = 1, 1000, 4, 128, 2
+    q, k, v = _random_logical(B, N, H, D, seed=61)
+    shards = [np.ascontiguousarray(synth.to_seq_shards(x, P)) for x in (q, k, v)]
+    (tmp_path / "in.bin").write_bytes(b"".join(x.tobytes() for x in shards))
+    run = subprocess.run([str(exe), str(B), str(N), str(H), str(D), str(P),
+                          str(tmp_path / "in.bin"), str(tmp_path / "out.bin")],
+                         capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    got = np.frombuffer((tmp_path / "out.bin").read_bytes(), dtype=np.uint16)
+    want, _ = _run_fused(q, k, v, P)
+    assert np.array_equal(got, want.reshape(-1))
+    rows = np.array([(0, h, i) for h in range(H) for i in range(0, N, 7)], dtype=np.int64)
+    _check_rows(got.reshape(want.shape), q, k, v, rows, P, "C program")
+
+
 @pytest.mark.parametrize("scale", [0.05, 0.2])
 def test_explicit_scale(scale):
     B, N, H, D, P = 1, 900, 2, 64, 2
