@@ -21,6 +21,9 @@ What it computes, and the passages it follows:
   over cubes of consecutive tokens (the sparse stage of video sparse
   attention, which the FastVideo page names with 64-token tiles), for the
   block-sparse kernel.
+* ``linear_rows`` -- the projection in front of attention (hidden state to
+  q, k and v), a plain fp64 matrix product, for the projection kernel whose
+  epilogue writes the attention layouts.
 * ``attention_rows`` -- the unsharded softmax(q K^T scale) V of one head,
   two-pass exact softmax in fp64; the sequence-parallel result must equal it
   for every degree (LTX-2 "Multi-GPU Inference" README, Capabilities table:
@@ -75,6 +78,8 @@ def _bind(path: str):
     lib.sp_oracle_attention_rows_masked.argtypes = [
         vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_double, i64, vp, vp, vp, ctypes.c_int]
     lib.sp_oracle_attention_rows_masked.restype = ctypes.c_int
+    lib.sp_oracle_linear_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, vp, ctypes.c_int]
+    lib.sp_oracle_linear_rows.restype = ctypes.c_int
     lib.sp_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
     lib.sp_oracle_e4m3_value.restype = ctypes.c_double
     return lib
@@ -254,6 +259,30 @@ def attention_rows_masked(q, k, v, mask, rows, scale: float = 0.0, cube: int = 6
     if rc != 0:
         raise RuntimeError(f"oracle attention failed ({rc})")
     return o, lse
+
+
+def linear_rows(x, w, bias, rows, threads: Optional[int] = None, lib=None):
+    """fp64 linear layer on bf16 inputs for the requested rows:
+    y[r][c] = sum_k x[rows[r]][k] * w[c][k] (+ bias[c]).  x: uint16 [M][K],
+    w: uint16 [nout][K], bias: uint16 [nout] or None.  Returns [R][nout]."""
+    assert x.dtype == np.uint16 and w.dtype == np.uint16 and x.ndim == 2 and w.ndim == 2
+    M, K = x.shape
+    nout, K2 = w.shape
+    assert K2 == K
+    x, w = np.ascontiguousarray(x), np.ascontiguousarray(w)
+    if bias is not None:
+        bias = np.ascontiguousarray(bias, dtype=np.uint16)
+        assert bias.shape == (nout,)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1)
+    y = np.empty((rows.size, nout), dtype=np.float64)
+    if threads is None:
+        threads = max(1, len(os.sched_getaffinity(0)))
+    rc = (lib or _load()).sp_oracle_linear_rows(
+        x.ctypes.data, w.ctypes.data, None if bias is None else bias.ctypes.data, M, K, nout,
+        rows.size, rows.ctypes.data, y.ctypes.data, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle linear failed ({rc})")
+    return y
 
 
 def attention_full(q, k, v, scale: float = 0.0, threads: Optional[int] = None,

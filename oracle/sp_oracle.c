@@ -35,6 +35,10 @@
  *    block of consecutive tokens, V one per channel (the contraction of q.k
  *    runs over channels and that of p.v over tokens, so these factors come
  *    out of the sums).
+ *  - the projection in front of attention (the step next to it in a DiT
+ *    block, which the pages never describe): one linear layer from each
+ *    token's hidden state to its q, k and v, with no rotary embedding or
+ *    normalisation.
  *  - block-sparse attention (the sparse stage of video sparse attention, named
  *    on "Pair two NVIDIA DGX Sparks" with 64-token tiles and sparsity 0.8,
  *    its block selection not defined there): a query attends only the keys
@@ -329,6 +333,70 @@ int sp_oracle_attention_rows_masked(const uint16_t *q, const uint16_t *k, const 
     J.nrows = nrows; J.rows = rows;
     J.out_o = out_o; J.out_lse = out_lse;
     return attention_rows_impl(&J, nthreads);
+}
+
+/*
+ * The projection in front of attention: a linear layer that maps each
+ * token's hidden state to its q, k and v (the transformer block around the
+ * attention; the pages describe no more of it, so no rotary embedding or
+ * normalisation is applied).  For every requested row m:
+ *     y[m][c] = sum_k x[m][k] * w[c][k]  (+ bias[c])     c = 0 .. nout-1
+ * with the output features laid out as q (H*D), then k, then v, a feature's
+ * weights in one row of w as a linear layer stores them.
+ * x [M][K], w [nout][K], bias [nout] or NULL: bf16 words; rows: nrows row
+ * indices; y: nrows x nout doubles.
+ */
+typedef struct {
+    const uint16_t *x, *w, *bias;
+    int64_t M, K, nout, nrows;
+    const int64_t *rows;
+    double *y;
+    int64_t next;
+    pthread_mutex_t lock;
+} linear_job_t;
+
+static void *linear_worker(void *arg) {
+    linear_job_t *J = (linear_job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t r = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (r >= J->nrows) break;
+        const uint16_t *xr = J->x + J->rows[r] * J->K;
+        double *yr = J->y + r * J->nout;
+        for (int64_t c = 0; c < J->nout; ++c) {
+            const uint16_t *wc = J->w + c * J->K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < J->K; ++k) acc += bf16_to_f64(xr[k]) * bf16_to_f64(wc[k]);
+            yr[c] = acc + (J->bias ? bf16_to_f64(J->bias[c]) : 0.0);
+        }
+    }
+    return NULL;
+}
+
+int sp_oracle_linear_rows(const uint16_t *x, const uint16_t *w, const uint16_t *bias,
+                          int64_t M, int64_t K, int64_t nout, int64_t nrows,
+                          const int64_t *rows, double *y, int nthreads) {
+    if (M < 1 || K < 1 || nout < 1 || nrows < 0) return -1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= M) return -1;
+    linear_job_t J;
+    memset(&J, 0, sizeof(J));
+    J.x = x; J.w = w; J.bias = bias;
+    J.M = M; J.K = K; J.nout = nout; J.nrows = nrows; J.rows = rows; J.y = y;
+    pthread_mutex_init(&J.lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 512) nthreads = 512;
+    pthread_t th[512];
+    int started = 0;
+    for (int t = 1; t < nthreads; ++t) {
+        if (pthread_create(&th[started], NULL, linear_worker, &J) != 0) break;
+        ++started;
+    }
+    linear_worker(&J);
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
 }
 
 static int attention_rows_impl(attn_job_t *JP, int nthreads) {

@@ -423,6 +423,30 @@ def check_masked_attention(lib=None):
     assert np.any(~sel[0, 1, 2].astype(bool))
 
 
+def check_linear_projection(lib=None):
+    """The projection oracle: a worked 2 x 2 example by hand, the identity
+    weight returning x exactly, and numpy's fp64 x @ w.T + b on random
+    shapes (row subsets in any order, with and without a bias)."""
+    x = synth.f32_to_bf16(np.array([[1, 2], [3, 4]], np.float32))
+    w = synth.f32_to_bf16(np.array([[1, 0], [1, 1], [0, -2]], np.float32))
+    b = synth.f32_to_bf16(np.array([0.5, -1, 0.25], np.float32))
+    y = oracle.linear_rows(x, w, b, [1, 0], threads=1, lib=lib)
+    assert np.array_equal(y, np.array([[3.5, 6.0, -7.75], [1.5, 2.0, -3.75]]))
+    rng = np.random.default_rng(RNG_SEED + 19)
+    xi = _bf16_normal((9, 16), rng)
+    eye = synth.f32_to_bf16(np.eye(16, dtype=np.float32))
+    assert np.array_equal(oracle.linear_rows(xi, eye, None, np.arange(9), threads=2, lib=lib),
+                          _f64(xi))
+    for (M, K, nout) in [(7, 33, 12), (20, 64, 48)]:
+        xr, wr = _bf16_normal((M, K), rng), _bf16_normal((nout, K), rng, 0.1)
+        br = _bf16_normal((nout,), rng)
+        rows = rng.permutation(M)[: M // 2]
+        for bias in (None, br):
+            got = oracle.linear_rows(xr, wr, bias, rows, threads=2, lib=lib)
+            want = _f64(xr)[rows] @ _f64(wr).T + (0.0 if bias is None else _f64(bias))
+            assert np.max(np.abs(got - want)) < 1e-12 * max(1.0, np.max(np.abs(want)))
+
+
 PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
                check_unpack_returns_shards, check_pack_degree_one_is_copy,
                check_exchange_chunks_hold_head_groups,
@@ -431,5 +455,6 @@ ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one
                     check_closed_forms, check_dominant_key, check_invariances,
                     check_two_token_example, check_rows_api,
                     check_e4m3_decode_matches_torch, check_fp8_attention_reduces_to_bf16,
-                    check_fp8_block_factors_match_dequantized_bf16, check_masked_attention]
+                    check_fp8_block_factors_match_dequantized_bf16, check_masked_attention,
+                    check_linear_projection]
 ALL_CHECKS = PACK_CHECKS + ATTENTION_CHECKS

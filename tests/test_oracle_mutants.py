@@ -63,6 +63,14 @@ MUTANTS = [
      "if (sel && !sel[i / J->cube]) {"),
     ("mask-head-ignored", "J->mask + (bh * J->ncube + i / J->cube) * J->ncube",
      "J->mask + (b * H * J->ncube + i / J->cube) * J->ncube"),
+    ("linear-bias-dropped", "yr[c] = acc + (J->bias ? bf16_to_f64(J->bias[c]) : 0.0);",
+     "yr[c] = acc;"),
+    ("linear-weight-row-of-next-feature", "const uint16_t *wc = J->w + c * J->K;",
+     "const uint16_t *wc = J->w + ((c + 1) % J->nout) * J->K;"),
+    ("linear-drops-last-input", "for (int64_t k = 0; k < J->K; ++k) acc +=",
+     "for (int64_t k = 0; k + 1 < J->K; ++k) acc +="),
+    ("linear-row-ignored", "const uint16_t *xr = J->x + J->rows[r] * J->K;",
+     "const uint16_t *xr = J->x + r * J->K;"),
     ("mask-empty-row-not-zero", "        if (J->out_lse) J->out_lse[r] = -INFINITY;\n        return;",
      "        if (J->out_lse) J->out_lse[r] = -INFINITY;\n        o[0] = 1.0;\n        return;"),
 ]
