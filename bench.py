@@ -474,6 +474,23 @@ def run_ours(args):
                                                                 stream=stream))
         sparse_flops = 4.0 * synth.attended_pairs(mask, s.N) * s.D
         del words, o_sp
+    # the projection in front of attention (hidden -> q, k, v) with its
+    # epilogue writing the sequence-sharded layout; cuBLAS on the same GEMM
+    # (x @ w^T, one contiguous output) timed beside it
+    t_proj = t_cublas = None
+    if not args.no_proj and s.D == 128:
+        hidden = s.H * s.D
+        M = s.P * s.B * shape.Nl
+        gen = torch.Generator(device=dev).manual_seed(5)
+        xw = torch.randn(M, hidden, device=dev, generator=gen).to(torch.bfloat16)
+        ww = (torch.randn(3 * hidden, hidden, device=dev, generator=gen)
+              / math.sqrt(hidden)).to(torch.bfloat16)
+        pq, pkk, pv = (torch.empty_like(qs) for _ in range(3))
+        t_proj = timed(lambda: sp.qkv_projection(xw, ww, None, pq, pkk, pv, shape, stream=stream))
+        yc = torch.empty(M, 3 * hidden, dtype=torch.bfloat16, device=dev)
+        t_cublas = timed(lambda: torch.matmul(xw, ww.t(), out=yc))
+        proj_flops = 2.0 * M * hidden * 3 * hidden
+        del xw, ww, pq, pkk, pv, yc
     if sp.device_status(stream) != sp.SP_OK:
         raise SystemExit("device status not ok after the unfused rows")
     pack_gbs = 2 * tensor_bytes / (t_pack * 1e-3) / 1e9
@@ -497,6 +514,12 @@ def run_ours(args):
             "ms": t_sparse, "speedup_vs_dense": per_launch_ms / t_sparse,
             "attended_TFLOP/s": sparse_flops / (t_sparse * 1e-3) / 1e12,
             "mask": "64-token cubes, density 0.2, one selection per 4 query cubes (synthetic)"},
+        "qkv_projection": None if t_proj is None else {
+            "ms": t_proj, "TFLOP/s": proj_flops / (t_proj * 1e-3) / 1e12,
+            "frac": proj_flops / (t_proj * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "cublas_ms": t_cublas, "cublas_TFLOP/s": proj_flops / (t_cublas * 1e-3) / 1e12,
+            "what": f"hidden {s.H * s.D} -> q, k, v (bf16) written as sequence shards; cuBLAS: "
+                    "the same GEMM into one [M][3HD] matrix"},
         "unfused_step_ms": 3 * t_pack + t_attn + t_unpack,
         "fused_step_ms": per_launch_ms,
     }
@@ -578,6 +601,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 row")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse row")
+    ap.add_argument("--no-proj", action="store_true", help="skip the projection row")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override N (same heads, head dim and degree); for profiling captures")
     ap.add_argument("--traffic-bytes", type=float, default=None,

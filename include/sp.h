@@ -170,6 +170,35 @@ sp_status sp_attention_fp8_seqsharded(const void *qs, const void *ks, const void
                                       const float *v_scale, void *os, float *lse,
                                       const sp_shape *shape, void *stream);
 
+/* Where sp_qkv_projection writes q, k and v. */
+typedef enum {
+  SP_QKV_SEQ_SHARDED = 0,  /* [P][B][Nl][H][D]: the fused attention's input */
+  SP_QKV_HEAD_SHARDED = 1, /* [P][B][Np][Hl][D]: sp_attention's input (the pack folded in) */
+  SP_QKV_SEND_CHUNKS = 2   /* [P][B][Nl][Hl][D] of one rank: its exchange pack folded in */
+} sp_qkv_layout;
+
+/* The projection in front of attention: each token's hidden state to its q,
+ * k and v, y[m][c] = sum_k x[m][k] * w[c][k] (+ bias[c]) with the 3*H*D output
+ * features ordered q, k, v (head-major, D per head) and a feature's weights in
+ * one row of w, as a linear layer stores them.  The pages never describe the
+ * transformer block around the attention; this is its plainest reading (no
+ * rotary embedding or normalisation).  The epilogue stores y straight into
+ * the layout `layout` names, so no permutation pass runs between the
+ * projection and attention.  fp32 accumulation, bf16 output (round to
+ * nearest even).
+ * x: device bf16 [P][B][Nl][hidden], the sequence-sharded hidden states
+ *   (padding slots included), or for SP_QKV_SEND_CHUNKS one rank's
+ *   [B][Nl][hidden]; 16-byte aligned; hidden a multiple of 8.
+ * w: device bf16 [3*H*D][hidden]; bias: device bf16 [3*H*D] or NULL.
+ * q, k, v: device bf16 outputs in `layout`, 16-byte aligned, written in full
+ *   (padding slots hold the projection of x's padding rows).
+ * shape: {B, N, H, D, P}; the head-split layouts need H % P == 0.
+ * Errors: SP_ERR_NULL, SP_ERR_ALIGN, SP_ERR_SHAPE (layout, hidden, sizes),
+ * SP_ERR_HEADS_NOT_DIVISIBLE, SP_ERR_UNSUPPORTED_D, SP_ERR_CUDA. */
+sp_status sp_qkv_projection(const void *x, const void *w, const void *bias, void *q, void *k,
+                            void *v, int32_t hidden, int32_t layout, const sp_shape *shape,
+                            void *stream);
+
 /* Tokens per cube of the block-sparse call's mask. */
 #define SP_SPARSE_CUBE 64
 

@@ -142,6 +142,18 @@ def test_argument_errors_return_before_launch(lib):
     assert sparse(C + 2) == sp.SP_ERR_ALIGN
     assert sparse(C, sp.Shape(1, 1000, 4, 64, 2)) == sp.SP_ERR_UNSUPPORTED_D
     assert sparse(C, sp.Shape(1, 128 * 16384 + 1, 1, 128, 1)) == sp.SP_ERR_SHAPE
+    proj = lambda x, w, b, q, k, v, hidden, layout, shp=sp.Shape(1, 1000, 4, 128, 2): \
+        lib.sp_qkv_projection(*[ctypes.c_void_p(t) if t else None for t in (x, w, b, q, k, v)],
+                              hidden, layout, ctypes.byref(shp.c()), None)
+    assert proj(A, A, 0, B_, B_, 0, 512, 0) == sp.SP_ERR_NULL
+    assert proj(A, A, 0, B_, B_, B_ + 8, 512, 0) == sp.SP_ERR_ALIGN
+    assert proj(A, A, C + 1, B_, B_, B_, 512, 0) == sp.SP_ERR_ALIGN          # bf16 bias
+    assert proj(A, A, 0, B_, B_, B_, 500, 0) == sp.SP_ERR_SHAPE              # hidden % 8
+    assert proj(A, A, 0, B_, B_, B_, 512, 3) == sp.SP_ERR_SHAPE              # no such layout
+    assert proj(A, A, 0, B_, B_, B_, 512, 1, sp.Shape(1, 1000, 6, 128, 4)) == \
+        sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    assert proj(A, A, 0, B_, B_, B_, 512, 0, sp.Shape(1, 1000, 6, 96, 4)) == \
+        sp.SP_ERR_UNSUPPORTED_D
     h = (ctypes.c_uint8 * sp.IPC_HANDLE_BYTES)()
     off = ctypes.c_int64()
     base = ctypes.c_void_p()

@@ -394,6 +394,80 @@ def test_sparse_cta_with_no_selected_tile():
     assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]), "junk bits")
 
 
+# ------------------------------------------------------------------ projection
+
+def _proj_inputs(B, N, H, D, P, hidden, seed, bias=True):
+    """Sequence-sharded hidden states [P][B][Nl][hidden] (padding slots zero),
+    weights [3HD][hidden] scaled by 1/sqrt(hidden), an optional bias."""
+    Nl = -(-N // P)
+    x = synth.normal_bf16(seed, 0, 0, P * B * Nl * hidden).reshape(P, B, Nl, hidden)
+    tok = np.arange(P)[:, None] * Nl + np.arange(Nl)[None, :]            # [P][Nl]
+    x[np.broadcast_to((tok >= N)[:, None, :], (P, B, Nl))] = 0
+    w = synth.normal_bf16(seed, 1, 0, 3 * H * D * hidden, mul=1.0 / math.sqrt(hidden))
+    w = w.reshape(3 * H * D, hidden)
+    b = synth.normal_bf16(seed, 2, 0, 3 * H * D, mul=0.1) if bias else None
+    return x, w, b
+
+
+def _run_proj(x, w, b, shape, layout):
+    out_shape = {"seq": shape.seq_sharded, "head": shape.head_sharded,
+                 "send": shape.send_chunks}[layout]
+    outs = [torch.full(out_shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+            for _ in range(3)]
+    sp.qkv_projection(to_dev(x), to_dev(w), None if b is None else to_dev(b), *outs, shape,
+                      layout=layout)
+    _status_ok()
+    return [to_host(o) for o in outs]
+
+
+def _check_proj(seq, x, w, b, rows, where):
+    """Rows of the sequence-sharded q/k/v output against the fp64 oracle: the
+    bf16 rounding of the output (2^-9 relative) plus fp32 accumulation."""
+    hidden = x.shape[-1]
+    X = x.reshape(-1, hidden)
+    ref = oracle.linear_rows(X, w, b, rows)
+    got = np.concatenate([synth.bf16_to_f32(t.reshape(X.shape[0], -1)[rows]) for t in seq],
+                         axis=1).astype(np.float64)
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-4 * np.max(np.abs(ref))
+    assert np.all(err <= bound), (where, float((err - bound).max()))
+
+
+@pytest.mark.parametrize("B,N,H,D,P,hidden,bias", [
+    (1, 1000, 4, 128, 2, 512, True), (2, 333, 6, 64, 3, 200, False),
+    (1, 4096, 12, 128, 4, 1536, True), (3, 130, 2, 64, 1, 72, True)])
+def test_qkv_projection_layouts(B, N, H, D, P, hidden, bias):
+    """The projection against the fp64 oracle on every row, and its three
+    layouts bit for bit against the pinned pack and exchange pack of the
+    sequence-sharded result (ragged rows, features and hidden sizes)."""
+    shape = sp.Shape(B, N, H, D, P)
+    x, w, b = _proj_inputs(B, N, H, D, P, hidden, seed=hidden + N, bias=bias)
+    seq = _run_proj(x, w, b, shape, "seq")
+    M = P * B * shape.Nl
+    _check_proj(seq, x, w, b, np.arange(M), f"projection {B},{N},{H},{D},{P},{hidden}")
+    head = _run_proj(x, w, b, shape, "head")
+    for t in range(3):
+        assert np.array_equal(head[t], oracle.pack(seq[t].reshape(shape.seq_sharded), N))
+    for r in range(P):
+        send = _run_proj(np.ascontiguousarray(x[r]), w, b, shape, "send")
+        for t in range(3):
+            want = oracle.exchange_pack(seq[t].reshape(shape.seq_sharded)[r], N, P)
+            assert np.array_equal(send[t], want)
+
+
+def test_qkv_projection_720p_sampled_rows():
+    """The 720p-shaped projection (75,600 tokens, hidden 5,120, 15,360
+    features) on sampled rows against the oracle."""
+    cfg = synth.CONFIGS["720p"]
+    s = cfg.shape
+    shape = sp.Shape(s.B, s.N, s.H, s.D, s.P)
+    x, w, b = _proj_inputs(s.B, s.N, s.H, s.D, s.P, s.H * s.D, seed=71)
+    seq = _run_proj(x, w, b, shape, "seq")
+    rows = np.unique(np.concatenate([[0, s.N - 1, 18899, 18900],
+                                     np.random.default_rng(71).integers(0, s.N, 40)]))
+    _check_proj(seq, x, w, b, rows, "projection 720p")
+
+
 # ------------------------------------------------------------------ guard bands
 
 GUARD = 4096  # elements of sentinel after every output buffer

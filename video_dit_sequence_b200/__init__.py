@@ -43,7 +43,7 @@ EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout",
             "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded",
             "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close",
-            "sp_attention_sparse_seqsharded")
+            "sp_attention_sparse_seqsharded", "sp_qkv_projection")
 
 
 class sp_shape(ctypes.Structure):
@@ -84,6 +84,9 @@ def load(path: str = LIB_PATH):
         f.restype = ctypes.c_int
     lib.sp_attention_fp8_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sp_p, vp]
     lib.sp_attention_fp8_seqsharded.restype = ctypes.c_int
+    lib.sp_qkv_projection.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int32, ctypes.c_int32,
+                                      sp_p, vp]
+    lib.sp_qkv_projection.restype = ctypes.c_int
     lib.sp_attention_sparse_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, sp_p, vp]
     lib.sp_attention_sparse_seqsharded.restype = ctypes.c_int
     lib.sp_attention_ulysses_peer.argtypes = [
@@ -365,6 +368,31 @@ class UlyssesRank:
         out = torch.empty(self.shape.rank_shard, dtype=back.dtype, device=back.device)
         exchange_unpack(back, out, self.shape, stream)
         return out
+
+
+QKV_LAYOUTS = {"seq": 0, "head": 1, "send": 2}   # sp_qkv_layout
+
+
+def qkv_projection(x, w, bias, q, k, v, shape: Shape, layout: str = "seq", stream=None):
+    """The projection in front of attention (sp_qkv_projection), arguments in
+    the C order: x the sequence-sharded hidden states [P][B][Nl][hidden] (one
+    rank's [B][Nl][hidden] for layout "send"), w [3*H*D][hidden], bias
+    [3*H*D] or None, all bf16; q, k, v receive the projection in `layout`:
+    "seq" [P][B][Nl][H][D], "head" [P][B][Np][Hl][D] or "send"
+    [P][B][Nl][Hl][D]."""
+    torch = _torch()
+    if layout not in QKV_LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(QKV_LAYOUTS)}")
+    hidden = int(w.shape[-1])
+    rows = shape.rank_shard[:2] if layout == "send" else shape.seq_sharded[:3]
+    out = {"seq": shape.seq_sharded, "head": shape.head_sharded, "send": shape.send_chunks}[layout]
+    s = shape.c()
+    with _same_device(x, w, bias, q, k, v):
+        _check(load().sp_qkv_projection(
+            _ptr(x, tuple(rows) + (hidden,), "x"), _ptr(w, (3 * shape.H * shape.D, hidden), "w"),
+            _ptr(bias, (3 * shape.H * shape.D,), "bias"), _ptr(q, out, "q"), _ptr(k, out, "k"),
+            _ptr(v, out, "v"), hidden, QKV_LAYOUTS[layout], ctypes.byref(s),
+            _stream(stream, x.device)), "sp_qkv_projection")
 
 
 SPARSE_CUBE = 64         # SP_SPARSE_CUBE

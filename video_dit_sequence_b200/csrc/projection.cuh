@@ -1,0 +1,261 @@
+// projection.cuh -- the projection in front of attention (each token's
+// hidden state to its q, k and v) as a tcgen05 GEMM whose epilogue writes
+// q, k and v straight into the layout the attention path reads.
+//
+// What it computes: y[m][c] = sum_k x[m][k] * w[c][k] (+ bias[c]) for the
+// rows m of x and the 3*H*D output features c (q, then k, then v; a
+// feature's weights are one row of w, as a linear layer stores them).  The
+// pages never describe the transformer block around the attention, so no
+// rotary embedding or normalisation is applied.  Feature c is element d of
+// head h of tensor t (c = t*H*D + h*D + d); row m is a token of the
+// sequence-sharded hidden states, and the epilogue stores y[m][c] at
+//   kProjSeqSharded  [P][B][Nl][H][D]   (the fused attention's input),
+//   kProjHeadSharded [P][B][Np][Hl][D]  (the pack folded in),
+//   kProjSendChunks  [P][B][Nl][Hl][D]  (one rank's exchange pack folded in),
+// so that no permutation pass runs between the projection and attention.
+//
+// A tile of y is 128 x 256: a TMA warp streams 64-wide K slices of x (128
+// rows) and w (256 rows) through a 4-stage ring, one thread issues
+// 128 x 256 x 16 tcgen05 MMAs into a 256-column TMEM accumulator, and four
+// epilogue warps (one per TMEM lane quarter) add the bias, round to bf16 and
+// store 64-byte runs.  The kernel is persistent, one CTA per SM, with two
+// accumulators so that one tile's epilogue overlaps the next tile's MMAs.
+// Tiles are ordered in groups of kProjGroupM row blocks so that CTAs working
+// at the same time share their x and w slices in L2.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace sp {
+
+enum ProjLayout { kProjSeqSharded = 0, kProjHeadSharded = 1, kProjSendChunks = 2 };
+
+struct ProjParams {
+  int32_t M, K, nout;        // rows of x, hidden size, 3*H*D
+  int32_t H, D, Hl;          // heads, head dim, heads per group (H / P)
+  int32_t P, B, Nl, Np;      // degree, batch, tokens per rank, P * Nl
+  int32_t layout;            // ProjLayout
+  int32_t tiles_m, tiles_n;  // ceil(M / 128), ceil(nout / 256)
+  __nv_bfloat16 *out[3];     // q, k, v
+  const __nv_bfloat16 *bias; // [nout] or null
+  int32_t *status;
+};
+
+constexpr int kProjBM = 128;
+constexpr int kProjBN = 256;
+constexpr int kProjBK = 64;                       // bf16 elements: one 128-byte row
+constexpr int kProjStages = 4;
+constexpr int kProjGroupM = 16;
+constexpr int kProjABytes = kProjBM * 128;        // 16 KB
+constexpr int kProjBBytes = kProjBN * 128;        // 32 KB
+constexpr int kProjStageBytes = kProjABytes + kProjBBytes;
+constexpr int kProjOffBar = kProjStages * kProjStageBytes;
+constexpr int kProjOffMisc = kProjOffBar + (2 * kProjStages + 4) * 8;
+constexpr int kProjSmemBytes = kProjOffMisc + 16 + 1024;
+constexpr int kProjThreads = 192;                 // TMA, MMA, four epilogue warps
+constexpr uint32_t kProjTmemCols = 512;               // two 256-column accumulators
+constexpr uint64_t kProjWaitNs = 2000000000ull;  // 2 s per wait
+constexpr int32_t kProjStatusTimeout = 7;         // SP_ERR_TIMEOUT
+
+// Tile t of the y matrix as (row block, column block): groups of
+// kProjGroupM row blocks, the column blocks of a group inside it.
+__device__ __forceinline__ void proj_tile(int t, int tiles_m, int tiles_n, int &tm, int &tn) {
+  const int per_group = kProjGroupM * tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * kProjGroupM;
+  const int gm = min(kProjGroupM, tiles_m - first_m);
+  const int in_group = t - g * per_group;
+  tm = first_m + in_group % gm;
+  tn = in_group / gm;
+}
+
+// Persistent: CTA c computes tiles c, c + gridDim.x, ...  The K ring runs on
+// across tiles, and two TMEM accumulators let the epilogue of one tile
+// overlap the MMAs of the next.
+__global__ void __launch_bounds__(kProjThreads, 1)
+qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
+                      const __grid_constant__ CUtensorMap tmW, const __grid_constant__ ProjParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t *sptr = smem_raw + (sbase - raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = p.tiles_m * p.tiles_n;
+  const int nk = (p.K + kProjBK - 1) / kProjBK;
+
+  const uint32_t bar_full = sbase + kProjOffBar;                 // [stages]
+  const uint32_t bar_empty = bar_full + 8 * kProjStages;          // [stages]
+  const uint32_t bar_acc_full = bar_empty + 8 * kProjStages;      // [2]
+  const uint32_t bar_acc_empty = bar_acc_full + 16;               // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + kProjOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kProjStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_acc_full + 8 * a, 1);
+      mbar_init(bar_acc_empty + 8 * a, 4);      // one arrival per epilogue warp
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kProjTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  bool ok = true;
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&tmX);
+      prefetch_tmap(&tmW);
+      const uint64_t pol = policy_evict_last();
+      int it = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        int tm, tn;
+        proj_tile(t, p.tiles_m, p.tiles_n, tm, tn);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kProjStages;
+          ok = mbar_wait(bar_empty + 8 * s, ((it / kProjStages) & 1) ^ 1u, abort_flag, kProjWaitNs);
+          if (!ok) break;
+          const uint32_t dst = sbase + s * kProjStageBytes;
+          mbar_arrive_expect_tx(bar_full + 8 * s, kProjStageBytes);
+          tma_load_4d(dst, &tmX, bar_full + 8 * s, kb * kProjBK, tm * kProjBM, 0, 0, pol);
+          tma_load_4d(dst + kProjABytes, &tmW, bar_full + 8 * s, kb * kProjBK, tn * kProjBN, 0, 0,
+                      pol);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_bf16(kProjBM, kProjBN, 0, 0);
+      const uint64_t dA = make_sdesc_sw128(sbase, 16, 1024);
+      const uint64_t dB = make_sdesc_sw128(sbase + kProjABytes, 16, 1024);
+      int it = 0, n = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++n) {
+        const int a = n & 1;                      // accumulator of this tile
+        ok = mbar_wait(bar_acc_empty + 8 * a, ((n >> 1) & 1) ^ 1u, abort_flag, kProjWaitNs);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(a * kProjBN);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % kProjStages;
+          ok = mbar_wait(bar_full + 8 * s, (it / kProjStages) & 1, abort_flag, kProjWaitNs);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t stage = static_cast<uint32_t>((s * kProjStageBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kProjBK / 16; ++kk)  // 32 bytes of K per MMA
+            umma_ss<false>(acc, dA + stage + kk * 2, dB + stage + kk * 2, idesc,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar_empty + 8 * s);
+        }
+        if (ok) umma_commit(bar_acc_full + 8 * a);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int wq = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;
+    const int HD = p.H * p.D;
+    const uint32_t lanes = static_cast<uint32_t>(wq * 32) << 16;
+    int n = 0;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++n) {
+      const int a = n & 1;
+      int tm, tn;
+      proj_tile(t, p.tiles_m, p.tiles_n, tm, tn);
+      const int m = tm * kProjBM + row, n0 = tn * kProjBN;
+      const bool got = mbar_wait(bar_acc_full + 8 * a, (n >> 1) & 1, abort_flag, kProjWaitNs);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // row part of the destination offset, per layout (m is a token row of
+      // the sequence-sharded hidden states)
+      int64_t row_seq = 0, row_head = 0;
+      if (m < p.M) {
+        row_seq = static_cast<int64_t>(m) * HD;
+        if (p.layout == kProjHeadSharded) {
+          const int bn = m % (p.B * p.Nl);                // m = (r*B + b)*Nl + n
+          const int r = m / (p.B * p.Nl), bb = bn / p.Nl, nn = bn - bb * p.Nl;
+          row_head = static_cast<int64_t>(bb) * p.Np + static_cast<int64_t>(r) * p.Nl + nn;
+        }
+      }
+      const uint32_t taddr = tmem + lanes + static_cast<uint32_t>(a * kProjBN);
+      for (int c = 0; c < kProjBN; c += 32) {
+        const int f = n0 + c;                             // first feature of the chunk
+        uint32_t accv[32];
+        __syncwarp();                                     // TMEM loads are warp-collective
+        tmem_ld32(taddr + c, accv);
+        tmem_wait_ld();
+        if (c + 32 == kProjBN) {
+          // the whole accumulator is in registers: hand it back to the MMAs
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_empty + 8 * a);
+        }
+        if (f >= p.nout || m >= p.M) continue;            // after the collective load
+        const int tt = f / HD, hd = f - tt * HD, h = hd / p.D, d = hd - h * p.D;
+        int64_t off;
+        if (p.layout == kProjSeqSharded) {
+          off = row_seq + hd;
+        } else {
+          const int j = h / p.Hl, hh = h - j * p.Hl;
+          const int64_t rows = p.layout == kProjHeadSharded
+                                   ? static_cast<int64_t>(j) * p.B * p.Np + row_head
+                                   : static_cast<int64_t>(j) * p.M + m;
+          off = (rows * p.Hl + hh) * p.D + d;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float y0 = __uint_as_float(accv[2 * i]), y1 = __uint_as_float(accv[2 * i + 1]);
+          if (p.bias != nullptr) {
+            y0 += __bfloat162float(p.bias[f + 2 * i]);
+            y1 += __bfloat162float(p.bias[f + 2 * i + 1]);
+          }
+          w[i] = pack_bf16x2(y0, y1);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(p.out[tt] + off);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  if (!ok) {
+    *abort_flag = 1;
+    atomicExch(p.status, kProjStatusTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 50000ull) {
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kProjTmemCols);
+  }
+}
+
+}  // namespace sp

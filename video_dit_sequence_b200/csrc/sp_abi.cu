@@ -15,6 +15,7 @@
 
 #include "attention.cuh"
 #include "permute.cuh"
+#include "projection.cuh"
 #include "sp.h"
 
 namespace {
@@ -411,6 +412,84 @@ sp_status attention_peer(const void *const *q_shards, const void *k_group, const
   return launch_status(cudaGetLastError());
 }
 
+// Tensor map over a row-major bf16 matrix [rows][cols] (cols contiguous), as
+// 4-D with unit outer dims; boxes of 64 columns x box_rows rows under the
+// 128-byte swizzle.  Rows past the end read as zeros.
+bool make_map_matrix(CUtensorMap *m, const void *base, int cols, int rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(cols) * 2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), 1, 1};
+  cuuint64_t strides[3] = {row, row * rows, row * rows};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q, void *k,
+                         void *v, int32_t hidden, int32_t layout, const sp_shape *s,
+                         void *stream) {
+  if (layout < SP_QKV_SEQ_SHARDED || layout > SP_QKV_SEND_CHUNKS) return SP_ERR_SHAPE;
+  sp_status st = check_common(s, layout != SP_QKV_SEQ_SHARDED);
+  if (st != SP_OK) return st;
+  if (x == nullptr || w == nullptr || q == nullptr || k == nullptr || v == nullptr)
+    return SP_ERR_NULL;
+  if (hidden < 8 || hidden % 8 != 0) return SP_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 1u) != 0))
+    return SP_ERR_ALIGN;
+  const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
+  const int Nl = (N + P - 1) / P;
+  const int64_t M64 = static_cast<int64_t>(layout == SP_QKV_SEND_CHUNKS ? 1 : P) * B * Nl;
+  const int64_t nout64 = 3ll * H * D;
+  if (M64 >= (int64_t(1) << 31) || nout64 >= (int64_t(1) << 31) ||
+      M64 * hidden >= (int64_t(1) << 40))
+    return SP_ERR_SHAPE;
+  int32_t *status = status_ptr();
+  if (status == nullptr) return SP_ERR_CUDA;
+  CUtensorMap mx, mw;
+  if (!make_map_matrix(&mx, x, hidden, static_cast<int>(M64), sp::kProjBM) ||
+      !make_map_matrix(&mw, w, hidden, static_cast<int>(nout64), sp::kProjBN))
+    return SP_ERR_CUDA;
+  sp::ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = static_cast<int32_t>(M64);
+  p.K = hidden;
+  p.nout = static_cast<int32_t>(nout64);
+  p.H = H;
+  p.D = D;
+  p.Hl = layout == SP_QKV_SEQ_SHARDED ? H : H / P;
+  p.P = P;
+  p.B = B;
+  p.Nl = Nl;
+  p.Np = Nl * P;
+  p.layout = layout;
+  p.tiles_m = static_cast<int32_t>((M64 + sp::kProjBM - 1) / sp::kProjBM);
+  p.tiles_n = static_cast<int32_t>((nout64 + sp::kProjBN - 1) / sp::kProjBN);
+  p.out[0] = static_cast<__nv_bfloat16 *>(q);
+  p.out[1] = static_cast<__nv_bfloat16 *>(k);
+  p.out[2] = static_cast<__nv_bfloat16 *>(v);
+  p.bias = static_cast<const __nv_bfloat16 *>(bias);
+  p.status = status;
+  static bool attr_set[kMaxDevices] = {};
+  cudaError_t e = set_smem_once(sp::qkv_projection_kernel, sp::kProjSmemBytes, attr_set);
+  if (e != cudaSuccess) return SP_ERR_CUDA;
+  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  if (tiles >= (int64_t(1) << 31)) return SP_ERR_SHAPE;
+  // persistent: one CTA per SM (or per tile when there are fewer tiles)
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SP_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  sp::qkv_projection_kernel<<<grid, sp::kProjThreads, sp::kProjSmemBytes,
+                              static_cast<cudaStream_t>(stream)>>>(mx, mw, p);
+  return launch_status(cudaGetLastError());
+}
+
 using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
 
 AddressRangeFn address_range_fn() {
@@ -510,6 +589,13 @@ sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const v
   NvtxRange range("sp_attention_sparse_seqsharded");
   if (mask == nullptr) return SP_ERR_NULL;
   return attention(qs, ks, vs, os, lse, shape, stream, true, nullptr, nullptr, nullptr, mask);
+}
+
+sp_status sp_qkv_projection(const void *x, const void *w, const void *bias, void *q, void *k,
+                            void *v, int32_t hidden, int32_t layout, const sp_shape *shape,
+                            void *stream) {
+  NvtxRange range("sp_qkv_projection");
+  return qkv_projection(x, w, bias, q, k, v, hidden, layout, shape, stream);
 }
 
 sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_group,
