@@ -244,6 +244,33 @@ def test_fused_peer_exchange_on_virtual_ranks(B, N, H, P):
     _check_rows(got, q, k, v, rows, P, f"peer step B={B} N={N} P={P}")
 
 
+def test_rank_classes_in_a_one_member_nccl_group():
+    """UlyssesPeerRank (CUDA IPC export, NCCL all-to-all, peer step, closing
+    all-reduce) and ulysses_attention_distributed run end to end as a
+    one-member NCCL group and give the fused call's output bit for bit."""
+    import torch.distributed as dist
+    B, N, H, D = 1, 1000, 4, 128
+    shape = sp.Shape(B, N, H, D, 1)
+    q, k, v = _random_logical(B, N, H, D, seed=73)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, 1)) for x in (q, k, v))
+    want, _ = _run_fused(q, k, v, 1)
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        pr = sp.UlyssesPeerRank(shape)
+        for _ in range(2):                                 # buffers reused across steps
+            out = pr.step(ks[0], vs[0], q=qs[0])
+            torch.cuda.synchronize()
+            assert np.array_equal(to_host(out).reshape(want.shape), want)
+        pr.close()
+        out2 = sp.ulysses_attention_distributed(qs[0], ks[0], vs[0], shape)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_host(out2).reshape(want.shape), want)
+        _status_ok()
+    finally:
+        dist.destroy_process_group()
+
+
 def test_peer_step_writes_only_its_head_group():
     B, N, H, D, P = 1, 1000, 8, 128, 4
     q, k, v = _random_logical(B, N, H, D, seed=21)
