@@ -5,11 +5,10 @@
  * The method (fal.ai, "Generate video with WAN 2.2 across four GPUs",
  * section "Splitting one generation across four GPUs"): the token sequence
  * of one generation is split across P ranks; at each attention layer an
- * all-to-all trades tokens for heads so that every rank sees the full
- * sequence for H/P of the H heads, attention runs per head over all tokens,
- * and the outputs return to the ranks that own the tokens.  The result is
- * numerically the single-GPU result (LTX-2 "Multi-GPU Inference" README,
- * Capabilities table).  On one GPU the exchange is a permutation in HBM
+ * all-to-all exchanges token shards for head groups, so that every rank
+ * attends over all tokens for H/P of the H heads, and the outputs go back to
+ * the ranks that own the tokens.  The result is the single-GPU result
+ * (LTX-2 "Multi-GPU Inference" README, Capabilities table).  On one GPU the exchange is a permutation in HBM
  * (sp_pack / sp_unpack) or disappears into the attention kernel's addressing
  * (sp_attention_seqsharded).  With one GPU per rank, sp_exchange_pack /
  * sp_exchange_unpack reorder a rank's shard around an all-to-all, and
@@ -70,9 +69,9 @@ typedef struct {
  * N < 1 or P < 1. */
 int64_t sp_padded_tokens(int32_t N, int32_t P);
 
-/* Validates a shape against the rules above; the degree rule ("the Ulysses
- * degree must divide the attention head count", fal.ai page, section
- * "Tuning cost and GPU count") gives SP_ERR_HEADS_NOT_DIVISIBLE. */
+/* Validates a shape against the rules above.  The degree rule of the fal.ai
+ * page, section "Tuning cost and GPU count" (P has to be a divisor of H),
+ * gives SP_ERR_HEADS_NOT_DIVISIBLE. */
 sp_status sp_check_shape(const sp_shape *shape);
 
 /* Pack: sequence-sharded -> head-sharded, the send reorder plus all-to-all
@@ -83,8 +82,8 @@ sp_status sp_check_shape(const sp_shape *shape);
  * not overlap. */
 sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream);
 
-/* Unpack: head-sharded -> sequence-sharded ("the shards return to their own
- * GPUs", same section); the inverse of sp_pack:
+/* Unpack: head-sharded -> sequence-sharded (the outputs go back to the ranks
+ * that own the tokens, same section); the inverse of sp_pack:
  *   os[r][b][n][j*Hl + hh][c] = oh[j][b][r*Nl + n][hh][c]
  * oh: device, [P][B][Np][Hl][D] bf16, read only.  os: device,
  * [P][B][Nl][H][D] bf16, written in full.  Bit-exact copy. */
@@ -104,7 +103,7 @@ sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *strea
  * (H % P == 0).  Bit-exact copy. */
 sp_status sp_exchange_pack(const void *xs_r, void *send, const sp_shape *shape, void *stream);
 
-/* Exchange unpack on one rank ("the shards return to their own GPUs"): the
+/* Exchange unpack on one rank (outputs back to the token owners): the
  * P chunks returned by the head groups, chunk j = group j's output for this
  * rank's tokens, become the rank's shard:
  *   os_r[b][n][j*Hl + hh][c] = recv[j][b][n][hh][c]
@@ -115,8 +114,8 @@ sp_status sp_exchange_unpack(const void *recv, void *os_r, const sp_shape *shape
 /* Attention per head group on head-sharded tensors: for every batch b,
  * group j, local head hh (global head h = j*Hl + hh) and query token i < N,
  *   oh[j][b][i][hh] = sum_{k<N} softmax_k(q_i . k_k * scale) v_k
- * non-causal, keys k >= N masked; "each GPU sees the full sequence" for its
- * heads (same section).  Accumulation in fp32, probabilities rounded to
+ * non-causal, keys k >= N masked; every rank attends over all tokens for
+ * its heads (same section).  Accumulation in fp32, probabilities rounded to
  * bf16 before the P*V product, output rounded to nearest-even bf16.  Rows
  * i in [N, Np) are written as zero.  The result for a given (b, h, i) does
  * not depend on P.
@@ -281,9 +280,14 @@ sp_status sp_ipc_open(const void *handle, void **base_out);
 /* Unmaps an allocation mapped by sp_ipc_open. */
 sp_status sp_ipc_close(void *base);
 
-/* Synchronises `stream`, then returns and clears the device status word:
- * SP_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
- * SP_ERR_CUDA if the stream reports an error, else SP_OK. */
+/* Takes the device status word of the current device and clears it in one
+ * atomic exchange enqueued on `stream`, then synchronises `stream` and
+ * returns what it took: SP_ERR_TIMEOUT if a kernel gave up on a bounded wait
+ * since the last call, SP_ERR_CUDA if the stream reports an error, else
+ * SP_OK.  The word is shared by every stream of the device: a timeout that a
+ * kernel on another stream records after the exchange is reported by the
+ * next call, never lost.  Synchronise every stream that launched sp kernels
+ * first to have all of them covered by this call. */
 sp_status sp_device_status(void *stream);
 
 /* Self-test of the bounded waits: enqueues one small kernel that waits on a

@@ -12,8 +12,8 @@ What it computes, and the passages it follows:
   the all-to-all and the reverse reorder after the return all-to-all.
 * ``pack`` / ``unpack`` -- the token<->head all-to-all of the fal.ai page
   "Generate video with WAN 2.2 across four GPUs", section "Splitting one
-  generation across four GPUs" (each GPU sees the full sequence for its share
-  of the heads, then the shards return).  Index formulas in ``sp_oracle.c``.
+  generation across four GPUs" (each GPU attends over all tokens for its
+  share of the heads, then the outputs go back to the token owners).  Index formulas in ``sp_oracle.c``.
 * ``attention_rows_e4m3`` -- the same attention on 8-bit (E4M3) inputs with
   scale factors per block of tokens for Q and K and per channel for V, for
   the FP8 variant of the kernel.
@@ -27,7 +27,7 @@ What it computes, and the passages it follows:
 * ``attention_rows`` -- the unsharded softmax(q K^T scale) V of one head,
   two-pass exact softmax in fp64; the sequence-parallel result must equal it
   for every degree (LTX-2 "Multi-GPU Inference" README, Capabilities table:
-  SP is numerically equivalent to single-GPU).
+  SP gives the single-GPU result).
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, invariants, a worked example, brute force and numpy's fp64 routines.

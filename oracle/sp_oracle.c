@@ -9,13 +9,13 @@
  * Sources of the definitions (web pages on the method):
  *  - fal.ai, "Generate video with WAN 2.2 across four GPUs", section
  *    "Splitting one generation across four GPUs": at every attention layer an
- *    all-to-all trades tokens for heads, each GPU then sees the full sequence
- *    for its share of the heads (10 of 40 at four GPUs), and the shards
- *    return to their own GPUs afterwards.
- *  - same page, section "Tuning cost and GPU count": the Ulysses degree must
- *    divide the attention head count.
+ *    all-to-all exchanges token shards for head groups, so that each GPU
+ *    attends over all tokens for its share of the heads (10 of 40 at four
+ *    GPUs); afterwards the outputs go back to the GPUs that own the tokens.
+ *  - same page, section "Tuning cost and GPU count": the degree has to be a
+ *    divisor of the head count.
  *  - LTX-2 "Multi-GPU Inference" README, Capabilities table: sequence
- *    parallelism is numerically equivalent to single-GPU inference.  The
+ *    parallelism gives the single-GPU result.  The
  *    oracle therefore computes the unsharded (single-GPU) attention for every
  *    degree P.
  *
@@ -103,8 +103,8 @@ int sp_oracle_pack(const uint16_t *xs, uint16_t *xh, int64_t B, int64_t N,
 }
 
 /*
- * Unpack (head-sharded -> sequence-sharded): "the shards return to their own
- * GPUs" in the same page section; the inverse of the pack:
+ * Unpack (head-sharded -> sequence-sharded): the outputs go back to the
+ * token owners (same page section); the inverse of the pack:
  *     os[r][b][n][j*Hl + hh][c] = oh[j][b][r*Nl + n][hh][c]
  */
 int sp_oracle_unpack(const uint16_t *oh, uint16_t *os, int64_t B, int64_t N,
@@ -148,7 +148,7 @@ int sp_oracle_exchange_pack(const uint16_t *xs_r, uint16_t *send, int64_t B, int
 }
 
 /*
- * Exchange unpack on one rank ("the shards return to their own GPUs"): the
+ * Exchange unpack on one rank (outputs back to the token owners): the
  * P chunks received back from the head groups, recv[j][b][n][hh][c] (group
  * j's output for this rank's tokens), become the shard [B][Nl][H][D]:
  *     os_r[b][n][j*Hl + hh][c] = recv[j][b][n][hh][c]

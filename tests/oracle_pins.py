@@ -9,7 +9,7 @@ Facts used:
 * page facts: after the exchange, head group j holds the full sequence for
   heads j*Hl .. j*Hl+Hl-1 (fal.ai WAN 2.2 page, "Splitting one generation
   across four GPUs"); the degree must divide the head count ("Tuning cost and
-  GPU count"); the shards return to their owners afterwards.
+  GPU count"); the outputs go back to the token owners afterwards.
 * library routines: numpy's reshape/transpose for the permutation and
   numpy fp64 matmul/exp for softmax(q K^T scale) V on small problems;
   scipy's logsumexp for the LSE.
@@ -83,7 +83,7 @@ def check_pack_matches_numpy_transpose(lib=None):
 
 
 def check_unpack_returns_shards(lib=None):
-    """The shards return to their owners: unpack(pack(x)) = x, and a
+    """Outputs go back to the token owners: unpack(pack(x)) = x, and a
     head-sharded result built from a logical tensor unpacks to its shards."""
     rng = np.random.default_rng(RNG_SEED + 2)
     for (B, N, H, D, P) in PACK_SHAPES:

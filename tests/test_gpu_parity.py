@@ -116,22 +116,48 @@ def test_pack_unpack_bit_exact(B, N, H, D, P):
     _status_ok()
 
 
-@pytest.mark.parametrize("name", ["720p", "sweep-N75601-P8"])
-def test_pack_full_size_bit_exact(name):
-    cfg = synth.CONFIGS.get(name) or synth.sweep_config(75601, 8)
-    s = cfg.shape
-    shape = sp.Shape(s.B, s.N, s.H, s.D, s.P)
-    q = synth.logical_tensor(cfg, synth.TID_Q)
-    xs = synth.to_seq_shards(q, s.P)
-    want = oracle.pack(xs, s.N)
-    d_xh = torch.empty(shape.head_sharded, dtype=torch.bfloat16, device="cuda")
+def _perm_full_size(q, N, H, P, where):
+    """Pack of the logical tensor q [B][N][H][D] as P shards, and unpack of an
+    independent head-sharded tensor of the same size whose padding rows are
+    not zero, both compared bit for bit with the oracle."""
+    B, _, _, D = q.shape
+    shape = sp.Shape(B, N, H, D, P)
+    xs = synth.to_seq_shards(q, P)
+    want = oracle.pack(xs, N)
+    d_xh = torch.full(shape.head_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
     sp.pack(to_dev(xs), d_xh, shape)
-    assert np.array_equal(to_host(d_xh).reshape(want.shape), want)
-    want_s = oracle.unpack(want, s.N, s.H)
-    d_os = torch.empty(shape.seq_sharded, dtype=torch.bfloat16, device="cuda")
-    sp.unpack(d_xh, d_os, shape)
-    assert np.array_equal(to_host(d_os).reshape(want_s.shape), want_s)
+    assert np.array_equal(to_host(d_xh).reshape(want.shape), want), f"{where}: pack"
+    del want
+    oh = synth.normal_bf16(300 + P, 4, 0, int(np.prod(shape.head_sharded)))
+    oh = oh.reshape(shape.head_sharded)
+    want_s = oracle.unpack(oh, N, H)
+    d_os = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.unpack(to_dev(oh), d_os, shape)
+    assert np.array_equal(to_host(d_os).reshape(want_s.shape), want_s), f"{where}: unpack"
+    # round trip on the device: unpack(pack(xs)) = xs (padding slots included)
+    d_back = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.unpack(d_xh, d_back, shape)
+    assert np.array_equal(to_host(d_back).reshape(xs.shape), xs), f"{where}: round trip"
     _status_ok()
+
+
+@pytest.mark.parametrize("name", ["480p", "720p", "1344x768"])
+def test_pack_full_size_bit_exact(name):
+    """The permutations on the full-size configurations, in the degree each
+    is quoted with (480p P = 2, 720p P = 4, 1344x768 P = 8)."""
+    cfg = synth.CONFIGS[name]
+    s = cfg.shape
+    _perm_full_size(synth.logical_tensor(cfg, synth.TID_Q), s.N, s.H, s.P, name)
+
+
+@pytest.mark.parametrize("N", synth.SWEEP_N)
+def test_pack_sweep_bit_exact(N):
+    """Layout sweep: pack and unpack alone for every (N, P) pair of the sweep,
+    N in {4096, 32760, 75600, 75601 (ragged)}, P in {1, 2, 4, 8}."""
+    base = synth.sweep_config(N, 1)
+    q = synth.logical_tensor(base, synth.TID_Q)
+    for P in synth.SWEEP_P:
+        _perm_full_size(q, N, base.shape.H, P, f"sweep N={N} P={P}")
 
 
 EXCHANGE_SHAPES = [(1, 1024, 4, 64, 2), (2, 1000, 8, 128, 4), (3, 77, 6, 128, 3),
@@ -960,8 +986,10 @@ def _sampled_check(cfg, per_head, fused=True, extra_P=()):
 
 @pytest.mark.parametrize("name", ["480p", "720p", "1344x768"])
 def test_full_size_configs_sampled_rows(name):
+    """256 sampled query rows per head on 480p and 720p (the survey's count;
+    about 30 s of oracle time at 720p on 16 host threads), 128 on 1344x768."""
     cfg = synth.CONFIGS[name]
-    per_head = 12 if name == "1344x768" else 16
+    per_head = 128 if name == "1344x768" else 256
     _sampled_check(cfg, per_head)
 
 
@@ -986,7 +1014,7 @@ def test_sweep_degrees_bit_identical_and_sampled():
             got = synth.from_seq_shards(out.reshape(P, 1, -1, 40, 128), N)
             if ref is None:
                 ref = got
-                rows = synth.sampled_rows(base, 6, extra_P=synth.SWEEP_P)
+                rows = synth.sampled_rows(base, 32, extra_P=synth.SWEEP_P)
                 rr = np.array([(0, h, i) for h in range(40) for i in rows], dtype=np.int64)
                 _check_rows(out, q, k, v, rr, 1, f"sweep N={N}")
             else:

@@ -8,9 +8,9 @@ device, the calls raise.
 
 The method (fal.ai, "Generate video with WAN 2.2 across four GPUs", section
 "Splitting one generation across four GPUs"): P ranks each hold N/P tokens
-of the sequence for all H heads; an all-to-all trades tokens for heads, each
-rank attends over the full sequence for H/P heads, and the outputs return to
-the token owners.  With P virtual ranks on one GPU the exchange is
+of the sequence for all H heads; an all-to-all exchanges token shards for
+head groups, each rank attends over all tokens for H/P heads, and the outputs
+go back to the token owners.  With P virtual ranks on one GPU the exchange is
 ``pack`` / ``unpack``; ``attention_seqsharded`` fuses all three steps.
 
 Layouts (bf16, contiguous):
@@ -468,6 +468,18 @@ def attention_ulysses_peer(q_shards, k_group, v_group, o_shards, shape: Shape, r
             ctypes.byref(s), _stream(stream, k_group.device)), "sp_attention_ulysses_peer")
 
 
+def _require_ipc_exportable():
+    """CUDA IPC exports allocations made by cudaMalloc.  With PyTorch's
+    expandable_segments option, its caching allocator maps memory with
+    cuMemCreate instead, and the export fails; say so before trying."""
+    for var in ("PYTORCH_CUDA_ALLOC_CONF", "PYTORCH_ALLOC_CONF"):
+        conf = os.environ.get(var, "").replace(" ", "").lower()
+        if "expandable_segments:true" in conf:
+            raise RuntimeError(
+                f"{var} enables expandable_segments: CUDA IPC cannot export those "
+                "allocations; unset it for the peer exchange")
+
+
 def ipc_export(t):
     """(handle, offset): the CUDA IPC handle (bytes) of the allocation that
     holds CUDA tensor t, and t's byte offset from that allocation's base."""
@@ -508,6 +520,7 @@ class CudaPeerBackend:
         return torch.empty(shape, dtype=dtype or torch.bfloat16, device=self.device)
 
     def export(self, t):
+        _require_ipc_exportable()
         return ipc_export(t)
 
     def open(self, handle: bytes, offset: int):
@@ -681,8 +694,11 @@ class HostPipeline:
         return freed
 
     def synchronize(self):
+        """Waits for everything submitted, then checks the device status word
+        (raises SpError when a kernel gave up on a bounded wait)."""
         for st in (self.h2d, self.compute, self.d2h):
             st.synchronize()
+        _check(device_status(self.compute), "HostPipeline")
 
 
 def device_status(stream=None, device=None) -> int:

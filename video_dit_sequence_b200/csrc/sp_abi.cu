@@ -31,6 +31,13 @@ struct NvtxRange {
 };
 
 __device__ int32_t g_status = 0;
+// Where status_take_kernel leaves the value it took out of g_status.
+__device__ int32_t g_status_taken = 0;
+
+// Takes the status word and clears it in one atomic exchange on the device,
+// so that a timeout recorded by a kernel on another stream is either taken
+// here or left for the next call, never lost between a read and a clear.
+__global__ void status_take_kernel() { g_status_taken = atomicExch(&g_status, 0); }
 
 std::atomic<uint64_t> g_launches{0};
 
@@ -638,16 +645,14 @@ sp_status sp_ipc_close(void *base) {
 sp_status sp_device_status(void *stream) {
   NvtxRange range("sp_device_status");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(cs) != cudaSuccess) return SP_ERR_CUDA;
-  int32_t *status = status_ptr();
-  if (status == nullptr) return SP_ERR_CUDA;
+  status_take_kernel<<<1, 1, 0, cs>>>();
+  if (cudaGetLastError() != cudaSuccess) return SP_ERR_CUDA;
   int32_t v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return SP_ERR_CUDA;
-  if (v != 0) {
-    const int32_t zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SP_ERR_CUDA;
-    return v == sp::kStatusTimeout ? SP_ERR_TIMEOUT : SP_ERR_CUDA;
-  }
+  if (cudaMemcpyFromSymbolAsync(&v, g_status_taken, sizeof(v), 0, cudaMemcpyDeviceToHost, cs) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(cs) != cudaSuccess)
+    return SP_ERR_CUDA;
+  if (v != 0) return v == sp::kStatusTimeout ? SP_ERR_TIMEOUT : SP_ERR_CUDA;
   return SP_OK;
 }
 
