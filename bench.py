@@ -15,15 +15,18 @@ V; attention on head-sharded tensors; unpack of O) are timed in the same run
 and reported under "rows" (GB/s for the permutations).  Q+K+V are 2.3 GB,
 far larger than the 126 MB L2, so no L2 flush is done between steps.
 
-With --gpus N > 1 (launched by torchrun, one rank per GPU) every rank runs
-the same single-GPU problem on its own GPU: independent problems, no
-data-path collective, weak scaling.  --mode ulysses instead splits the one
-problem across the N GPUs the way the method does (P = N ranks, NCCL
-all-to-all of the sequence shards, each GPU attends H/N heads over the whole
-sequence, all-to-all back): strong scaling.  --mode ulysses-peer exchanges
-only K and V that way; the attention kernel reads Q tiles from the ranks
-that hold them and stores O rows into the ranks that own them over peer
-memory (CUDA IPC).
+With --gpus N > 1 (launched by torchrun, one rank per GPU) the one 720p
+problem is split across the N GPUs the way the method does (--mode ulysses,
+the default: P = N ranks, NCCL all-to-all of the sequence shards, each GPU
+attends H/N heads over the whole sequence, all-to-all back): strong
+scaling.  --mode ulysses-peer moves the exchanges into the kernels: each
+rank stores its K/V chunks straight into the head groups' buffers over peer
+memory (CUDA IPC) and the attention kernel starts on the chunks that have
+arrived while the rest are in flight, reads Q tiles from the ranks that hold
+them and stores O rows into the ranks that own them (--kv-exchange nccl
+keeps an NCCL all-to-all for K/V).  --mode replicas runs the single-GPU
+problem independently on every GPU instead (no data-path collective, weak
+scaling).
 
 --impl reference times the fp64 CPU oracle on the host cores instead, each
 step a bounded sample (query rows) of the same workload.
@@ -223,8 +226,10 @@ def run_ulysses(args):
     """--mode ulysses / ulysses-peer: the multi-GPU form, one rank per GPU.
     ulysses: Q, K and V exchanged by NCCL all-to-alls around the fused
     attention of the head group, O exchanged back the same way.
-    ulysses-peer: K and V exchanged by NCCL, Q read and O written by the
-    attention kernel itself over peer memory (UlyssesPeerRank)."""
+    ulysses-peer: K and V pushed into the head groups over peer memory and
+    attended as they arrive (or, with --kv-exchange nccl, exchanged by an
+    NCCL all-to-all); Q read and O written by the attention kernel itself
+    over peer memory (UlyssesPeerRank)."""
     import datetime
 
     import numpy as np
@@ -267,7 +272,7 @@ def run_ulysses(args):
     out = [None]
     peer = args.mode == "ulysses-peer"
     if peer:
-        pr = sp.UlyssesPeerRank(shape, device=dev)
+        pr = sp.UlyssesPeerRank(shape, device=dev, kv_exchange=args.kv_exchange)
         pr.q_shard.copy_(dq)                 # Q lives in the exported shard buffer
         q_in = pr.q_shard
 
@@ -275,9 +280,10 @@ def run_ulysses(args):
             out[0] = pr.step(dk, dv)
     else:
         q_in = dq
+        ur = sp.UlyssesRank(shape)           # exchange buffers reused across steps
 
         def step():
-            out[0] = sp.ulysses_attention_distributed(dq, dk, dv, shape, a2a)
+            out[0] = sp.ulysses_attention_distributed(dq, dk, dv, shape, a2a, rank=ur)
 
     def timed(fn):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -326,9 +332,12 @@ def run_ulysses(args):
                 "ms_per_step": t_max / args.steps, "higher_is_better": True,
                 "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": dict(workload_desc(cfg), P=world, parallelism=f"ulysses{world}",
-                               exchange=("K/V: NCCL all_to_all_single; Q/O: inside the "
-                                         "attention kernel over peer memory (CUDA IPC)")
-                               if peer else "NCCL all_to_all_single"),
+                               exchange=(("K/V: pushed into the head groups over peer memory, "
+                                          "attention overlapped with their arrival"
+                                          if args.kv_exchange == "push" else
+                                          "K/V: NCCL all_to_all_single")
+                                         + "; Q/O: inside the attention kernel over peer memory "
+                                           "(CUDA IPC)") if peer else "NCCL all_to_all_single"),
                 "e2e": {"value": args.steps * flops / (te * 1e-3) / 1e12, "unit": UNIT,
                         "h2d_bytes_per_step": int(3 * shard_bytes),
                         "d2h_bytes_per_step": int(shard_bytes)},
@@ -477,7 +486,7 @@ def run_ours(args):
     # the projection in front of attention (hidden -> q, k, v) with its
     # epilogue writing the sequence-sharded layout; cuBLAS on the same GEMM
     # (x @ w^T, one contiguous output) timed beside it
-    t_proj = t_cublas = None
+    t_proj = t_cublas = t_oproj = t_oproj_cublas = None
     if not args.no_proj and s.D == 128:
         hidden = s.H * s.D
         M = s.P * s.B * shape.Nl
@@ -491,6 +500,16 @@ def run_ours(args):
         t_cublas = timed(lambda: torch.matmul(xw, ww.t(), out=yc))
         proj_flops = 2.0 * M * hidden * 3 * hidden
         del xw, ww, pq, pkk, pv, yc
+        # the output projection after attention (O as sequence shards -> hidden),
+        # on the fused call's output; cuBLAS on the same GEMM beside it
+        wo = (torch.randn(hidden, s.H * s.D, device=dev, generator=gen)
+              / math.sqrt(s.H * s.D)).to(torch.bfloat16)
+        yo = torch.empty(M, hidden, dtype=torch.bfloat16, device=dev)
+        t_oproj = timed(lambda: sp.out_projection(os_, wo, None, yo, shape, stream=stream))
+        o2d = os_.view(M, s.H * s.D)
+        t_oproj_cublas = timed(lambda: torch.matmul(o2d, wo.t(), out=yo))
+        oproj_flops = 2.0 * M * s.H * s.D * hidden
+        del wo, yo
     if sp.device_status(stream) != sp.SP_OK:
         raise SystemExit("device status not ok after the unfused rows")
     pack_gbs = 2 * tensor_bytes / (t_pack * 1e-3) / 1e9
@@ -520,6 +539,13 @@ def run_ours(args):
             "cublas_ms": t_cublas, "cublas_TFLOP/s": proj_flops / (t_cublas * 1e-3) / 1e12,
             "what": f"hidden {s.H * s.D} -> q, k, v (bf16) written as sequence shards; cuBLAS: "
                     "the same GEMM into one [M][3HD] matrix"},
+        "out_projection": None if t_oproj is None else {
+            "ms": t_oproj, "TFLOP/s": oproj_flops / (t_oproj * 1e-3) / 1e12,
+            "frac": oproj_flops / (t_oproj * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "cublas_ms": t_oproj_cublas,
+            "cublas_TFLOP/s": oproj_flops / (t_oproj_cublas * 1e-3) / 1e12,
+            "what": f"attention output {s.H * s.D} -> hidden {s.H * s.D} (bf16), O read as "
+                    "sequence shards; cuBLAS: the same GEMM"},
         "unfused_step_ms": 3 * t_pack + t_attn + t_unpack,
         "fused_step_ms": per_launch_ms,
     }
@@ -591,9 +617,13 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--mode", choices=["replicas", "ulysses", "ulysses-peer"], default="replicas",
-                    help="N > 1 only: independent problems per GPU (default) or one problem "
-                         "split across the GPUs with the Ulysses all-to-all")
+    ap.add_argument("--mode", choices=["replicas", "ulysses", "ulysses-peer"], default=None,
+                    help="N > 1 only: one problem split across the GPUs with the Ulysses "
+                         "all-to-all (ulysses, the default), the same with the exchanges in the "
+                         "kernels (ulysses-peer), or independent problems per GPU (replicas)")
+    ap.add_argument("--kv-exchange", choices=["push", "nccl"], default="push",
+                    help="ulysses-peer: K/V pushed over peer memory and overlapped with "
+                         "attention (default) or exchanged by an NCCL all-to-all")
     ap.add_argument("--config", default="720p")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
@@ -609,6 +639,8 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode is None:
+        args.mode = "ulysses" if args.gpus > 1 else "replicas"
     if args.mode in ("ulysses", "ulysses-peer"):
         return run_ulysses(args)
     return run_ours(args)

@@ -198,6 +198,40 @@ sp_status sp_qkv_projection(const void *x, const void *w, const void *bias, void
                             void *v, int32_t hidden, int32_t layout, const sp_shape *shape,
                             void *stream);
 
+/* Where sp_out_projection reads the attention output O. */
+typedef enum {
+  SP_O_SEQ_SHARDED = 0,  /* [P][B][Nl][H][D]: the fused attention's output */
+  SP_O_HEAD_SHARDED = 1, /* [P][B][Np][Hl][D]: sp_attention's output (the unpack folded in) */
+  SP_O_RECV_CHUNKS = 2   /* [P][B][Nl][Hl][D] of one rank: the P chunks returned to it
+                            (its exchange unpack folded in) */
+} sp_o_layout;
+
+/* The projection after attention: each token's attention output (all H
+ * heads, H*D features, head-major) to its hidden state,
+ *   y[m][c] = sum_k o[m][k] * w[c][k] (+ bias[c]),   k = h*D + d,
+ * with a feature's weights in one row of w, as a linear layer stores them.
+ * The pages place sequence parallelism inside the transformer block (LTX-2
+ * "Multi-GPU Inference" README, section "Pages": the SP builder and its
+ * attention manager swap in per block) but never describe the block; this is
+ * the plainest reading of the step after attention (one linear layer).  The
+ * layout work is folded into the operand loads: O is read in the layout
+ * `layout` names, so neither sp_unpack nor sp_exchange_unpack runs between
+ * attention and this projection.  fp32 accumulation, bf16 output (round to
+ * nearest even).
+ * o: device bf16 in `layout`, 16-byte aligned, read only.
+ * w: device bf16 [hidden][H*D]; bias: device bf16 [hidden] or NULL.
+ * y: device bf16 [P][B][Nl][hidden], the sequence-sharded hidden states
+ *   (one rank's [B][Nl][hidden] for SP_O_RECV_CHUNKS), 16-byte aligned,
+ *   written in full (padding slots hold the projection of O's padding rows,
+ *   which attention writes as zero).
+ * hidden: a multiple of 8.  shape: {B, N, H, D, P}; the head-split layouts
+ *   need H % P == 0.
+ * Errors: SP_ERR_NULL, SP_ERR_ALIGN, SP_ERR_SHAPE (layout, hidden, sizes),
+ * SP_ERR_HEADS_NOT_DIVISIBLE, SP_ERR_UNSUPPORTED_D, SP_ERR_CUDA.  The result
+ * does not depend on the layout (bit for bit). */
+sp_status sp_out_projection(const void *o, const void *w, const void *bias, void *y,
+                            int32_t hidden, int32_t layout, const sp_shape *shape, void *stream);
+
 /* Tokens per cube of the block-sparse call's mask. */
 #define SP_SPARSE_CUBE 64
 
@@ -264,6 +298,64 @@ sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_g
                                     const void *v_group, void *const *o_shards, float *lse,
                                     int32_t rank, const sp_shape *shape, void *stream);
 
+/* ---------------------------------------------------------------------
+ * The same step with the K/V exchange overlapped with attention.
+ *
+ * In sp_attention_ulysses_peer, K and V reach the head groups through an
+ * all-to-all before the attention kernel starts.  Here each rank stores its
+ * K/V chunks straight into the head groups' buffers over peer memory
+ * (sp_exchange_push: the send-buffer reorder fused with the transfer, no
+ * send buffer and no all-to-all) and counts each finished piece in the
+ * receiving rank's arrival counters; the attention kernel
+ * (sp_attention_ulysses_overlap) walks key tiles in their fixed order and,
+ * before loading the tiles of source rank r's chunk (and the Q tiles of rank
+ * r's shard), waits with a bounded wait until r's counter shows that the
+ * chunk has arrived.  Attention on the first chunks runs while the later
+ * ones are in flight; the order of the arithmetic is unchanged, so results
+ * equal sp_attention_seqsharded's bit for bit.
+ * Protocol: every rank owns a counter array uint64 [P] (zeroed once, before
+ * any rank's first push) and a received-group buffer for K and for V.  Step
+ * e = 1, 2, ... of every rank: write Q into its Q shard, then
+ * sp_exchange_push(..., epoch = e), then sp_attention_ulysses_overlap(...,
+ * epoch = e), then a collective that follows every rank's attention kernel
+ * (as for sp_attention_ulysses_peer) before the next step overwrites any
+ * buffer a peer reads.
+ */
+
+/* Rank `rank` stores its K and V chunks for every head group j into rank
+ * j's received groups at chunk slot `rank`:
+ *   k_groups[j][rank][b][n][hh][c] = k_r[b][n][j*Hl + hh][c]   (v alike)
+ * and adds its finished pieces to counts[j][rank] with release semantics at
+ * system scope (after step e that counter holds e times the pieces of one
+ * step).
+ * k_r, v_r: this rank's shards [B][Nl][H][D] bf16, local, read only.
+ * k_groups, v_groups: HOST arrays of P device addresses valid in this
+ *   process (this rank's own buffers and the peers' mapped with sp_ipc_open);
+ *   each [P][B][Nl][Hl][D] bf16, 16-byte aligned; only chunk slot `rank` is
+ *   written.
+ * counts: HOST array of P device addresses of each rank's uint64 [P]
+ *   arrival counters, 8-byte aligned.
+ * epoch: this step's number, >= 1.  shape: the whole problem; H % P == 0,
+ *   P <= SP_MAX_PEERS, 0 <= rank < P.
+ * Errors: SP_ERR_NULL, SP_ERR_ALIGN, SP_ERR_SHAPE (also epoch 0),
+ * SP_ERR_HEADS_NOT_DIVISIBLE, SP_ERR_UNSUPPORTED_D, SP_ERR_CUDA. */
+sp_status sp_exchange_push(const void *k_r, const void *v_r, void *const *k_groups,
+                           void *const *v_groups, uint64_t *const *counts, uint64_t epoch,
+                           int32_t rank, const sp_shape *shape, void *stream);
+
+/* sp_attention_ulysses_peer on this rank's received groups while they
+ * arrive: before loading key tiles or Q tiles of source rank r, the kernel
+ * waits until counts[r] (this rank's own counter array, local, 8-byte
+ * aligned) shows step `epoch`'s pieces of r's chunk, at most wait_ns
+ * nanoseconds per wait (0: 2 s).  A wait that runs out stops the kernel:
+ * its in-flight copies and MMAs are drained, nothing is left running, and
+ * SP_ERR_TIMEOUT is recorded in the device status word (sp_device_status).
+ * Other arguments and results as for sp_attention_ulysses_peer. */
+sp_status sp_attention_ulysses_overlap(const void *const *q_shards, const void *k_group,
+                                       const void *v_group, void *const *o_shards, float *lse,
+                                       const uint64_t *counts, uint64_t epoch, uint64_t wait_ns,
+                                       int32_t rank, const sp_shape *shape, void *stream);
+
 /* Bytes of a CUDA IPC memory handle. */
 #define SP_IPC_HANDLE_BYTES 64
 
@@ -290,11 +382,14 @@ sp_status sp_ipc_close(void *base);
  * first to have all of them covered by this call. */
 sp_status sp_device_status(void *stream);
 
-/* Self-test of the bounded waits: enqueues one small kernel that waits on a
- * shared-memory barrier nothing will complete, with a limit of limit_ns
- * nanoseconds (clamped to 1 s).  The wait runs out, the kernel records
- * SP_ERR_TIMEOUT in the device status word and returns; the next
- * sp_device_status call reports it.  No GPU fault is involved. */
+/* Self-test of the bounded waits and of the abort path: enqueues one small
+ * kernel that starts a bulk copy into shared memory and one tensor-core MMA,
+ * then waits on a shared-memory barrier nothing will complete, with a limit
+ * of limit_ns nanoseconds (clamped to 1 s).  The wait runs out; the kernel
+ * waits for the copy and the MMA it issued, releases its tensor memory,
+ * records SP_ERR_TIMEOUT in the device status word and returns; the next
+ * sp_device_status call reports it (SP_ERR_CUDA if the drain did not
+ * finish).  No GPU fault is involved. */
 sp_status sp_selftest_wait_timeout(uint64_t limit_ns, void *stream);
 
 /* Number of kernels this library has enqueued since it was loaded. */

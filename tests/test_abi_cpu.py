@@ -154,6 +154,50 @@ def test_argument_errors_return_before_launch(lib):
         sp.SP_ERR_HEADS_NOT_DIVISIBLE
     assert proj(A, A, 0, B_, B_, B_, 512, 0, sp.Shape(1, 1000, 6, 96, 4)) == \
         sp.SP_ERR_UNSUPPORTED_D
+    oproj = lambda o, w, b, y, hidden, layout, shp=sp.Shape(1, 1000, 4, 128, 2): \
+        lib.sp_out_projection(*[ctypes.c_void_p(t) if t else None for t in (o, w, b, y)],
+                              hidden, layout, ctypes.byref(shp.c()), None)
+    assert oproj(0, A, 0, B_, 512, 0) == sp.SP_ERR_NULL
+    assert oproj(A, 0, 0, B_, 512, 0) == sp.SP_ERR_NULL
+    assert oproj(A, A, 0, 0, 512, 0) == sp.SP_ERR_NULL
+    assert oproj(A + 8, A, 0, B_, 512, 0) == sp.SP_ERR_ALIGN
+    assert oproj(A, A, C + 1, B_, 512, 0) == sp.SP_ERR_ALIGN                 # bf16 bias
+    assert oproj(A, A, 0, B_, 500, 0) == sp.SP_ERR_SHAPE                     # hidden % 8
+    assert oproj(A, A, 0, B_, 512, 3) == sp.SP_ERR_SHAPE                     # no such layout
+    assert oproj(A, A, 0, B_, 512, -1) == sp.SP_ERR_SHAPE
+    assert oproj(A, A, 0, B_, 512, 2, sp.Shape(1, 1000, 6, 128, 4)) == \
+        sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    assert oproj(A, A, 0, B_, 512, 0, sp.Shape(1, 1000, 6, 96, 4)) == sp.SP_ERR_UNSUPPORTED_D
+    # the overlapped form: push of K/V into every rank's groups, the step that
+    # waits for them
+    arr = lambda xs: None if xs is None else (ctypes.c_void_p * len(xs))(*xs)
+    grp = [A + 0x1000 * r for r in range(4)]
+    cnt = [C + 0x100 * r for r in range(4)]
+    push = lambda k, v, kg, vg, cn, epoch, rank, shp=s4: lib.sp_exchange_push(
+        ctypes.c_void_p(k) if k else None, ctypes.c_void_p(v) if v else None, arr(kg), arr(vg),
+        arr(cn), epoch, rank, ctypes.byref(shp.c()), None)
+    assert push(0, A, grp, grp, cnt, 1, 0) == sp.SP_ERR_NULL
+    assert push(A, A, None, grp, cnt, 1, 0) == sp.SP_ERR_NULL
+    assert push(A, A, grp, grp, None, 1, 0) == sp.SP_ERR_NULL
+    assert push(A, A, grp[:3] + [0], grp, cnt, 1, 0) == sp.SP_ERR_NULL
+    assert push(A + 8, A, grp, grp, cnt, 1, 0) == sp.SP_ERR_ALIGN
+    assert push(A, A, grp, grp[:3] + [A + 8], cnt, 1, 0) == sp.SP_ERR_ALIGN
+    assert push(A, A, grp, grp, cnt[:3] + [C + 4], 1, 0) == sp.SP_ERR_ALIGN   # 8-byte counters
+    assert push(A, A, grp, grp, cnt, 0, 0) == sp.SP_ERR_SHAPE                  # epoch >= 1
+    assert push(A, A, grp, grp, cnt, 1, 4) == sp.SP_ERR_SHAPE
+    assert push(A, A, grp, grp, cnt, 1, 0, sp.Shape(1, 1000, 6, 128, 4)) == \
+        sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    assert push(A * 1, A, grp * 4, grp * 4, cnt * 4, 1, 0, sp.Shape(1, 1000, 16, 128, 16)) == \
+        sp.SP_ERR_SHAPE
+    over = lambda qs, k, v, os_, cn, epoch, rank, shp=s4: lib.sp_attention_ulysses_overlap(
+        arr(qs), ctypes.c_void_p(k) if k else None, ctypes.c_void_p(v) if v else None, arr(os_),
+        None, ctypes.c_void_p(cn) if cn else None, epoch, 0, rank, ctypes.byref(shp.c()), None)
+    assert over(ok_q, A, A, ok_o, 0, 1, 0) == sp.SP_ERR_NULL
+    assert over(ok_q, A, A, ok_o, C + 4, 1, 0) == sp.SP_ERR_ALIGN
+    assert over(ok_q, A, A, ok_o, C, 0, 0) == sp.SP_ERR_SHAPE
+    assert over(ok_q, A, A, ok_o, C, 1, 4) == sp.SP_ERR_SHAPE
+    assert over(ok_q, A, A + 2, ok_o, C, 1, 0) == sp.SP_ERR_ALIGN
+    assert over(ok_q, A, A, ok_o, C, 1, 0, sp.Shape(1, 1000, 8, 64, 4)) == sp.SP_ERR_UNSUPPORTED_D
     h = (ctypes.c_uint8 * sp.IPC_HANDLE_BYTES)()
     off = ctypes.c_int64()
     base = ctypes.c_void_p()

@@ -270,10 +270,115 @@ def test_fused_peer_exchange_on_virtual_ranks(B, N, H, P):
     _check_rows(got, q, k, v, rows, P, f"peer step B={B} N={N} P={P}")
 
 
-def test_rank_classes_in_a_one_member_nccl_group():
-    """UlyssesPeerRank (CUDA IPC export, NCCL all-to-all, peer step, closing
-    all-reduce) and ulysses_attention_distributed run end to end as a
-    one-member NCCL group and give the fused call's output bit for bit."""
+def _push_blocks(shape):
+    """Pieces a push kernel counts per (tensor, destination): one CTA per 1,024
+    16-byte vectors of a chunk."""
+    chunk_vec = shape.B * shape.Nl * shape.Hl * shape.D // 8
+    return -(-chunk_vec // 1024)
+
+
+class _VirtualPushRanks:
+    """P virtual ranks of the overlapped form on one GPU: every rank's Q
+    shard, O shard, received K/V groups and arrival counters are allocations
+    of their own (standing in for peers' memory).  A step runs every rank's
+    push first and then every rank's attention step, one launch after the
+    other, so the counters are complete before any kernel looks at them."""
+
+    def __init__(self, shape):
+        self.shape = s = shape
+        self.q = [torch.empty(s.rank_shard, dtype=torch.bfloat16, device="cuda") for _ in range(s.P)]
+        self.o = [torch.full(s.rank_shard, float("nan"), dtype=torch.bfloat16, device="cuda")
+                  for _ in range(s.P)]
+        self.kg = [torch.full(s.send_chunks, float("nan"), dtype=torch.bfloat16, device="cuda")
+                   for _ in range(s.P)]
+        self.vg = [torch.full(s.send_chunks, float("nan"), dtype=torch.bfloat16, device="cuda")
+                   for _ in range(s.P)]
+        self.counts = [torch.zeros(s.P, dtype=torch.int64, device="cuda") for _ in range(s.P)]
+
+    def push(self, r, ks, vs, epoch):
+        sp.exchange_push(ks[r], vs[r], self.kg, self.vg, self.counts, epoch, self.shape, r)
+
+    def attend(self, j, epoch, lse=None, wait_ns=0):
+        sp.attention_ulysses_overlap(self.q, self.kg[j], self.vg[j], self.o, self.counts[j], epoch,
+                                     self.shape, j, lse=lse, wait_ns=wait_ns)
+
+
+@pytest.mark.parametrize("B,N,H,P", [(1, 1000, 8, 4), (1, 4096, 8, 2), (2, 777, 6, 3),
+                                     (3, 300, 16, 8), (1, 2048, 40, 8)])
+def test_overlapped_exchange_on_virtual_ranks(B, N, H, P):
+    """K and V pushed into the head groups' buffers over (stand-in) peer
+    memory and attended as they arrive: two steps with different inputs on
+    the same buffers.  The received groups equal the pinned exchange pack
+    after an all-to-all, the counters count every piece of every step, and
+    the output and LSE equal the one-GPU fused call bit for bit."""
+    D = 128
+    shape = sp.Shape(B, N, H, D, P)
+    vr = _VirtualPushRanks(shape)
+    for epoch, seed in ((1, 3 * N + P), (2, 5 * N + P)):
+        q, k, v = _random_logical(B, N, H, D, seed=seed)
+        qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+        for r in range(P):
+            vr.q[r].copy_(qs[r])
+            vr.push(r, ks, vs, epoch)
+        lses = {}
+        for j in range(P):
+            lses[j] = torch.full((B, shape.Hl, shape.Np), float("nan"), dtype=torch.float32,
+                                 device="cuda")
+            vr.attend(j, epoch, lse=lses[j])
+        _status_ok()
+        for x, groups in ((k, vr.kg), (v, vr.vg)):
+            sends = [oracle.exchange_pack(synth.to_seq_shards(x, P)[r], N, P) for r in range(P)]
+            for j in range(P):
+                want = np.stack([sends[r][j] for r in range(P)])
+                assert np.array_equal(to_host(groups[j]).reshape(want.shape), want), (epoch, j)
+        for j in range(P):
+            assert vr.counts[j].cpu().tolist() == [epoch * 2 * _push_blocks(shape)] * P
+        one, lse1 = _run_fused(q, k, v, P, lse=True)
+        got = to_host(torch.stack(vr.o))
+        assert np.array_equal(got.reshape(one.shape), one), epoch
+        Hl = H // P
+        for j in range(P):
+            assert np.array_equal(lses[j].cpu().numpy(), lse1[:, j * Hl:(j + 1) * Hl],
+                                  equal_nan=True)
+    rows = np.array([(b, h, i) for b in range(B) for h in range(H)
+                     for i in sorted({0, N - 1, *range(0, N, max(1, N // 16))})], dtype=np.int64)
+    _check_rows(got, q, k, v, rows, P, f"overlapped step B={B} N={N} P={P}")
+
+
+def test_overlap_wait_times_out_when_a_chunk_never_arrives():
+    """Step 2 of four virtual ranks, rank 1 never pushes: rank 0's attention
+    step waits for rank 1's chunk (and for its Q shard) at most 2 ms per wait,
+    gives up, drains what it has in flight and reports SP_ERR_TIMEOUT; the
+    device stays usable.  Nothing else runs that could set the counter."""
+    B, N, H, D, P = 1, 1000, 8, 128, 4
+    shape = sp.Shape(B, N, H, D, P)
+    vr = _VirtualPushRanks(shape)
+    q, k, v = _random_logical(B, N, H, D, seed=17)
+    qs, ks, vs = (to_dev(synth.to_seq_shards(x, P)) for x in (q, k, v))
+    for r in range(P):
+        vr.q[r].copy_(qs[r])
+        vr.push(r, ks, vs, 1)
+    for j in range(P):
+        vr.attend(j, 1)
+    _status_ok()
+    for r in (0, 2, 3):
+        vr.push(r, ks, vs, 2)
+    vr.attend(0, 2, wait_ns=2_000_000)
+    assert sp.device_status() == sp.SP_ERR_TIMEOUT
+    assert sp.device_status() == sp.SP_OK
+    one, _ = _run_fused(q, k, v, P)          # the context still works
+    for j in range(P):                        # and step 1's counters still count
+        vr.attend(j, 1)
+    _status_ok()
+    assert np.array_equal(to_host(torch.stack(vr.o)).reshape(one.shape), one)
+
+
+@pytest.mark.parametrize("kv_exchange", ["push", "nccl"])
+def test_rank_classes_in_a_one_member_nccl_group(kv_exchange):
+    """UlyssesPeerRank (CUDA IPC export; K/V pushed with arrival counters, or
+    exchanged by an NCCL all-to-all; peer step; closing all-reduce) and
+    ulysses_attention_distributed run end to end as a one-member NCCL group
+    and give the fused call's output bit for bit."""
     import torch.distributed as dist
     B, N, H, D = 1, 1000, 4, 128
     shape = sp.Shape(B, N, H, D, 1)
@@ -283,7 +388,7 @@ def test_rank_classes_in_a_one_member_nccl_group():
     dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
                             device_id=torch.device("cuda", torch.cuda.current_device()))
     try:
-        pr = sp.UlyssesPeerRank(shape)
+        pr = sp.UlyssesPeerRank(shape, kv_exchange=kv_exchange)
         for _ in range(2):                                 # buffers reused across steps
             out = pr.step(ks[0], vs[0], q=qs[0])
             torch.cuda.synchronize()
@@ -521,6 +626,81 @@ def test_qkv_projection_720p_sampled_rows():
     _check_proj(seq, x, w, b, rows, "projection 720p")
 
 
+def _oproj_inputs(B, N, H, D, P, hidden, seed, bias=True):
+    """An attention output in the sequence-sharded layout [P][B][Nl][H][D]
+    (padding slots zero, as attention writes them), weights [hidden][H*D]
+    scaled by 1/sqrt(H*D), an optional bias."""
+    Nl = -(-N // P)
+    o = synth.normal_bf16(seed, 0, 0, P * B * Nl * H * D, mul=0.1).reshape(P, B, Nl, H, D)
+    tok = np.arange(P)[:, None] * Nl + np.arange(Nl)[None, :]
+    o[np.broadcast_to((tok >= N)[:, None, :], (P, B, Nl))] = 0
+    w = synth.normal_bf16(seed, 1, 0, hidden * H * D, mul=1.0 / math.sqrt(H * D))
+    w = w.reshape(hidden, H * D)
+    b = synth.normal_bf16(seed, 2, 0, hidden, mul=0.1) if bias else None
+    return o, w, b
+
+
+def _run_oproj(o, w, b, shape, layout):
+    hidden = w.shape[0]
+    rows = shape.rank_shard[:2] if layout == "recv" else shape.seq_sharded[:3]
+    y = torch.full(tuple(rows) + (hidden,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.out_projection(to_dev(o), to_dev(w), None if b is None else to_dev(b), y, shape,
+                      layout=layout)
+    _status_ok()
+    return to_host(y)
+
+
+def _check_oproj(y, o_seq, w, b, rows, where):
+    """Rows of y against the fp64 oracle's linear layer on the logical O rows
+    (the bf16 rounding of y, 2^-9 relative, plus fp32 accumulation)."""
+    hidden = w.shape[0]
+    O = o_seq.reshape(-1, w.shape[1])
+    ref = oracle.linear_rows(O, w, b, rows)
+    got = synth.bf16_to_f32(y.reshape(-1, hidden)[rows]).astype(np.float64)
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-4 * np.max(np.abs(ref))
+    assert np.all(err <= bound), (where, float((err - bound).max()))
+
+
+@pytest.mark.parametrize("B,N,H,D,P,hidden,bias", [
+    (1, 1000, 4, 128, 2, 512, True), (2, 333, 6, 64, 3, 200, False),
+    (1, 4096, 12, 128, 4, 1536, True), (3, 130, 2, 64, 1, 72, True),
+    (2, 517, 8, 128, 8, 264, True)])
+def test_out_projection_layouts(B, N, H, D, P, hidden, bias):
+    """The output projection against the fp64 oracle on every row, reading O
+    as sequence shards; reading O as head groups (the pinned pack of it) and,
+    per rank, as the chunks returned to that rank (the pinned exchange pack of
+    its shard) gives the same y bit for bit."""
+    shape = sp.Shape(B, N, H, D, P)
+    o, w, b = _oproj_inputs(B, N, H, D, P, hidden, seed=hidden + N + 7, bias=bias)
+    y = _run_oproj(o, w, b, shape, "seq")
+    _check_oproj(y, o, w, b, np.arange(P * B * shape.Nl), f"out projection {B},{N},{H},{D},{P}")
+    yh = _run_oproj(oracle.pack(o, N), w, b, shape, "head")
+    assert np.array_equal(yh, y)
+    for r in range(P):
+        recv = oracle.exchange_pack(np.ascontiguousarray(o[r]), N, P)
+        yr = _run_oproj(recv, w, b, shape, "recv")
+        assert np.array_equal(yr.reshape(shape.rank_shard[:2] + (hidden,)),
+                              y.reshape(shape.seq_sharded[:3] + (hidden,))[r])
+
+
+def test_out_projection_720p_sampled_rows():
+    """The 720p-shaped output projection (75,600 tokens, 5,120 attention
+    features to hidden 5,120) on sampled rows against the oracle; the rank-1
+    chunk layout (P = 4) bit for bit against the sequence-shard call."""
+    cfg = synth.CONFIGS["720p"]
+    s = cfg.shape
+    shape = sp.Shape(s.B, s.N, s.H, s.D, s.P)
+    o, w, b = _oproj_inputs(s.B, s.N, s.H, s.D, s.P, s.H * s.D, seed=73)
+    y = _run_oproj(o, w, b, shape, "seq")
+    rows = np.unique(np.concatenate([[0, s.N - 1, 18899, 18900],
+                                     np.random.default_rng(73).integers(0, s.N, 40)]))
+    _check_oproj(y, o, w, b, rows, "out projection 720p")
+    recv = oracle.exchange_pack(np.ascontiguousarray(o[1]), s.N, s.P)
+    yr = _run_oproj(recv, w, b, shape, "recv")
+    assert np.array_equal(yr.reshape(-1), y.reshape(s.P, -1)[1])
+
+
 # ------------------------------------------------------------------ guard bands
 
 GUARD = 4096  # elements of sentinel after every output buffer
@@ -573,6 +753,16 @@ def test_outputs_stay_inside_their_buffers():
     words = torch.from_numpy(sp.sparse_mask_words(mask).view(np.int32)).cuda()
     osp, c = _guarded(shape.seq_sharded, torch.bfloat16); checks.append(c)
     sp.attention_sparse_seqsharded(qs, ks, vs, words, osp, shape)
+
+    # the output projection from each O layout (hidden 264: a partial last
+    # 32-feature chunk and a partial last 256-feature tile)
+    hidden = 264
+    wo = to_dev(synth.normal_bf16(43, 1, 0, hidden * H * D, mul=0.05).reshape(hidden, H * D))
+    bo = to_dev(synth.normal_bf16(43, 2, 0, hidden, mul=0.1))
+    for layout, src, rows in (("seq", of, shape.seq_sharded[:3]), ("head", oh, shape.seq_sharded[:3]),
+                              ("recv", send, shape.rank_shard[:2])):
+        y, c = _guarded(tuple(rows) + (hidden,), torch.bfloat16); checks.append(c)
+        sp.out_projection(src, wo, bo, y, shape, layout=layout)
 
     q8, k8, v8, f = _fp8_inputs(B, N, H, D, seed=41)
     dev8 = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, P))).cuda()

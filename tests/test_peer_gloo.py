@@ -10,7 +10,14 @@ group's head columns.  The test checks the handle exchange, the address
 tables in rank order, the K/V exchange that feeds the peer step, and the
 closing collective that orders the peers' O stores before a rank reads its
 shard: rank 0's peer step is delayed, so a rank that read its shard too
-early would miss head group 0."""
+early would miss head group 0.
+
+With kv_exchange="push" the backend also plays sp_exchange_push (rank r
+writes its chunk for group j into rank j's received groups at slot r, then
+raises rank j's arrival counter for r to the step number) and the waiting
+side of sp_attention_ulysses_overlap (the step starts on the received groups
+only once every counter shows this step).  Rank P-1 pushes late, so a rank
+that did not wait for its chunks would attend stale K/V."""
 import math
 import os
 import socket
@@ -28,7 +35,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _peer_rank_main(rank, world, port, q, shape_args):
+def _peer_rank_main(rank, world, port, q, shape_args, kv_exchange):
     sys.path.insert(0, ROOT)
     import datetime
     import time
@@ -64,20 +71,45 @@ def _peer_rank_main(rank, world, port, q, shape_args):
             self.own[t.data_ptr()] = shm
             return t
 
+        zeros = empty
+
         def export(self, t):
             return self.own[t.data_ptr()].name, 0   # the whole block
 
         def open(self, name, offset):
+            """A peer's block as raw bytes (the product code only passes it on)."""
             assert offset == 0
             shm = shared_memory.SharedMemory(name=name)
             resource_tracker.unregister(shm._name, "shared_memory")  # the owner unlinks it
             self.maps.append(shm)
-            shp = (2,) + tuple(self.shape.rank_shard)
-            return torch.frombuffer(shm.buf, dtype=torch.bfloat16, count=math.prod(shp)).view(shp)
+            return torch.frombuffer(shm.buf, dtype=torch.uint8, count=shm.size)
 
         @staticmethod
         def part(x, i, shape):
+            if x.dtype == torch.uint8:
+                return x.view(torch.bfloat16).view(2, -1)[i]
             return x[i]
+
+        @staticmethod
+        def _counts(x):
+            return x.view(torch.int64) if x.dtype == torch.uint8 else x
+
+        def push(self, k, v, k_addrs, v_addrs, count_addrs, epoch, r, shape):
+            if r == shape.P - 1:
+                time.sleep(0.5)                                   # a late pusher
+            for x, dst in ((k, k_addrs), (v, v_addrs)):
+                send = oracle.exchange_pack(words(x), shape.N, shape.P)   # [P][B][Nl][Hl][D]
+                for j in range(shape.P):
+                    words(dst[j]).reshape(send.shape)[r] = send[j]
+            for j in range(shape.P):
+                self._counts(count_addrs[j])[r] = epoch
+
+        def overlap_step(self, q_addrs, k_group, v_group, o_addrs, counts, epoch, j, shape):
+            t0 = time.time()
+            while int(counts.min()) < epoch:                      # every chunk of this step
+                assert time.time() - t0 < 30, "chunks never arrived"
+                time.sleep(0.01)
+            self.peer_step(q_addrs, k_group, v_group, o_addrs, j, shape)
 
         def exchange_pack(self, x, send, shape):
             send.copy_(bf16(oracle.exchange_pack(words(x), shape.N, shape.P)))
@@ -87,14 +119,16 @@ def _peer_rank_main(rank, world, port, q, shape_args):
                 time.sleep(0.5)
             N, H, P = shape.N, shape.H, shape.P
             Hl = H // P
-            q_all = np.stack([words(x) for x in q_addrs])             # [P][B][Nl][H][D]
+            shard = tuple(shape.rank_shard)
+            q_all = np.stack([words(x).reshape(shard) for x in q_addrs])   # [P][B][Nl][H][D]
             qg = synth.from_seq_shards(q_all, N)[:, :, j * Hl:(j + 1) * Hl]
-            kg, vg = (synth.from_seq_shards(words(x), N) for x in (k_group, v_group))
+            kg, vg = (synth.from_seq_shards(words(x).reshape(shape.send_chunks), N)
+                      for x in (k_group, v_group))
             O, _ = oracle.attention_full(np.ascontiguousarray(qg), kg, vg,
                                          scale=1.0 / np.sqrt(shape.D), threads=1)
             o_sh = synth.to_seq_shards(synth.f32_to_bf16(O.astype(np.float32)), P)
             for r in range(P):
-                words(o_addrs[r])[:, :, j * Hl:(j + 1) * Hl] = o_sh[r]
+                words(o_addrs[r]).reshape(shard)[:, :, j * Hl:(j + 1) * Hl] = o_sh[r]
 
         def close(self):
             for shm in self.maps:
@@ -114,7 +148,7 @@ def _peer_rank_main(rank, world, port, q, shape_args):
         P = world
         shape = sp.Shape(B, N, H, D, P)
         be = ShmBackend(shape)
-        pr = sp.UlyssesPeerRank(shape, backend=be)
+        pr = sp.UlyssesPeerRank(shape, backend=be, kv_exchange=kv_exchange)
         results = []
         for seed in (31, 32):                                     # two steps, buffers reused
             cfg = synth.Config("p", synth.Shape(B, N, H, D, 1), seed=seed)
@@ -132,12 +166,13 @@ def _peer_rank_main(rank, world, port, q, shape_args):
 
 
 @pytest.mark.timeout(240)
+@pytest.mark.parametrize("kv_exchange", ["push", "nccl"])
 @pytest.mark.parametrize("world,shape_args", [(2, (1, 100, 4, 16)), (4, (2, 37, 8, 16))])
-def test_peer_rank_host_logic(world, shape_args):
+def test_peer_rank_host_logic(world, shape_args, kv_exchange):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_peer_rank_main, args=(r, world, port, q, shape_args))
+    procs = [ctx.Process(target=_peer_rank_main, args=(r, world, port, q, shape_args, kv_exchange))
              for r in range(world)]
     for p in procs:
         p.start()

@@ -43,7 +43,8 @@ EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_launch_count", "sp_status_str", "sp_selftest_wait_timeout",
             "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded",
             "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close",
-            "sp_attention_sparse_seqsharded", "sp_qkv_projection")
+            "sp_attention_sparse_seqsharded", "sp_qkv_projection", "sp_out_projection",
+            "sp_exchange_push", "sp_attention_ulysses_overlap")
 
 
 class sp_shape(ctypes.Structure):
@@ -87,11 +88,20 @@ def load(path: str = LIB_PATH):
     lib.sp_qkv_projection.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int32, ctypes.c_int32,
                                       sp_p, vp]
     lib.sp_qkv_projection.restype = ctypes.c_int
+    lib.sp_out_projection.argtypes = [vp, vp, vp, vp, ctypes.c_int32, ctypes.c_int32, sp_p, vp]
+    lib.sp_out_projection.restype = ctypes.c_int
     lib.sp_attention_sparse_seqsharded.argtypes = [vp, vp, vp, vp, vp, vp, sp_p, vp]
     lib.sp_attention_sparse_seqsharded.restype = ctypes.c_int
     lib.sp_attention_ulysses_peer.argtypes = [
         ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), vp, ctypes.c_int32, sp_p, vp]
     lib.sp_attention_ulysses_peer.restype = ctypes.c_int
+    lib.sp_exchange_push.argtypes = [vp, vp, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                     ctypes.POINTER(vp), ctypes.c_uint64, ctypes.c_int32, sp_p, vp]
+    lib.sp_exchange_push.restype = ctypes.c_int
+    lib.sp_attention_ulysses_overlap.argtypes = [
+        ctypes.POINTER(vp), vp, vp, ctypes.POINTER(vp), vp, vp, ctypes.c_uint64, ctypes.c_uint64,
+        ctypes.c_int32, sp_p, vp]
+    lib.sp_attention_ulysses_overlap.restype = ctypes.c_int
     lib.sp_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int64)]
     lib.sp_ipc_export.restype = ctypes.c_int
     lib.sp_ipc_open.argtypes = [vp, ctypes.POINTER(vp)]
@@ -343,31 +353,53 @@ class UlyssesRank:
       finish(back)        P returned chunks -> this rank's output shard
                           (sp_exchange_unpack)
     Keeping the phases apart lets the caller choose the exchange (NCCL over
-    NVLink, or a copy between virtual ranks on one GPU)."""
+    NVLink, or a copy between virtual ranks on one GPU).  The buffers a phase
+    returns belong to this object and are reused by the next step: each
+    step overwrites the previous step's results."""
 
     def __init__(self, shape: Shape):
         self.shape = shape
+        self._bufs = {}
+
+    def _buf(self, name, shape, like):
+        torch = _torch()
+        b = self._bufs.get(name)
+        if b is None or b.device != like.device or b.dtype != like.dtype:
+            b = self._bufs[name] = torch.empty(shape, dtype=like.dtype, device=like.device)
+        return b
 
     def send_qkv(self, q, k, v, stream=None):
-        torch = _torch()
         out = []
-        for x in (q, k, v):
-            send = torch.empty(self.shape.send_chunks, dtype=x.dtype, device=x.device)
+        for name, x in (("send_q", q), ("send_k", k), ("send_v", v)):
+            send = self._buf(name, self.shape.send_chunks, x)
             exchange_pack(x, send, self.shape, stream)
             out.append(send)
         return out
 
+    def recv_buffers(self, like):
+        """Three [P][B][Nl][Hl][D] buffers for the received Q, K, V chunks."""
+        return [self._buf(n, self.shape.send_chunks, like) for n in ("recv_q", "recv_k", "recv_v")]
+
     def attend(self, q, k, v, lse=None, stream=None):
-        torch = _torch()
-        o = torch.empty_like(q)
+        o = self._buf("o", self.shape.send_chunks, q)
         attention_seqsharded(q, k, v, o, self.shape.head_group(), lse=lse, stream=stream)
         return o
 
     def finish(self, back, stream=None):
-        torch = _torch()
-        out = torch.empty(self.shape.rank_shard, dtype=back.dtype, device=back.device)
+        out = self._buf("out", self.shape.rank_shard, back)
         exchange_unpack(back, out, self.shape, stream)
         return out
+
+    def step(self, q, k, v, all_to_all):
+        """The whole step with all_to_all(send, recv) filling recv: returns
+        this rank's output shard (this object's buffer)."""
+        recv = self.recv_buffers(q)
+        for send, r in zip(self.send_qkv(q, k, v), recv):
+            all_to_all(send, r)
+        o = self.attend(*recv)
+        back = self._buf("back", self.shape.send_chunks, o)
+        all_to_all(o, back)
+        return self.finish(back)
 
 
 QKV_LAYOUTS = {"seq": 0, "head": 1, "send": 2}   # sp_qkv_layout
@@ -393,6 +425,29 @@ def qkv_projection(x, w, bias, q, k, v, shape: Shape, layout: str = "seq", strea
             _ptr(bias, (3 * shape.H * shape.D,), "bias"), _ptr(q, out, "q"), _ptr(k, out, "k"),
             _ptr(v, out, "v"), hidden, QKV_LAYOUTS[layout], ctypes.byref(s),
             _stream(stream, x.device)), "sp_qkv_projection")
+
+
+O_LAYOUTS = {"seq": 0, "head": 1, "recv": 2}     # sp_o_layout
+
+
+def out_projection(o, w, bias, y, shape: Shape, layout: str = "seq", stream=None):
+    """The projection after attention (sp_out_projection), arguments in the C
+    order: o the attention output in `layout` -- "seq" [P][B][Nl][H][D],
+    "head" [P][B][Np][Hl][D] or "recv" one rank's P returned chunks
+    [P][B][Nl][Hl][D] --, w [hidden][H*D], bias [hidden] or None, all bf16;
+    y receives [P][B][Nl][hidden] (one rank's [B][Nl][hidden] for "recv")."""
+    if layout not in O_LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(O_LAYOUTS)}")
+    hidden = int(w.shape[0])
+    o_shape = {"seq": shape.seq_sharded, "head": shape.head_sharded,
+               "recv": shape.send_chunks}[layout]
+    rows = shape.rank_shard[:2] if layout == "recv" else shape.seq_sharded[:3]
+    s = shape.c()
+    with _same_device(o, w, bias, y):
+        _check(load().sp_out_projection(
+            _ptr(o, o_shape, "o"), _ptr(w, (hidden, shape.H * shape.D), "w"),
+            _ptr(bias, (hidden,), "bias"), _ptr(y, tuple(rows) + (hidden,), "y"), hidden,
+            O_LAYOUTS[layout], ctypes.byref(s), _stream(stream, o.device)), "sp_out_projection")
 
 
 SPARSE_CUBE = 64         # SP_SPARSE_CUBE
@@ -480,6 +535,63 @@ def _require_ipc_exportable():
                 "allocations; unset it for the peer exchange")
 
 
+def _addr_array(xs, shape_, name):
+    """ctypes array of device addresses: CUDA tensors (checked against
+    shape_) or ints (peer addresses valid in this process)."""
+    def addr(x, i):
+        if isinstance(x, int):
+            return x
+        if shape_ is None:
+            if not isinstance(x, _torch().Tensor) or not x.is_cuda:
+                raise TypeError(f"{name}[{i}] must be a CUDA tensor or an address")
+            return x.data_ptr()
+        return _ptr(x, shape_, f"{name}[{i}]").value
+    return (ctypes.c_void_p * len(xs))(*[addr(x, i) for i, x in enumerate(xs)])
+
+
+def exchange_push(k, v, k_groups, v_groups, counts, epoch: int, shape: Shape, rank: int,
+                  stream=None):
+    """One rank's K/V exchange over peer memory (sp_exchange_push): k, v this
+    rank's shards [B][Nl][H][D]; k_groups / v_groups / counts: P entries in
+    rank order, each a CUDA tensor or a peer address (ipc_open) -- every
+    rank's received groups [P][B][Nl][Hl][D] bf16 and arrival counters
+    int64 [P]; epoch: the step number (>= 1)."""
+    torch = _torch()
+    P = shape.P
+    if not (len(k_groups) == len(v_groups) == len(counts) == P):
+        raise ValueError(f"need {P} entries per address list")
+    local = [x for x in (*k_groups, *v_groups, *counts) if not isinstance(x, int)]
+    s = shape.c()
+    with _same_device(k, v, *local):
+        _check(load().sp_exchange_push(
+            _ptr(k, shape.rank_shard, "k"), _ptr(v, shape.rank_shard, "v"),
+            _addr_array(k_groups, shape.send_chunks, "k_groups"),
+            _addr_array(v_groups, shape.send_chunks, "v_groups"),
+            _addr_array(counts, None, "counts"), int(epoch), int(rank), ctypes.byref(s),
+            _stream(stream, k.device)), "sp_exchange_push")
+
+
+def attention_ulysses_overlap(q_shards, k_group, v_group, o_shards, counts, epoch: int,
+                              shape: Shape, rank: int, lse=None, wait_ns: int = 0, stream=None):
+    """The peer step while K/V chunks arrive (sp_attention_ulysses_overlap):
+    as attention_ulysses_peer, and counts is this rank's arrival counters
+    (int64 [P], CUDA tensor) for step `epoch`."""
+    torch = _torch()
+    P = shape.P
+    if len(q_shards) != P or len(o_shards) != P:
+        raise ValueError(f"need {P} Q and {P} O shard addresses")
+    local = [x for x in (*q_shards, *o_shards) if not isinstance(x, int)]
+    s = shape.c()
+    group = shape.send_chunks
+    with _same_device(k_group, v_group, counts, lse, *local):
+        _check(load().sp_attention_ulysses_overlap(
+            _addr_array(q_shards, shape.rank_shard, "q_shards"), _ptr(k_group, group, "k_group"),
+            _ptr(v_group, group, "v_group"), _addr_array(o_shards, shape.rank_shard, "o_shards"),
+            _ptr(lse, (shape.B, shape.Hl, shape.Np), "lse", torch.float32),
+            _ptr(counts, (P,), "counts", torch.int64), int(epoch), int(wait_ns), int(rank),
+            ctypes.byref(s), _stream(stream, k_group.device)), "sp_attention_ulysses_overlap")
+
+
 def ipc_export(t):
     """(handle, offset): the CUDA IPC handle (bytes) of the allocation that
     holds CUDA tensor t, and t's byte offset from that allocation's base."""
@@ -519,6 +631,13 @@ class CudaPeerBackend:
         torch = _torch()
         return torch.empty(shape, dtype=dtype or torch.bfloat16, device=self.device)
 
+    def zeros(self, shape, dtype=None):
+        """Zeroed and complete on the device before any peer can see it."""
+        torch = _torch()
+        t = torch.zeros(shape, dtype=dtype or torch.bfloat16, device=self.device)
+        torch.cuda.synchronize(self.device)
+        return t
+
     def export(self, t):
         _require_ipc_exportable()
         return ipc_export(t)
@@ -544,6 +663,13 @@ class CudaPeerBackend:
     def peer_step(self, q_addrs, k_group, v_group, o_addrs, rank: int, shape: Shape):
         attention_ulysses_peer(q_addrs, k_group, v_group, o_addrs, shape, rank)
 
+    def push(self, k, v, k_addrs, v_addrs, count_addrs, epoch: int, rank: int, shape: Shape):
+        exchange_push(k, v, k_addrs, v_addrs, count_addrs, epoch, shape, rank)
+
+    def overlap_step(self, q_addrs, k_group, v_group, o_addrs, counts, epoch: int, rank: int,
+                     shape: Shape):
+        attention_ulysses_overlap(q_addrs, k_group, v_group, o_addrs, counts, epoch, shape, rank)
+
     def close(self):
         torch = _torch()
         with torch.cuda.device(self.device):
@@ -553,29 +679,40 @@ class CudaPeerBackend:
 
 
 class UlyssesPeerRank:
-    """One rank of the multi-GPU form with the Q and O exchanges fused into
-    the attention kernel.
+    """One rank of the multi-GPU form with the exchanges fused into the
+    kernels.
 
     Construction allocates this rank's Q shard and output shard
-    ([B][Nl][H][D] each, one buffer), exports it, gathers every rank's export
-    over the process group and maps the peers' buffers (each once), so that
-    every rank holds the P Q-shard and P O-shard addresses in rank order.  step(k, v, q) then
-      writes q into the Q shard (or the caller wrote it),
-      reorders k and v into send chunks (sp_exchange_pack) and exchanges
-        them (all-to-all: chunk j of every rank to rank j),
-      runs the peer step (Q tiles read from the ranks that hold them, O rows
-        stored into the ranks that own them),
+    ([B][Nl][H][D] each, one buffer) and, with kv_exchange="push" (the
+    default), its received K and V groups ([P][B][Nl][Hl][D] each, one
+    buffer) and its arrival counters (int64 [P], zeroed); it exports them,
+    gathers every rank's exports over the process group and maps the peers'
+    buffers (each once), so that every rank holds all ranks' addresses in rank
+    order.  step(k, v, q) then
+      writes q into the Q shard (or the caller wrote it);
+      push: stores k and v straight into every rank's received groups over
+        peer memory (sp_exchange_push), and runs the attention step that
+        waits for each chunk as it arrives (sp_attention_ulysses_overlap):
+        Q tiles read from the ranks that hold them, O rows stored into the
+        ranks that own them;
+      nccl: reorders k and v into send chunks (sp_exchange_pack), exchanges
+        them with an all-to-all, then runs the peer step
+        (sp_attention_ulysses_peer);
       and ends with a one-element all-reduce.
-    The all-to-all follows every rank's Q write in that rank's stream order,
-    so when it completes here every Q shard is complete; the closing
+    A rank's Q write precedes its push (or its all-to-all) in its stream, so
+    a peer that has seen the chunk has seen the Q shard; the closing
     all-reduce follows every rank's kernel, so when it completes here every
-    row of this rank's output shard has been written.  The returned output
-    shard stays valid until the next step."""
+    row of this rank's output shard has been written and no peer still reads
+    a buffer the next step overwrites.  The returned output shard stays valid
+    until the next step."""
 
-    def __init__(self, shape: Shape, group=None, backend=None, device=None):
+    def __init__(self, shape: Shape, group=None, backend=None, device=None,
+                 kv_exchange: str = "push"):
         import torch.distributed as dist
         torch = _torch()
-        self.shape, self.group = shape, group
+        if kv_exchange not in ("push", "nccl"):
+            raise ValueError("kv_exchange must be 'push' or 'nccl'")
+        self.shape, self.group, self.kv_exchange = shape, group, kv_exchange
         self.rank = dist.get_rank(group)
         if dist.get_world_size(group) != shape.P:
             raise ValueError(f"group of {dist.get_world_size(group)} ranks, shape has P = {shape.P}")
@@ -586,27 +723,48 @@ class UlyssesPeerRank:
         self.backend = be = backend
         self._qo = be.empty((2,) + tuple(shape.rank_shard))     # [Q shard, O shard]
         self.q_shard, self.o_shard = self._qo[0], self._qo[1]
-        self._k_send, self._v_send, self._k_recv, self._v_recv = (
-            be.empty(shape.send_chunks) for _ in range(4))
         self._flag = be.empty((1,), torch.float32)
+        self.epoch = 0
+        push = kv_exchange == "push"
+        if push:
+            self._kv = be.empty((2,) + tuple(shape.send_chunks))  # [K group, V group]
+            self.counts = be.zeros((shape.P,), torch.int64)
+            mine = (be.export(self._qo), be.export(self._kv), be.export(self.counts))
+        else:
+            self._k_send, self._v_send, self._k_recv, self._v_recv = (
+                be.empty(shape.send_chunks) for _ in range(4))
+            mine = (be.export(self._qo),)
         table = [None] * shape.P
-        dist.all_gather_object(table, be.export(self._qo), group=group)
+        dist.all_gather_object(table, mine, group=group)
         self.q_addrs, self.o_addrs = [], []
+        self.k_addrs, self.v_addrs, self.count_addrs = [], [], []
         for r, exported in enumerate(table):
-            x = self._qo if r == self.rank else be.open(*exported)
-            self.q_addrs.append(be.part(x, 0, shape))
-            self.o_addrs.append(be.part(x, 1, shape))
+            own = r == self.rank
+            qo = self._qo if own else be.open(*exported[0])
+            self.q_addrs.append(be.part(qo, 0, shape))
+            self.o_addrs.append(be.part(qo, 1, shape))
+            if push:
+                kv = self._kv if own else be.open(*exported[1])
+                self.k_addrs.append(be.part(kv, 0, shape))
+                self.v_addrs.append(be.part(kv, 1, shape))
+                self.count_addrs.append(self.counts if own else be.open(*exported[2]))
 
     def step(self, k, v, q=None):
         import torch.distributed as dist
         be, s = self.backend, self.shape
         if q is not None:
             self.q_shard.copy_(q)
-        be.exchange_pack(k, self._k_send, s)
-        be.exchange_pack(v, self._v_send, s)
-        dist.all_to_all_single(self._k_recv, self._k_send, group=self.group)
-        dist.all_to_all_single(self._v_recv, self._v_send, group=self.group)
-        be.peer_step(self.q_addrs, self._k_recv, self._v_recv, self.o_addrs, self.rank, s)
+        self.epoch += 1
+        if self.kv_exchange == "push":
+            be.push(k, v, self.k_addrs, self.v_addrs, self.count_addrs, self.epoch, self.rank, s)
+            be.overlap_step(self.q_addrs, self._kv[0], self._kv[1], self.o_addrs, self.counts,
+                            self.epoch, self.rank, s)
+        else:
+            be.exchange_pack(k, self._k_send, s)
+            be.exchange_pack(v, self._v_send, s)
+            dist.all_to_all_single(self._k_recv, self._k_send, group=self.group)
+            dist.all_to_all_single(self._v_recv, self._v_send, group=self.group)
+            be.peer_step(self.q_addrs, self._k_recv, self._v_recv, self.o_addrs, self.rank, s)
         self._flag.zero_()
         dist.all_reduce(self._flag, group=self.group)
         return self.o_shard
@@ -621,25 +779,29 @@ class UlyssesPeerRank:
 
 def nccl_all_to_all(group=None):
     """Exchange through torch.distributed: chunk j of this rank's [P][...]
-    buffer goes to rank j; the result holds every rank's chunk in rank order."""
+    buffer goes to rank j; the result holds every rank's chunk in rank order.
+    exchange(send, recv=None) fills recv (a new buffer when None) and
+    returns it."""
     import torch.distributed as dist
 
-    def exchange(send):
+    def exchange(send, recv=None):
         torch = _torch()
-        recv = torch.empty_like(send)
+        if recv is None:
+            recv = torch.empty_like(send)
         dist.all_to_all_single(recv, send, group=group)
         return recv
     return exchange
 
 
-def ulysses_attention_distributed(q, k, v, shape: Shape, all_to_all=None):
+def ulysses_attention_distributed(q, k, v, shape: Shape, all_to_all=None, rank=None):
     """One rank's Ulysses attention step: q, k, v are this rank's shards
     [B][Nl][H][D] (rank = position in the group of shape.P ranks); returns
-    the output shard.  all_to_all defaults to NCCL over the default group."""
+    the output shard.  all_to_all defaults to NCCL over the default group.
+    Pass the same UlyssesRank as `rank` on every step to reuse its buffers
+    (the returned shard is then overwritten by the next step)."""
     all_to_all = all_to_all or nccl_all_to_all()
-    rank = UlyssesRank(shape)
-    rq, rk, rv = (all_to_all(x) for x in rank.send_qkv(q, k, v))
-    return rank.finish(all_to_all(rank.attend(rq, rk, rv)))
+    rank = rank or UlyssesRank(shape)
+    return rank.step(q, k, v, all_to_all)
 
 
 class HostPipeline:

@@ -72,6 +72,15 @@ struct AttnParams {
   // tokens; bit c of word w in query cube qc's row selects key cube 32w + c.
   const uint32_t *mask;
   int32_t ncube, nwords;
+  // Peer step with the K/V exchange overlapped (null: everything has
+  // arrived before the launch).  counts[r] counts the finished pieces of
+  // source rank r's K/V chunk (and, through stream order on rank r, covers
+  // its Q shard); the chunk has arrived when counts[r] >= count_target.
+  // Tokens of chunk r are r*count_nl .. r*count_nl + count_nl - 1.
+  const unsigned long long *counts;
+  unsigned long long count_target;
+  int32_t count_nl;
+  uint64_t count_wait_ns;
 };
 
 constexpr int32_t kStatusTimeout = 7;
@@ -120,7 +129,7 @@ struct AttnCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
-  static constexpr int kNumBar = 1 + 2 * kStages + 8;
+  static constexpr int kNumBar = 1 + 2 * kStages + 9;  // ..., bar_o[2], bar_drain
   static constexpr int kOffMisc = kOffBar + kNumBar * 8;
   // Block-sparse variant: one bit per key tile, set when any query cube of
   // the CTA selects either key cube of the tile.
@@ -177,6 +186,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   const uint32_t bar_s = bar_kv_empty + 8 * C::kStages;  // [2]
   const uint32_t bar_p = bar_s + 16;                      // [2 tiles][2 key halves]
   const uint32_t bar_o = bar_p + 32;                      // [2]
+  const uint32_t bar_drain = bar_o + 16;                  // the MMA thread's last commit
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sptr + C::kOffMisc + 4);
   uint32_t *sel_bits = reinterpret_cast<uint32_t *>(sptr + C::kOffSel);
@@ -228,6 +238,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       mbar_init(bar_p + 16 * t + 8, 128);
       mbar_init(bar_o + 8 * t, 1);
     }
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -241,6 +252,10 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
+  // K/V ring loads this thread issued (the TMA producer's lane 0): on the
+  // abort path the last kStages of them may still be in flight.
+  int issued = 0;
+  bool q_issued = false;
   // Block-sparse kernel: 12 warps, so that its per-row mask state fits.  The
   // third warpgroup (TMA, MMA and two idle warps) gives registers to the two
   // softmax warpgroups: 384 x 168 at launch = 2 x 128 x 208 + 128 x 88, and
@@ -290,11 +305,33 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
           const int rk = tok / nl, n = tok - rk * nl;
           const int64_t off = ((static_cast<int64_t>(rk) * p.B + b) * nl + n) * p.H * C::kRowBytes +
                               static_cast<int64_t>(map_head) * C::kRowBytes + cc * 16;
-          val = ld_global_nc_v4(base + off);
+          // the peer step's K/V may arrive while the kernel runs: no
+          // non-coherent loads there
+          val = kPeer ? ld_global_v4(base + off) : ld_global_nc_v4(base + off);
         }
         st_shared_v4(dst + (cc >> 3) * C::kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4), val);
       }
       fence_proxy_async_smem();
+    };
+    // Overlapped peer step: before the first load of tokens t0 .. t1, lane 0
+    // waits (bounded) until the chunk of every rank holding one of them has
+    // arrived, then orders its later TMA loads after that observation; the
+    // other lanes' loads follow through __shfl_sync.  `arrived` (lane 0 only)
+    // keeps the ranks already seen.
+    uint32_t arrived = 0u;
+    auto await_tokens = [&](int t0, int t1) -> bool {
+      if (!kPeer || p.counts == nullptr) return true;
+      bool good = true;
+      if (lane == 0) {
+        const int last = t1 < p.N - 1 ? t1 : p.N - 1;
+        for (int r = t0 / p.count_nl; t0 <= last && r <= last / p.count_nl && good; ++r) {
+          if ((arrived >> r) & 1u) continue;
+          good = wait_counter_geq(p.counts + r, p.count_target, abort_flag, p.count_wait_ns);
+          if (good) arrived |= 1u << r;
+        }
+        if (good) fence_proxy_async_global();
+      }
+      return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
     };
     // Peer Q: a tile inside one rank's shard is one TMA box per column block
     // from that rank's map; a tile that crosses ranks is gathered row by row.
@@ -320,8 +357,9 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       fence_proxy_async_smem();
     };
     // Q: both tiles complete one barrier.
+    ok = await_tokens(q0, q0 + 2 * C::kBM - 1);
     uint32_t q_tx = 0;
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < 2 && ok; ++t) {
       const uint32_t dst = sbase + C::kOffQ + t * C::kTileBytes;
       if (kPeer) {
         if (peer_q_ok(q0 + t * C::kBM)) q_tx += C::kTileBytes;
@@ -332,7 +370,8 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       }
     }
     __syncwarp();
-    if (lane == 0) {
+    q_issued = ok;
+    if (lane == 0 && ok) {
       mbar_arrive_expect_tx(bar_q, q_tx);
       for (int t = 0; t < 2; ++t) {
         const int t0 = q0 + t * C::kBM;
@@ -351,6 +390,10 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
     }
     int it = 0;
     for (int j = next_tile(-1); j < T && ok; j = next_tile(j)) {
+      if (!await_tokens(j * C::kBN, j * C::kBN + C::kBN - 1)) {
+        ok = false;
+        break;
+      }
       for (int kv = 0; kv < 2; ++kv, ++it) {
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
@@ -372,6 +415,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
           if (lane == 0) mbar_arrive(bar);
         }
         __syncwarp();
+        issued = it + 1;
       }
     }
   } else if (warp == 9) {
@@ -704,11 +748,22 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {
-    // Let copies and MMAs already in flight land before the CTA's shared and
-    // tensor memory are released (bounded: 50 us).
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 50000ull) {
+    // Before the CTA's shared and tensor memory are released, let the
+    // asynchronous work it issued land: the TMA copies of Q and of the last
+    // kStages ring loads (earlier slots were consumed, so they landed), and
+    // every MMA the issuing thread enqueued (one more commit, then its
+    // barrier).  None of these depends on another thread, so each bounded
+    // wait ends; if one does not, the status word already holds the error.
+    if (warp == 8 && lane == 0) {
+      if (q_issued) mbar_wait_drain(bar_q, 0, kWaitLimitNs);
+      for (int i = issued > C::kStages ? issued - C::kStages : 0; i < issued; ++i)
+        mbar_wait_drain(bar_kv_full + 8 * (i % C::kStages), (i / C::kStages) & 1, kWaitLimitNs);
     }
+    if (warp == 9 && lane == 0) {
+      umma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, kWaitLimitNs);
+    }
+    __syncthreads();
   }
   if (warp == 9) {
     tc_fence_after();

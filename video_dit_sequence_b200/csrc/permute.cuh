@@ -151,4 +151,65 @@ permute_kernel(const PermuteParams p) {
   }
 }
 
+// ------------------------------------------------------------------ push
+// One rank's K/V exchange over peer memory, for the multi-GPU form in which
+// the attention kernel overlaps the arrival of the K/V chunks: rank `rank`
+// stores its chunk for head group j straight into rank j's received-group
+// buffers (the exchange pack fused with the transfer; no send buffer, no
+// all-to-all), at chunk slot `rank`:
+//   group_j[rank][b][n][hh][:] = x_rank[b][n][j*Hl + hh][:]     (x = K, V)
+// and then counts itself done in rank j's arrival counter for source `rank`.
+// A CTA covers kPermThreads * kPermUnroll vectors of one (tensor, j) chunk;
+// rank j's counter for this rank reaches 2 * blocks_per_chunk per step (K
+// and V), so after step e it is e * 2 * blocks_per_chunk.
+constexpr int kMaxPushPeers = 8;
+
+struct PushParams {
+  const uint4 *src[2];                            // this rank's K and V shards
+  uint4 *dst[2][kMaxPushPeers];                   // rank j's received K and V groups
+  unsigned long long *count[kMaxPushPeers];       // rank j's arrival counters [P]
+  FastDiv vr;                                     // vectors per run: Hl*D/8
+  uint32_t chunk_vec;                             // vectors of one chunk: B*Nl*Hl*D/8
+  uint32_t H_vec, Hl_vec;
+  uint32_t rank;
+};
+
+__host__ __device__ constexpr uint32_t push_blocks_per_chunk(uint32_t chunk_vec) {
+  return (chunk_vec + kPermThreads * kPermUnroll - 1) / (kPermThreads * kPermUnroll);
+}
+
+// Release-add at system scope: the stores this thread observed before it
+// (the whole CTA's, through the barrier before the call) are visible to a
+// thread of any GPU that acquires the counter value.
+__device__ __forceinline__ void red_release_sys_add(unsigned long long *p, unsigned long long v) {
+  asm volatile("red.release.sys.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__global__ void __launch_bounds__(kPermThreads)
+exchange_push_kernel(const __grid_constant__ PushParams p) {
+  const int tensor = blockIdx.z, j = blockIdx.y;
+  const uint4 *src = p.src[tensor];
+  uint4 *dst = p.dst[tensor][j] + static_cast<uint64_t>(p.rank) * p.chunk_vec;
+  const uint32_t base = blockIdx.x * (kPermThreads * kPermUnroll) + threadIdx.x;
+  uint4 v[kPermUnroll];
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    const uint32_t o = base + u * kPermThreads;
+    if (o < p.chunk_vec) {
+      const uint32_t row = fdiv(o, p.vr);
+      const uint32_t k = o - row * p.vr.d;
+      v[u] = ld_stream(src + static_cast<uint64_t>(row) * p.H_vec +
+                       static_cast<uint64_t>(j) * p.Hl_vec + k);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    const uint32_t o = base + u * kPermThreads;
+    if (o < p.chunk_vec) dst[o] = v[u];
+  }
+  __threadfence_system();
+  __syncthreads();
+  if (threadIdx.x == 0) red_release_sys_add(p.count[j] + p.rank, 1ull);
+}
+
 }  // namespace sp

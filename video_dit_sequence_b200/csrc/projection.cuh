@@ -22,6 +22,19 @@
 // accumulators so that one tile's epilogue overlaps the next tile's MMAs.
 // Tiles are ordered in groups of kProjGroupM row blocks so that CTAs working
 // at the same time share their x and w slices in L2.
+//
+// The same kernel computes the projection after attention (the output
+// projection y = o * w_o^T (+ bias), hidden features per token from the
+// H*D attention outputs).  There the layout work moves to the operand side:
+// the TMA loads of A read O where attention left it,
+//   kALoadMatrix  [P][B][Nl][H][D]  sequence shards (the fused call's output)
+//   kALoadHeads   [P][B][Np][Hl][D] head groups (sp_attention's output; the
+//                 unpack folded in: a 64-wide K slice lies inside one head
+//                 group, so it is one box of group j's rows)
+//   kALoadChunks  [P][B][Nl][Hl][D] one rank's returned chunks (the exchange
+//                 unpack folded in: K slice k lies in chunk k / (Hl*D))
+// and the epilogue stores plain rows of y [P][B][Nl][hidden] (one rank's
+// [B][Nl][hidden] for chunks).
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -32,16 +45,25 @@
 namespace sp {
 
 enum ProjLayout { kProjSeqSharded = 0, kProjHeadSharded = 1, kProjSendChunks = 2 };
+// How the A operand's K slices are addressed (see the header comment).
+enum ProjALoad { kALoadMatrix = 0, kALoadChunks = 1, kALoadHeads = 2 };
 
 struct ProjParams {
-  int32_t M, K, nout;        // rows of x, hidden size, 3*H*D
+  int32_t M, K, nout;        // rows of A, reduction size, output features
   int32_t H, D, Hl;          // heads, head dim, heads per group (H / P)
   int32_t P, B, Nl, Np;      // degree, batch, tokens per rank, P * Nl
-  int32_t layout;            // ProjLayout
-  int32_t tiles_m, tiles_n;  // ceil(M / 128), ceil(nout / 256)
+  int32_t layout;            // ProjLayout (q, k, v projection)
+  int32_t tiles_m, tiles_n;  // row blocks (all batch slots), ceil(nout / 256)
   __nv_bfloat16 *out[3];     // q, k, v
   const __nv_bfloat16 *bias; // [nout] or null
   int32_t *status;
+  // Output projection (out_proj = 1): A read through a_load, y row-major.
+  int32_t out_proj;
+  int32_t a_load;            // ProjALoad
+  int32_t a_cols;            // Hl*D: K columns of one head group / chunk
+  int32_t rows_per_slot;     // A rows of one batch slot (Np for heads, else M)
+  int32_t tiles_per_slot;    // ceil(rows_per_slot / 128)
+  __nv_bfloat16 *y;          // [rows][nout]
 };
 
 constexpr int kProjBM = 128;
@@ -53,7 +75,7 @@ constexpr int kProjABytes = kProjBM * 128;        // 16 KB
 constexpr int kProjBBytes = kProjBN * 128;        // 32 KB
 constexpr int kProjStageBytes = kProjABytes + kProjBBytes;
 constexpr int kProjOffBar = kProjStages * kProjStageBytes;
-constexpr int kProjOffMisc = kProjOffBar + (2 * kProjStages + 4) * 8;
+constexpr int kProjOffMisc = kProjOffBar + (2 * kProjStages + 5) * 8;  // ..., bar_drain
 constexpr int kProjSmemBytes = kProjOffMisc + 16 + 1024;
 constexpr int kProjThreads = 192;                 // TMA, MMA, four epilogue warps
 constexpr uint32_t kProjTmemCols = 512;               // two 256-column accumulators
@@ -76,7 +98,7 @@ __device__ __forceinline__ void proj_tile(int t, int tiles_m, int tiles_n, int &
 // across tiles, and two TMEM accumulators let the epilogue of one tile
 // overlap the MMAs of the next.
 __global__ void __launch_bounds__(kProjThreads, 1)
-qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
+projection_kernel(const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmW, const __grid_constant__ ProjParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -91,6 +113,7 @@ qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
   const uint32_t bar_empty = bar_full + 8 * kProjStages;          // [stages]
   const uint32_t bar_acc_full = bar_empty + 8 * kProjStages;      // [2]
   const uint32_t bar_acc_empty = bar_acc_full + 16;               // [2]
+  const uint32_t bar_drain = bar_acc_empty + 16;                  // the MMA thread's last commit
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + kProjOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -103,6 +126,7 @@ qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
       mbar_init(bar_acc_full + 8 * a, 1);
       mbar_init(bar_acc_empty + 8 * a, 4);      // one arrival per epilogue warp
     }
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -116,6 +140,7 @@ qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
+  int issued = 0;  // ring loads issued by the producer thread (abort-path drain)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
@@ -126,15 +151,28 @@ qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         int tm, tn;
         proj_tile(t, p.tiles_m, p.tiles_n, tm, tn);
+        // A rows of this tile: slot (batch) `slot`, rows row0 .. row0+127 of it
+        const int slot = tm / p.tiles_per_slot;
+        const int row0 = (tm - slot * p.tiles_per_slot) * kProjBM;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kProjStages;
           ok = mbar_wait(bar_empty + 8 * s, ((it / kProjStages) & 1) ^ 1u, abort_flag, kProjWaitNs);
           if (!ok) break;
           const uint32_t dst = sbase + s * kProjStageBytes;
           mbar_arrive_expect_tx(bar_full + 8 * s, kProjStageBytes);
-          tma_load_4d(dst, &tmX, bar_full + 8 * s, kb * kProjBK, tm * kProjBM, 0, 0, pol);
-          tma_load_4d(dst + kProjABytes, &tmW, bar_full + 8 * s, kb * kProjBK, tn * kProjBN, 0, 0,
-                      pol);
+          const int k0 = kb * kProjBK;
+          if (p.a_load == kALoadMatrix) {
+            tma_load_4d(dst, &tmX, bar_full + 8 * s, k0, row0, 0, 0, pol);
+          } else {
+            // a 64-wide K slice lies inside one head group (a_cols = Hl*D)
+            const int grp = k0 / p.a_cols, c0 = k0 - grp * p.a_cols;
+            if (p.a_load == kALoadChunks)
+              tma_load_4d(dst, &tmX, bar_full + 8 * s, c0, row0, grp, 0, pol);
+            else
+              tma_load_4d(dst, &tmX, bar_full + 8 * s, c0, row0, slot, grp, pol);
+          }
+          tma_load_4d(dst + kProjABytes, &tmW, bar_full + 8 * s, k0, tn * kProjBN, 0, 0, pol);
+          issued = it + 1;
         }
       }
     }
@@ -186,6 +224,53 @@ qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
         break;
       }
       tc_fence_after();
+      if (p.out_proj) {
+        // output projection: row `row` of the tile is A row row0 + row of
+        // slot `slot`; its y row is the sequence-shard row of that token
+        const int slot = tm / p.tiles_per_slot;
+        const int ar = (tm - slot * p.tiles_per_slot) * kProjBM + row;
+        int64_t yrow = -1;
+        if (ar < p.rows_per_slot) {
+          if (p.a_load == kALoadHeads) {  // token ar of batch slot `slot`
+            const int r = ar / p.Nl, nn = ar - r * p.Nl;
+            yrow = (static_cast<int64_t>(r) * p.B + slot) * p.Nl + nn;
+          } else {
+            yrow = ar;
+          }
+        }
+        const uint32_t taddr = tmem + lanes + static_cast<uint32_t>(a * kProjBN);
+        for (int c = 0; c < kProjBN; c += 32) {
+          const int f = n0 + c;
+          uint32_t accv[32];
+          __syncwarp();
+          tmem_ld32(taddr + c, accv);
+          tmem_wait_ld();
+          if (c + 32 == kProjBN) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_acc_empty + 8 * a);
+          }
+          if (f >= p.nout || yrow < 0) continue;
+          // nout is a multiple of 8: the chunk's last 16-byte vectors may lie
+          // past the end of the row and are neither computed nor stored
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float y0 = __uint_as_float(accv[2 * i]), y1 = __uint_as_float(accv[2 * i + 1]);
+            if (p.bias != nullptr && f + 2 * i < p.nout) {
+              y0 += __bfloat162float(p.bias[f + 2 * i]);
+              y1 += __bfloat162float(p.bias[f + 2 * i + 1]);
+            }
+            w[i] = pack_bf16x2(y0, y1);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(p.y + yrow * p.nout + f);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (f + 8 * i < p.nout)
+              dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+        continue;
+      }
       // row part of the destination offset, per layout (m is a token row of
       // the sequence-sharded hidden states)
       int64_t row_seq = 0, row_head = 0;
@@ -248,9 +333,17 @@ qkv_projection_kernel(const __grid_constant__ CUtensorMap tmX,
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 50000ull) {
+    // Let the asynchronous work this CTA issued land before its shared and
+    // tensor memory are released: the last kProjStages ring loads (earlier
+    // ones were consumed) and every MMA (one more commit, then its barrier).
+    if (warp == 0 && lane == 0)
+      for (int i = issued > kProjStages ? issued - kProjStages : 0; i < issued; ++i)
+        mbar_wait_drain(bar_full + 8 * (i % kProjStages), (i / kProjStages) & 1, kProjWaitNs);
+    if (warp == 1 && lane == 0) {
+      umma_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, kProjWaitNs);
     }
+    __syncthreads();
   }
   if (warp == 1) {
     tc_fence_after();

@@ -78,6 +78,46 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Waits for a barrier phase that work already issued by this CTA completes
+// (TMA copies, a tcgen05.commit), ignoring the abort flag: used on the abort
+// path to let in-flight asynchronous operations land before the CTA releases
+// its shared and tensor memory.  Returns false after limit_ns.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
+// Acquire load at system scope (a counter another GPU releases).
+__device__ __forceinline__ unsigned long long ld_acquire_sys_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *counter >= target (acquire, so that the data the counter
+// publishes is visible to this thread afterwards), or until `*abort` is set,
+// or until limit_ns passed.  Returns false when it gave up.
+__device__ __forceinline__ bool wait_counter_geq(const unsigned long long *counter,
+                                                 unsigned long long target, volatile int *abort,
+                                                 uint64_t limit_ns) {
+  if (ld_acquire_sys_u64(counter) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(256);
+    if (ld_acquire_sys_u64(counter) >= target) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Orders this thread's earlier generic-proxy accesses of global memory (the
+// acquire above) before its later async-proxy ones (TMA loads of the data).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -302,6 +302,7 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
     return SP_ERR_CUDA;
   }
   sp::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
   p.N = N;
   p.Np = Np;
   p.H = H;
@@ -348,7 +349,8 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
 // into the attention kernel (see sp_attention_ulysses_peer in sp.h).
 sp_status attention_peer(const void *const *q_shards, const void *k_group, const void *v_group,
                          void *const *o_shards, float *lse, int32_t rank, const sp_shape *s,
-                         void *stream) {
+                         void *stream, const uint64_t *counts = nullptr, uint64_t epoch = 0,
+                         uint64_t wait_ns = 0) {
   sp_status st = check_common(s, true);
   if (st != SP_OK) return st;
   if (s->D != 128) return SP_ERR_UNSUPPORTED_D;
@@ -409,6 +411,14 @@ sp_status attention_peer(const void *const *q_shards, const void *k_group, const
   p.k = static_cast<const uint8_t *>(k_group);
   p.v = static_cast<const uint8_t *>(v_group);
   p.nblk = p.num_kv_tiles;
+  if (counts != nullptr) {
+    // every source rank's chunk is counted by its push kernel's CTAs (K and V)
+    const uint32_t chunk_vec = static_cast<uint32_t>(static_cast<int64_t>(B) * Nl * Hl * D / 8);
+    p.counts = reinterpret_cast<const unsigned long long *>(counts);
+    p.count_target = epoch * 2ull * sp::push_blocks_per_chunk(chunk_vec);
+    p.count_nl = Nl;
+    p.count_wait_ns = wait_ns > 0 ? wait_ns : sp::kWaitLimitNs;
+  }
   using C = sp::AttnCfg<128>;
   static bool attr_set[kMaxDevices] = {};
   cudaError_t e = set_smem_once(sp::attention_peer_kernel, C::kSmemBytes, attr_set);
@@ -416,6 +426,45 @@ sp_status attention_peer(const void *const *q_shards, const void *k_group, const
   dim3 grid((Np + 2 * C::kBM - 1) / (2 * C::kBM), Hl, B);
   sp::attention_peer_kernel<<<grid, C::kThreads, C::kSmemBytes,
                               static_cast<cudaStream_t>(stream)>>>(pa, mk, mv, p);
+  return launch_status(cudaGetLastError());
+}
+
+// One rank's K/V exchange over peer memory (see sp_exchange_push in sp.h).
+sp_status exchange_push(const void *k_r, const void *v_r, void *const *k_groups,
+                        void *const *v_groups, uint64_t *const *counts, uint64_t epoch,
+                        int32_t rank, const sp_shape *s, void *stream) {
+  sp_status st = check_common(s, true);
+  if (st != SP_OK) return st;
+  if (s->P > sp::kMaxPushPeers || rank < 0 || rank >= s->P) return SP_ERR_SHAPE;
+  if (epoch < 1) return SP_ERR_SHAPE;
+  if (k_r == nullptr || v_r == nullptr || k_groups == nullptr || v_groups == nullptr ||
+      counts == nullptr)
+    return SP_ERR_NULL;
+  if (!aligned16(k_r) || !aligned16(v_r)) return SP_ERR_ALIGN;
+  const int P = s->P, B = s->B, H = s->H, D = s->D;
+  const int Hl = H / P;
+  const int Nl = (s->N + P - 1) / P;
+  sp::PushParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.src[0] = static_cast<const uint4 *>(k_r);
+  p.src[1] = static_cast<const uint4 *>(v_r);
+  for (int j = 0; j < P; ++j) {
+    if (k_groups[j] == nullptr || v_groups[j] == nullptr || counts[j] == nullptr)
+      return SP_ERR_NULL;
+    if (!aligned16(k_groups[j]) || !aligned16(v_groups[j]) ||
+        (reinterpret_cast<uintptr_t>(counts[j]) & 7u) != 0)
+      return SP_ERR_ALIGN;
+    p.dst[0][j] = static_cast<uint4 *>(k_groups[j]);
+    p.dst[1][j] = static_cast<uint4 *>(v_groups[j]);
+    p.count[j] = reinterpret_cast<unsigned long long *>(counts[j]);
+  }
+  p.chunk_vec = static_cast<uint32_t>(static_cast<int64_t>(B) * Nl * Hl * D / 8);
+  p.vr = sp::make_fastdiv(Hl * D / 8);
+  p.H_vec = H * D / 8;
+  p.Hl_vec = Hl * D / 8;
+  p.rank = static_cast<uint32_t>(rank);
+  dim3 grid(sp::push_blocks_per_chunk(p.chunk_vec), P, 2);
+  sp::exchange_push_kernel<<<grid, sp::kPermThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
   return launch_status(cudaGetLastError());
 }
 
@@ -435,6 +484,9 @@ bool make_map_matrix(CUtensorMap *m, const void *base, int cols, int rows, int b
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+sp_status launch_projection(const CUtensorMap &mx, const CUtensorMap &mw, const sp::ProjParams &p,
+                            void *stream);
 
 sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q, void *k,
                          void *v, int32_t hidden, int32_t layout, const sp_shape *s,
@@ -481,8 +533,107 @@ sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q
   p.out[2] = static_cast<__nv_bfloat16 *>(v);
   p.bias = static_cast<const __nv_bfloat16 *>(bias);
   p.status = status;
+  p.a_load = sp::kALoadMatrix;
+  p.rows_per_slot = p.M;
+  p.tiles_per_slot = p.tiles_m;
+  return launch_projection(mx, mw, p, stream);
+}
+
+// Tensor map over a bf16 operand viewed as 4-D [d3][d2][d1 rows][d0 cols]
+// (cols contiguous; strides in elements), boxes of 64 columns x box_rows rows
+// under the 128-byte swizzle.  Coordinates past an extent read as zeros.
+bool make_map_rows4(CUtensorMap *m, const void *base, int64_t d0, int64_t d1, int64_t d2,
+                    int64_t d3, int64_t s1, int64_t s2, int64_t s3, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
+                        static_cast<cuuint64_t>(d2), static_cast<cuuint64_t>(d3)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s1) * 2, static_cast<cuuint64_t>(s2) * 2,
+                           static_cast<cuuint64_t>(s3) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The projection after attention (see sp_out_projection in sp.h): the GEMM
+// of the q, k, v projection with A = O read through a tensor map over the
+// layout attention left it in, and y stored as plain sequence-shard rows.
+sp_status out_projection(const void *o, const void *w, const void *bias, void *y,
+                         int32_t hidden, int32_t layout, const sp_shape *s, void *stream) {
+  if (layout < SP_O_SEQ_SHARDED || layout > SP_O_RECV_CHUNKS) return SP_ERR_SHAPE;
+  sp_status st = check_common(s, layout != SP_O_SEQ_SHARDED);
+  if (st != SP_OK) return st;
+  if (o == nullptr || w == nullptr || y == nullptr) return SP_ERR_NULL;
+  if (hidden < 8 || hidden % 8 != 0) return SP_ERR_SHAPE;
+  if (!aligned16(o) || !aligned16(w) || !aligned16(y) ||
+      (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 1u) != 0))
+    return SP_ERR_ALIGN;
+  const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
+  const int Nl = (N + P - 1) / P, Np = Nl * P;
+  const int Hl = H / P;
+  const int64_t K = static_cast<int64_t>(H) * D;
+  const int64_t rows = static_cast<int64_t>(layout == SP_O_RECV_CHUNKS ? 1 : P) * B * Nl;
+  if (rows >= (int64_t(1) << 31) || rows * hidden >= (int64_t(1) << 40) ||
+      static_cast<int64_t>(hidden) * K >= (int64_t(1) << 40))
+    return SP_ERR_SHAPE;
+  int32_t *status = status_ptr();
+  if (status == nullptr) return SP_ERR_CUDA;
+  CUtensorMap ma, mw;
+  sp::ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int64_t gcols = static_cast<int64_t>(Hl) * D;
+  bool ok_a;
+  if (layout == SP_O_SEQ_SHARDED) {
+    // [P][B][Nl][H][D] = rows x (H*D), row-major
+    ok_a = make_map_rows4(&ma, o, K, rows, 1, 1, K, K * rows, K * rows, sp::kProjBM);
+    p.a_load = sp::kALoadMatrix;
+    p.rows_per_slot = static_cast<int32_t>(rows);
+    p.tiles_per_slot = static_cast<int32_t>((rows + sp::kProjBM - 1) / sp::kProjBM);
+    p.tiles_m = p.tiles_per_slot;
+  } else if (layout == SP_O_HEAD_SHARDED) {
+    // [P (group)][B][Np][Hl*D]: one slot per batch, rows = tokens of the slot
+    ok_a = make_map_rows4(&ma, o, gcols, Np, B, P, gcols, gcols * Np, gcols * Np * B, sp::kProjBM);
+    p.a_load = sp::kALoadHeads;
+    p.rows_per_slot = Np;
+    p.tiles_per_slot = (Np + sp::kProjBM - 1) / sp::kProjBM;
+    p.tiles_m = p.tiles_per_slot * B;
+  } else {
+    // one rank's [P (chunk)][B*Nl][Hl*D]
+    ok_a = make_map_rows4(&ma, o, gcols, rows, P, 1, gcols, gcols * rows, gcols * rows * P,
+                          sp::kProjBM);
+    p.a_load = sp::kALoadChunks;
+    p.rows_per_slot = static_cast<int32_t>(rows);
+    p.tiles_per_slot = static_cast<int32_t>((rows + sp::kProjBM - 1) / sp::kProjBM);
+    p.tiles_m = p.tiles_per_slot;
+  }
+  if (!ok_a || !make_map_matrix(&mw, w, static_cast<int>(K), hidden, sp::kProjBN))
+    return SP_ERR_CUDA;
+  p.M = static_cast<int32_t>(rows);
+  p.K = static_cast<int32_t>(K);
+  p.nout = hidden;
+  p.H = H;
+  p.D = D;
+  p.Hl = Hl;
+  p.P = P;
+  p.B = B;
+  p.Nl = Nl;
+  p.Np = Np;
+  p.a_cols = static_cast<int32_t>(gcols);
+  p.tiles_n = (hidden + sp::kProjBN - 1) / sp::kProjBN;
+  p.out_proj = 1;
+  p.y = static_cast<__nv_bfloat16 *>(y);
+  p.bias = static_cast<const __nv_bfloat16 *>(bias);
+  p.status = status;
+  return launch_projection(ma, mw, p, stream);
+}
+
+sp_status launch_projection(const CUtensorMap &mx, const CUtensorMap &mw, const sp::ProjParams &p,
+                            void *stream) {
   static bool attr_set[kMaxDevices] = {};
-  cudaError_t e = set_smem_once(sp::qkv_projection_kernel, sp::kProjSmemBytes, attr_set);
+  cudaError_t e = set_smem_once(sp::projection_kernel, sp::kProjSmemBytes, attr_set);
   if (e != cudaSuccess) return SP_ERR_CUDA;
   const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
   if (tiles >= (int64_t(1) << 31)) return SP_ERR_SHAPE;
@@ -492,7 +643,7 @@ sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return SP_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  sp::qkv_projection_kernel<<<grid, sp::kProjThreads, sp::kProjSmemBytes,
+  sp::projection_kernel<<<grid, sp::kProjThreads, sp::kProjSmemBytes,
                               static_cast<cudaStream_t>(stream)>>>(mx, mw, p);
   return launch_status(cudaGetLastError());
 }
@@ -513,20 +664,59 @@ AddressRangeFn address_range_fn() {
   return fn;
 }
 
-__global__ void wait_timeout_kernel(uint64_t limit_ns, int32_t *status) {
-  __shared__ __align__(8) uint64_t bar;
+// Source of the self-test's bulk copy (contents irrelevant).
+__device__ __align__(128) uint8_t g_selftest_src[4096];
+
+// The abort path of the kernels in miniature, on one warp: asynchronous work
+// is in flight (a bulk copy into shared memory and one tcgen05 MMA into a
+// TMEM accumulator) when a wait on a barrier that nothing completes runs out;
+// the thread then drains what it issued (the copy's barrier, one more commit
+// after the MMA) before the TMEM is released, and records SP_ERR_TIMEOUT.  A
+// drain that did not finish, or a wait that did not run out, records a
+// different code, so the caller sees it.
+__global__ void __launch_bounds__(32, 1) wait_timeout_kernel(uint64_t limit_ns, int32_t *status) {
+  __shared__ __align__(1024) uint8_t tiles[2 * 16384];  // A and B of one 128x128x16 MMA
+  __shared__ __align__(128) uint8_t copy_dst[sizeof(g_selftest_src)];
+  __shared__ __align__(8) uint64_t bars[3];              // never completed, copy, drain
+  __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  const uint32_t never = sp::smem_u32(&bars[0]), copied = never + 8, drained = never + 16;
   if (threadIdx.x == 0) {
-    sp::mbar_init(sp::smem_u32(&bar), 1);
+    sp::mbar_init(never, 1);
+    sp::mbar_init(copied, 1);
+    sp::mbar_init(drained, 1);
     abort_flag = 0;
     sp::fence_mbar_init();
   }
-  __syncthreads();
+  __syncwarp();
+  sp::tmem_alloc(sp::smem_u32(&tmem_slot), 128);
+  sp::tmem_relinquish();
+  sp::tc_fence_before();
+  __syncwarp();
+  sp::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
   if (threadIdx.x == 0) {
-    // Nothing ever arrives on `bar`: the wait must give up after limit_ns.
-    if (!sp::mbar_wait(sp::smem_u32(&bar), 0, &abort_flag, limit_ns))
-      atomicExch(status, sp::kStatusTimeout);
+    sp::mbar_arrive_expect_tx(copied, sizeof(g_selftest_src));
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(sp::smem_u32(copy_dst)), "l"(reinterpret_cast<uint64_t>(g_selftest_src)),
+          "r"(static_cast<uint32_t>(sizeof(g_selftest_src))), "r"(copied)
+        : "memory");
+    const uint32_t a = sp::smem_u32(tiles);
+    sp::umma_ss<false>(tmem, sp::make_sdesc_sw128(a, 16, 1024),
+                       sp::make_sdesc_sw128(a + 16384, 16, 1024),
+                       sp::make_idesc_bf16(128, 128, 0, 0), 0u);
+    // Nothing ever arrives on `never`: the wait must give up after limit_ns.
+    const bool timed_out = !sp::mbar_wait(never, 0, &abort_flag, limit_ns);
+    bool ok = sp::mbar_wait_drain(copied, 0, sp::kWaitLimitNs);
+    sp::umma_commit(drained);
+    ok = sp::mbar_wait_drain(drained, 0, sp::kWaitLimitNs) && ok;
+    atomicExch(status, timed_out && ok ? sp::kStatusTimeout : sp::kStatusTimeout - 1);
   }
+  sp::tc_fence_before();
+  __syncwarp();
+  sp::tc_fence_after();
+  sp::tmem_dealloc(tmem, 128);
 }
 
 }  // namespace
@@ -605,11 +795,36 @@ sp_status sp_qkv_projection(const void *x, const void *w, const void *bias, void
   return qkv_projection(x, w, bias, q, k, v, hidden, layout, shape, stream);
 }
 
+sp_status sp_out_projection(const void *o, const void *w, const void *bias, void *y,
+                            int32_t hidden, int32_t layout, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_out_projection");
+  return out_projection(o, w, bias, y, hidden, layout, shape, stream);
+}
+
 sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_group,
                                     const void *v_group, void *const *o_shards, float *lse,
                                     int32_t rank, const sp_shape *shape, void *stream) {
   NvtxRange range("sp_attention_ulysses_peer");
   return attention_peer(q_shards, k_group, v_group, o_shards, lse, rank, shape, stream);
+}
+
+sp_status sp_exchange_push(const void *k_r, const void *v_r, void *const *k_groups,
+                           void *const *v_groups, uint64_t *const *counts, uint64_t epoch,
+                           int32_t rank, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_exchange_push");
+  return exchange_push(k_r, v_r, k_groups, v_groups, counts, epoch, rank, shape, stream);
+}
+
+sp_status sp_attention_ulysses_overlap(const void *const *q_shards, const void *k_group,
+                                       const void *v_group, void *const *o_shards, float *lse,
+                                       const uint64_t *counts, uint64_t epoch, uint64_t wait_ns,
+                                       int32_t rank, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_attention_ulysses_overlap");
+  if (counts == nullptr) return SP_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(counts) & 7u) != 0) return SP_ERR_ALIGN;
+  if (epoch < 1) return SP_ERR_SHAPE;
+  return attention_peer(q_shards, k_group, v_group, o_shards, lse, rank, shape, stream, counts,
+                        epoch, wait_ns);
 }
 
 sp_status sp_ipc_export(const void *dev_ptr, void *handle_out, int64_t *offset_out) {
