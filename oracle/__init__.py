@@ -63,7 +63,7 @@ def _bind(path: str):
     i64 = ctypes.c_int64
     vp = ctypes.c_void_p
     for name in ("sp_oracle_pack", "sp_oracle_unpack", "sp_oracle_exchange_pack",
-                 "sp_oracle_exchange_unpack"):
+                 "sp_oracle_exchange_unpack", "sp_oracle_shard", "sp_oracle_unshard"):
         f = getattr(lib, name)
         f.argtypes = [vp, vp, i64, i64, i64, i64, i64]
         f.restype = ctypes.c_int
@@ -136,6 +136,30 @@ def unpack(oh: np.ndarray, N: int, H: int, lib=None) -> np.ndarray:
     oh = np.ascontiguousarray(oh)
     out = np.empty((P, B, Nl, H, D), dtype=np.uint16)
     rc = (lib or _load()).sp_oracle_unpack(oh.ctypes.data, out.ctypes.data, B, N, H, D, P)
+    assert rc == 0
+    return out
+
+
+def shard(x: np.ndarray, P: int, lib=None) -> np.ndarray:
+    """Logical [B][N][H][D] -> P token shards [P][B][Nl][H][D], padding zero."""
+    assert x.dtype == np.uint16 and x.ndim == 4
+    B, N, H, D = x.shape
+    Nl = _dims(N, P)[0]
+    x = np.ascontiguousarray(x)
+    out = np.empty((P, B, Nl, H, D), dtype=np.uint16)
+    rc = (lib or _load()).sp_oracle_shard(x.ctypes.data, out.ctypes.data, B, N, H, D, P)
+    assert rc == 0
+    return out
+
+
+def unshard(xs: np.ndarray, N: int, lib=None) -> np.ndarray:
+    """P token shards [P][B][Nl][H][D] -> logical [B][N][H][D]."""
+    assert xs.dtype == np.uint16 and xs.ndim == 5
+    P, B, Nl, H, D = xs.shape
+    assert Nl == _dims(N, P)[0]
+    xs = np.ascontiguousarray(xs)
+    out = np.empty((B, N, H, D), dtype=np.uint16)
+    rc = (lib or _load()).sp_oracle_unshard(xs.ctypes.data, out.ctypes.data, B, N, H, D, P)
     assert rc == 0
     return out
 

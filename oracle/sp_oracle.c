@@ -125,6 +125,46 @@ int sp_oracle_unpack(const uint16_t *oh, uint16_t *os, int64_t B, int64_t N,
 }
 
 /*
+ * Shard: the token sequence of one generation divided across the P ranks
+ * (same page section), rank r holding tokens r*Nl .. r*Nl+Nl-1 of the
+ * logical [B][N][H][D] tensor; slots past the last token are zero:
+ *     xs[r][b][n][h][c] = x[b][r*Nl + n][h][c]   if r*Nl + n < N, else 0
+ */
+int sp_oracle_shard(const uint16_t *x, uint16_t *xs, int64_t B, int64_t N,
+                    int64_t H, int64_t D, int64_t P) {
+    if (P < 1) return -1;
+    int64_t Nl = (N + P - 1) / P;
+    for (int64_t r = 0; r < P; ++r)
+        for (int64_t b = 0; b < B; ++b)
+            for (int64_t n = 0; n < Nl; ++n)
+                for (int64_t h = 0; h < H; ++h)
+                    for (int64_t c = 0; c < D; ++c) {
+                        int64_t t = r * Nl + n;
+                        int64_t dst = (((r * B + b) * Nl + n) * H + h) * D + c;
+                        xs[dst] = t < N ? x[((b * N + t) * H + h) * D + c] : 0;
+                    }
+    return 0;
+}
+
+/*
+ * Unshard: the P shards back to the logical tensor, padding slots dropped:
+ *     x[b][t][h][c] = xs[t / Nl][b][t % Nl][h][c]
+ */
+int sp_oracle_unshard(const uint16_t *xs, uint16_t *x, int64_t B, int64_t N,
+                      int64_t H, int64_t D, int64_t P) {
+    if (P < 1) return -1;
+    int64_t Nl = (N + P - 1) / P;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t t = 0; t < N; ++t)
+            for (int64_t h = 0; h < H; ++h)
+                for (int64_t c = 0; c < D; ++c) {
+                    int64_t r = t / Nl, n = t % Nl;
+                    x[((b * N + t) * H + h) * D + c] = xs[(((r * B + b) * Nl + n) * H + h) * D + c];
+                }
+    return 0;
+}
+
+/*
  * Exchange pack on one rank (the send-buffer reorder in front of the
  * all-to-all of "Splitting one generation across four GPUs" when every rank
  * is its own GPU): rank r's shard xs_r [B][Nl][H][D] becomes P send chunks,

@@ -447,10 +447,46 @@ def check_linear_projection(lib=None):
             assert np.max(np.abs(got - want)) < 1e-12 * max(1.0, np.max(np.abs(want)))
 
 
+def check_shard_splits_the_sequence(lib=None):
+    """Rank r holds tokens r*Nl .. r*Nl+Nl-1 of the logical tensor (the page's
+    division of the token sequence, written as numpy slicing); the slots past
+    the last token are zero."""
+    rng = np.random.default_rng(RNG_SEED + 40)
+    for (B, N, H, D, P) in PACK_SHAPES + [(2, 3, 2, 8, 8)]:
+        X = _codes((B, N, H, D), rng)
+        X[X == 0] = 1
+        xs = oracle.shard(X, P, lib=lib)
+        Nl = -(-N // P)
+        assert xs.shape == (P, B, Nl, H, D)
+        for r in range(P):
+            lo, hi = min(r * Nl, N), min(r * Nl + Nl, N)
+            assert np.array_equal(xs[r][:, :hi - lo], X[:, lo:hi]), (B, N, H, D, P, r)
+            assert not xs[r][:, hi - lo:].any()
+
+
+def check_shard_matches_numpy_and_inverts(lib=None):
+    """Library formulation: zero-pad the sequence to P*Nl and move
+    [B][P][Nl] to [P][B][Nl] with numpy; unshard inverts shard and, on shards
+    with junk in the padding slots, equals numpy's inverse reshape."""
+    rng = np.random.default_rng(RNG_SEED + 41)
+    for (B, N, H, D, P) in PACK_SHAPES + [(2, 3, 2, 8, 8)]:
+        X = _codes((B, N, H, D), rng)
+        Nl = -(-N // P)
+        pad = np.zeros((B, P * Nl, H, D), dtype=np.uint16)
+        pad[:, :N] = X
+        ref = pad.reshape(B, P, Nl, H, D).transpose(1, 0, 2, 3, 4)
+        assert np.array_equal(oracle.shard(X, P, lib=lib), ref)
+        assert np.array_equal(oracle.unshard(oracle.shard(X, P, lib=lib), N, lib=lib), X)
+        xs = _codes((P, B, Nl, H, D), rng)
+        want = xs.transpose(1, 0, 2, 3, 4).reshape(B, P * Nl, H, D)[:, :N]
+        assert np.array_equal(oracle.unshard(xs, N, lib=lib), want)
+
+
 PACK_CHECKS = [check_pack_heads_for_full_sequence, check_pack_matches_numpy_transpose,
                check_unpack_returns_shards, check_pack_degree_one_is_copy,
                check_exchange_chunks_hold_head_groups,
-               check_exchange_matches_numpy_and_single_gpu_pack]
+               check_exchange_matches_numpy_and_single_gpu_pack,
+               check_shard_splits_the_sequence, check_shard_matches_numpy_and_inverts]
 ATTENTION_CHECKS = [check_attention_matches_numpy, check_softmax_rows_sum_to_one,
                     check_closed_forms, check_dominant_key, check_invariances,
                     check_two_token_example, check_rows_api,

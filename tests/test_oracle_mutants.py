@@ -24,6 +24,11 @@ MUTANTS = [
     ("exchange-unpack-wrong-chunk",
      "recv[(((j * B + b) * Nl + n) * Hl + hh) * D + c];",
      "recv[((((P - 1 - j) * B + b) * Nl + n) * Hl + hh) * D + c];"),
+    ("shard-interleaves-tokens", "int64_t t = r * Nl + n;", "int64_t t = n * P + r;"),
+    ("shard-pads-with-last-token",
+     "xs[dst] = t < N ? x[((b * N + t) * H + h) * D + c] : 0;",
+     "xs[dst] = x[((b * N + (t < N ? t : N - 1)) * H + h) * D + c];"),
+    ("unshard-wrong-rank", "int64_t r = t / Nl, n = t % Nl;", "int64_t r = t % P, n = t / P;"),
     ("scale-dropped", "s[kk] = J->scale * dot;", "s[kk] = dot;"),
     ("lse-sign", "m + log(l)", "m - log(l)"),
     ("no-normalisation", "o[c] /= l;", "o[c] /= 1.0;"),
