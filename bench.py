@@ -482,7 +482,13 @@ def run_ours(args):
         t_sparse = timed(lambda: sp.attention_sparse_seqsharded(qs, ks, vs, words, o_sp, shape,
                                                                 stream=stream))
         sparse_flops = 4.0 * synth.attended_pairs(mask, s.N) * s.D
-        del words, o_sp
+        # the same density with an independent selection per query cube
+        mask_ind = synth.cube_mask(cfg, density=0.2, group=1)
+        words_ind = torch.from_numpy(sp.sparse_mask_words(mask_ind).view(np.int32)).to(dev)
+        t_sparse_ind = timed(lambda: sp.attention_sparse_seqsharded(qs, ks, vs, words_ind, o_sp,
+                                                                    shape, stream=stream))
+        sparse_ind_flops = 4.0 * synth.attended_pairs(mask_ind, s.N) * s.D
+        del words, words_ind, o_sp
     # the projection in front of attention (hidden -> q, k, v) with its
     # epilogue writing the sequence-sharded layout; cuBLAS on the same GEMM
     # (x @ w^T, one contiguous output) timed beside it
@@ -532,7 +538,11 @@ def run_ours(args):
         "sparse": None if t_sparse is None else {
             "ms": t_sparse, "speedup_vs_dense": per_launch_ms / t_sparse,
             "attended_TFLOP/s": sparse_flops / (t_sparse * 1e-3) / 1e12,
-            "mask": "64-token cubes, density 0.2, one selection per 4 query cubes (synthetic)"},
+            "mask": "64-token cubes, density 0.2, one selection per 4 query cubes (synthetic)",
+            "independent": {
+                "ms": t_sparse_ind, "speedup_vs_dense": per_launch_ms / t_sparse_ind,
+                "attended_TFLOP/s": sparse_ind_flops / (t_sparse_ind * 1e-3) / 1e12,
+                "mask": "64-token cubes, density 0.2, an independent selection per query cube"}},
         "qkv_projection": None if t_proj is None else {
             "ms": t_proj, "TFLOP/s": proj_flops / (t_proj * 1e-3) / 1e12,
             "frac": proj_flops / (t_proj * 1e-3) / 1e12 / pk["bf16_tflops"],

@@ -74,6 +74,20 @@ int64_t sp_padded_tokens(int32_t N, int32_t P);
  * gives SP_ERR_HEADS_NOT_DIVISIBLE. */
 sp_status sp_check_shape(const sp_shape *shape);
 
+/* Shard: the logical sequence of one generation divided across the P ranks
+ * (page section "Splitting one generation across four GPUs"), rank r
+ * holding tokens r*Nl .. r*Nl+Nl-1; token slots at or past N are zero:
+ *   xs[r][b][n][h][c] = x[b][r*Nl + n][h][c]   (r*Nl + n < N), else +0.0
+ * x: device [B][N][H][D] bf16, read only.  xs: device [P][B][Nl][H][D],
+ * written in full.  Bit-exact copy.  Any P >= 1 (no heads are split). */
+sp_status sp_shard(const void *x, void *xs, const sp_shape *shape, void *stream);
+
+/* Unshard: the inverse of sp_shard, padding slots dropped:
+ *   x[b][t][h][c] = xs[t / Nl][b][t % Nl][h][c]
+ * xs: device [P][B][Nl][H][D] bf16, read only.  x: device [B][N][H][D],
+ * written in full.  Bit-exact copy. */
+sp_status sp_unshard(const void *xs, void *x, const sp_shape *shape, void *stream);
+
 /* Pack: sequence-sharded -> head-sharded, the send reorder plus all-to-all
  * of the page section "Splitting one generation across four GPUs":
  *   xh[j][b][r*Nl + n][hh][c] = xs[r][b][n][j*Hl + hh][c]
@@ -248,11 +262,11 @@ sp_status sp_out_projection(const void *o, const void *w, const void *bias, void
  *   key cube 32*w + c; bits for cubes >= ncube are ignored.  Read only,
  *   4-byte aligned.
  * qs, ks, vs, os, lse as for sp_attention_seqsharded; D must be 128 and
- * ceil(N / 128) <= 16384 (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  The kernel
- * visits, for each pair of 128-row query tiles, only the 128-key tiles that
- * one of their four query cubes selects.  With every cube selected the
- * result equals sp_attention_seqsharded's bit for bit; results do not depend
- * on P. */
+ * ceil(N / 64) <= 16384 (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  The kernel
+ * visits, for each pair of 128-row query tiles, only the key cubes that one
+ * of their four query cubes selects, two cubes per 128-key tile in
+ * increasing order.  With every cube selected the result equals
+ * sp_attention_seqsharded's bit for bit; results do not depend on P. */
 sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const void *vs,
                                          const uint32_t *mask, void *os, float *lse,
                                          const sp_shape *shape, void *stream);

@@ -206,6 +206,10 @@ def test_argument_errors_return_before_launch(lib):
     assert lib.sp_ipc_open(None, ctypes.byref(base)) == sp.SP_ERR_NULL
     assert lib.sp_ipc_open(h, None) == sp.SP_ERR_NULL
     assert lib.sp_ipc_close(None) == sp.SP_ERR_NULL
+    for fn in (lib.sp_shard, lib.sp_unshard):
+        assert _call(fn, 0, B_, shape=shape) == sp.SP_ERR_NULL
+        assert _call(fn, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN
+        assert _call(fn, A, B_, shape=sp.Shape(1, 1024, 4, 80, 2)) == sp.SP_ERR_UNSUPPORTED_D
     for fn in (lib.sp_exchange_pack, lib.sp_exchange_unpack):
         assert _call(fn, 0, B_, shape=shape) == sp.SP_ERR_NULL
         assert _call(fn, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN

@@ -160,6 +160,46 @@ def test_pack_sweep_bit_exact(N):
         _perm_full_size(q, N, base.shape.H, P, f"sweep N={N} P={P}")
 
 
+SHARD_SHAPES = [(1, 1024, 4, 64, 2), (3, 1001, 6, 128, 4), (2, 77, 5, 64, 3), (1, 3, 2, 128, 8),
+                (4, 130, 2, 64, 1), (1, 75601, 40, 128, 8)]
+
+
+@pytest.mark.parametrize("B,N,H,D,P", SHARD_SHAPES)
+def test_shard_unshard_bit_exact(B, N, H, D, P):
+    """The logical sequence into P zero-padded token shards and back, bit for
+    bit against the oracle (ragged N, B > 1, P not dividing H, the ragged
+    75,601-token sweep shape); unshard of shards with junk in the padding."""
+    shape = sp.Shape(B, N, H, D, P)
+    X = synth.normal_bf16(500 + N, 0, 0, B * N * H * D).reshape(B, N, H, D)
+    d_xs = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.shard(to_dev(X), d_xs, shape)
+    assert np.array_equal(to_host(d_xs).reshape(shape.seq_sharded), oracle.shard(X, P))
+    xs = synth.normal_bf16(600 + N, 1, 0, int(np.prod(shape.seq_sharded))).reshape(shape.seq_sharded)
+    d_x = torch.full((B, N, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sp.unshard(to_dev(xs), d_x, shape)
+    assert np.array_equal(to_host(d_x).reshape(B, N, H, D), oracle.unshard(xs, N))
+    _status_ok()
+
+
+@pytest.mark.parametrize("B,N,H,P,fused", [(3, 1001, 6, 4, True), (2, 777, 8, 4, False),
+                                           (1, 513, 4, 3, True)])
+def test_user_level_call(B, N, H, P, fused):
+    """ulysses_attention on logical [B, N, H, D] tensors (ragged N, B > 1):
+    the library shards, attends and unshards; the result equals the fused
+    call on the oracle's shards bit for bit and the oracle within the bars."""
+    D = 128
+    q, k, v = _random_logical(B, N, H, D, seed=19 * N + P)
+    out = sp.ulysses_attention(to_dev(q), to_dev(k), to_dev(v), P, fused=fused)
+    _status_ok()
+    got = to_host(out).reshape(B, N, H, D)
+    one, _ = _run_fused(q, k, v, P)
+    assert np.array_equal(got, oracle.unshard(one.reshape(P, B, -1, H, D), N))
+    rows = _rows_all(B, N, H)[::7]
+    ref, _ = oracle.attention_rows(q, k, v, rows)
+    assert_parity(compare(got[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]),
+                  f"user call B={B} N={N} P={P}")
+
+
 EXCHANGE_SHAPES = [(1, 1024, 4, 64, 2), (2, 1000, 8, 128, 4), (3, 77, 6, 128, 3),
                    (1, 4096, 40, 128, 8), (2, 9, 8, 128, 8)]
 

@@ -44,7 +44,7 @@ EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded",
             "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close",
             "sp_attention_sparse_seqsharded", "sp_qkv_projection", "sp_out_projection",
-            "sp_exchange_push", "sp_attention_ulysses_overlap")
+            "sp_exchange_push", "sp_attention_ulysses_overlap", "sp_shard", "sp_unshard")
 
 
 class sp_shape(ctypes.Structure):
@@ -75,7 +75,8 @@ def load(path: str = LIB_PATH):
     lib.sp_padded_tokens.restype = ctypes.c_int64
     lib.sp_check_shape.argtypes = [sp_p]
     lib.sp_check_shape.restype = ctypes.c_int
-    for name in ("sp_pack", "sp_unpack", "sp_exchange_pack", "sp_exchange_unpack"):
+    for name in ("sp_pack", "sp_unpack", "sp_exchange_pack", "sp_exchange_unpack", "sp_shard",
+                 "sp_unshard"):
         f = getattr(lib, name)
         f.argtypes = [vp, vp, sp_p, vp]
         f.restype = ctypes.c_int
@@ -255,6 +256,25 @@ def _same_device(*tensors):
 def _check(status: int, where: str):
     if status != SP_OK:
         raise SpError(status, where)
+
+
+def shard(x, xs, shape: Shape, stream=None):
+    """Logical [B][N][H][D] -> P token shards [P][B][Nl][H][D], padding slots
+    zero (bit-exact)."""
+    s = shape.c()
+    with _same_device(x, xs):
+        _check(load().sp_shard(_ptr(x, (shape.B, shape.N, shape.H, shape.D), "x"),
+                               _ptr(xs, shape.seq_sharded, "xs"), ctypes.byref(s),
+                               _stream(stream, x.device)), "sp_shard")
+
+
+def unshard(xs, x, shape: Shape, stream=None):
+    """P token shards [P][B][Nl][H][D] -> logical [B][N][H][D] (bit-exact)."""
+    s = shape.c()
+    with _same_device(xs, x):
+        _check(load().sp_unshard(_ptr(xs, shape.seq_sharded, "xs"),
+                                 _ptr(x, (shape.B, shape.N, shape.H, shape.D), "x"),
+                                 ctypes.byref(s), _stream(stream, xs.device)), "sp_unshard")
 
 
 def pack(xs, xh, shape: Shape, stream=None):
@@ -883,19 +903,19 @@ def selftest_wait_timeout(limit_ns: int, stream=None, device=None):
 
 def ulysses_attention(q, k, v, P: int, scale: float = 0.0, fused: bool = True):
     """User-level call: q, k, v are [B, N, H, D] bf16 CUDA tensors (logical,
-    unsharded); returns O [B, N, H, D].  The tensors are laid out as P
-    sequence shards (zero-padded to Np tokens), attended with P virtual ranks
-    and read back.  fused=False runs pack -> attention -> unpack instead of
-    the fused kernel."""
+    unsharded, contiguous); returns O [B, N, H, D].  The tensors are laid out
+    as P sequence shards (sp_shard, zero-padded to Np tokens), attended with
+    P virtual ranks and read back (sp_unshard).  fused=False runs pack ->
+    attention -> unpack instead of the fused kernel."""
     torch = _torch()
     B, N, H, D = q.shape
     shape = Shape(B, N, H, D, P, scale)
-    Nl, Np = shape.Nl, shape.Np
+    ss = shape.seq_sharded
 
     def shards(x):
-        buf = torch.zeros((B, Np, H, D), dtype=x.dtype, device=x.device)
-        buf[:, :N] = x
-        return buf.view(B, P, Nl, H, D).transpose(0, 1).contiguous()
+        xs = torch.empty(ss, dtype=x.dtype, device=x.device)
+        shard(x, xs, shape)
+        return xs
 
     qs, ks, vs = shards(q), shards(k), shards(v)
     os_ = torch.empty_like(qs)
@@ -909,4 +929,6 @@ def ulysses_attention(q, k, v, P: int, scale: float = 0.0, fused: bool = True):
         pack(vs, vh, shape)
         attention(qh, kh, vh, oh, shape)
         unpack(oh, os_, shape)
-    return os_.transpose(0, 1).reshape(B, Np, H, D)[:, :N]
+    out = torch.empty_like(q)
+    unshard(os_, out, shape)
+    return out

@@ -131,9 +131,9 @@ struct AttnCfg {
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   static constexpr int kNumBar = 1 + 2 * kStages + 9;  // ..., bar_o[2], bar_drain
   static constexpr int kOffMisc = kOffBar + kNumBar * 8;
-  // Block-sparse variant: one bit per key tile, set when any query cube of
-  // the CTA selects either key cube of the tile.
-  static constexpr int kMaxSelWords = 512;                  // 16,384 key tiles
+  // Block-sparse variant: one bit per 64-token key cube, set when any query
+  // cube of the CTA selects it.
+  static constexpr int kMaxSelWords = 512;                  // 16,384 key cubes
   static constexpr int kOffSel = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffSel + 4 * kMaxSelWords + 1024;  // + alignment slack
   static constexpr int kThreads = 320;
@@ -145,15 +145,6 @@ struct AttnCfg {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
-
-// Bit i (i < 16) of the result: bit 2i or bit 2i+1 of x.
-__device__ __forceinline__ uint32_t pair_bits(uint32_t x) {
-  x = (x | (x >> 1)) & 0x55555555u;
-  x = (x | (x >> 1)) & 0x33333333u;
-  x = (x | (x >> 2)) & 0x0F0F0F0Fu;
-  x = (x | (x >> 4)) & 0x00FF00FFu;
-  return (x | (x >> 8)) & 0x0000FFFFu;
-}
 
 // The kernel body.  kPeer: Q tiles come from the ranks' shards through
 // `peer` (tmQ unused) and O rows go to the ranks' output shards; K and V are
@@ -190,39 +181,45 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sptr + C::kOffMisc + 4);
   uint32_t *sel_bits = reinterpret_cast<uint32_t *>(sptr + C::kOffSel);
-  const int ntw = (T + 31) >> 5;
   const int64_t mask_row0 = (static_cast<int64_t>(b) * p.H + hg) * p.ncube;
   if constexpr (kSparse) {
-    // Key tiles this CTA visits: tile j when any of its four query cubes
-    // selects key cube 2j or 2j + 1.
+    // Key cubes this CTA visits: cube c when any of its four query cubes
+    // selects it (bits past the last cube are ignored).
     const int qc0 = blockIdx.x * 4;
-    for (int w = threadIdx.x; w < ntw; w += blockDim.x) {
-      uint32_t lo = 0u, hi = 0u;
-      for (int qc = qc0; qc < qc0 + 4 && qc < p.ncube; ++qc) {
-        const uint32_t *m = p.mask + (mask_row0 + qc) * p.nwords;
-        if (2 * w < p.nwords) lo |= __ldg(m + 2 * w);
-        if (2 * w + 1 < p.nwords) hi |= __ldg(m + 2 * w + 1);
-      }
-      uint32_t bits = pair_bits(lo) | (pair_bits(hi) << 16);
-      if (w == ntw - 1 && (T & 31)) bits &= (1u << (T & 31)) - 1u;
+    for (int w = threadIdx.x; w < p.nwords; w += blockDim.x) {
+      uint32_t bits = 0u;
+      for (int qc = qc0; qc < qc0 + 4 && qc < p.ncube; ++qc)
+        bits |= __ldg(p.mask + (mask_row0 + qc) * p.nwords + w);
+      if (w == p.nwords - 1 && (p.ncube & 31)) bits &= (1u << (p.ncube & 31)) - 1u;
       sel_bits[w] = bits;
     }
   }
-  // The key tile visited after tile j (T when none); all roles walk the same
-  // sequence.
+  // Block-sparse walk: the visited cubes in increasing order, two per
+  // 128-key tile (the first in keys 0..63 of the tile, the second in 64..127;
+  // an odd last cube is paired with zero rows).  A tile is named by its first
+  // cube; next_cube(c) is the visited cube after c (ncube when none).
+  auto next_cube = [&](int c) -> int {
+    const int n = c + 1;
+    int w = n >> 5;
+    if (w >= p.nwords) return p.ncube;
+    uint32_t x = sel_bits[w] & (0xffffffffu << (n & 31));
+    while (x == 0u) {
+      if (++w >= p.nwords) return p.ncube;
+      x = sel_bits[w];
+    }
+    return (w << 5) + __ffs(x) - 1;
+  };
+  // One past the last tile name: the walk of every role ends there.
+  const int T_end = kSparse ? p.ncube : T;
+  // The tile visited after tile j (T_end when none; j = -1: the first one);
+  // all roles walk the same sequence.
   auto next_tile = [&](int j) -> int {
     if constexpr (!kSparse) {
       return j + 1;
     } else {
-      const int n = j + 1;
-      int w = n >> 5;
-      if (w >= ntw) return T;
-      uint32_t x = sel_bits[w] & (0xffffffffu << (n & 31));
-      while (x == 0u) {
-        if (++w >= ntw) return T;
-        x = sel_bits[w];
-      }
-      return (w << 5) + __ffs(x) - 1;
+      if (j < 0) return next_cube(-1);
+      const int second = next_cube(j);
+      return second >= p.ncube ? p.ncube : next_cube(second);
     }
   };
 
@@ -295,11 +292,14 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
                       b, r0, pol);
       }
     };
-    auto copy_tile = [&](const uint8_t *base, uint32_t dst, int t0) {
+    // Rows r0 .. r0 + nrows - 1 of the tile hold tokens t0 .. t0 + nrows - 1
+    // (zeros past N).
+    auto copy_tile = [&](const uint8_t *base, uint32_t dst, int t0, int r0 = 0,
+                         int nrows = C::kBM) {
       constexpr int kChunks = C::kRowBytes / 16;  // 16-byte chunks per token row
-      for (int idx = lane; idx < C::kBM * kChunks; idx += 32) {
-        const int r = idx / kChunks, cc = idx % kChunks;
-        const int tok = t0 + r;
+      for (int idx = lane; idx < nrows * kChunks; idx += 32) {
+        const int r = r0 + idx / kChunks, cc = idx % kChunks;
+        const int tok = t0 + (r - r0);
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
         if (tok < p.N) {
           const int rk = tok / nl, n = tok - rk * nl;
@@ -388,9 +388,28 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         }
       }
     }
+    // Block-sparse: 64 rows of cube c into rows r0 .. r0 + 63 of a K or V
+    // tile, one TMA box per 128-byte column block (the maps' boxes are 64
+    // rows); a row coordinate at or past N reads zeros.
+    auto tma_cube = [&](const CUtensorMap *m, uint32_t dst, uint32_t bar, int t0, int r0) {
+      for (int h = 0; h < C::kHalves; ++h) {
+        const uint32_t d = dst + h * C::kBlockBytes + r0 * 128;
+        if (nl == 0) {
+          tma_load_4d(d, m, bar, h * C::kBoxInner, map_head, t0, map_batch, pol_kv);
+        } else {
+          const int r = t0 / nl;
+          tma_load_5d(d, m, bar, h * C::kBoxInner, map_head, t0 - r * nl, b, r, pol_kv);
+        }
+      }
+    };
+    auto tma_cube_ok = [&](int t0) {
+      if (nl == 0) return true;
+      const int r = t0 / nl;
+      return t0 - r * nl + 64 <= nl;
+    };
     int it = 0;
-    for (int j = next_tile(-1); j < T && ok; j = next_tile(j)) {
-      if (!await_tokens(j * C::kBN, j * C::kBN + C::kBN - 1)) {
+    for (int j = next_tile(-1); j < T_end && ok; j = next_tile(j)) {
+      if (!kSparse && !await_tokens(j * C::kBN, j * C::kBN + C::kBN - 1)) {
         ok = false;
         break;
       }
@@ -404,7 +423,24 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         }
         const uint32_t dst = sbase + C::kOffKV + s * C::kTileBytes;
         const uint32_t bar = bar_kv_full + 8 * s;
-        if (tma_ok(j * C::kBN)) {
+        if constexpr (kSparse) {
+          // cube j in keys 0..63, the next visited cube (or zero rows) in 64..127
+          const int cb = next_cube(j);
+          const int t1 = cb < p.ncube ? 64 * cb : 64 * p.ncube;
+          const bool tma0 = tma_cube_ok(64 * j);
+          const bool tma1 = cb < p.ncube ? tma_cube_ok(t1) : nl == 0;
+          const uint8_t *src = kv == 0 ? p.k : p.v;
+          // one copy loop for both halves (the producer runs on 88 registers)
+          for (int hf = 0; hf < 2; ++hf)
+            if (!(hf ? tma1 : tma0)) copy_tile(src, dst, hf ? t1 : 64 * j, 64 * hf, 64);
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar, (tma0 ? C::kTileBytes / 2 : 0) + (tma1 ? C::kTileBytes / 2 : 0));
+            const CUtensorMap *m = kv == 0 ? tmK : tmV;
+            if (tma0) tma_cube(m, dst, bar, 64 * j, 0);
+            if (tma1) tma_cube(m, dst, bar, t1, 64);
+          }
+        } else if (tma_ok(j * C::kBN)) {
           if (lane == 0) {
             mbar_arrive_expect_tx(bar, C::kTileBytes);
             tma_tile(kv == 0 ? tmK : tmV, dst, bar, j * C::kBN, pol_kv);
@@ -471,14 +507,14 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       // Q has landed before anything else happens (also when no key tile is
       // selected, so that no copy into shared memory outlives the CTA).
       ok = mbar_wait(bar_q, 0, abort_flag, kWaitLimitNs);
-      if (ok && j0 >= T) {
+      if (ok && j0 >= T_end) {
         // no key tile selected for this CTA: O is never written (the rows
         // come out as zeros), the epilogue only needs its barrier
         umma_commit(bar_o);
         umma_commit(bar_o + 8);
       }
-      ok = ok && (j0 >= T || mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs));
-      if (ok && j0 < T) {
+      ok = ok && (j0 >= T_end || mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs));
+      if (ok && j0 < T_end) {
         tc_fence_after();
         issue_s(0, 0);
         umma_commit(bar_s);
@@ -487,7 +523,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         umma_commit(bar_kv_empty);
         it = 1;
       }
-      for (int j = j0, jj = 0; j < T && ok; ++jj) {
+      for (int j = j0, jj = 0; j < T_end && ok; ++jj) {
         const int jn = next_tile(j);
         // Both K/V waits come first: the loads landed long ago, and no
         // barrier wait sits between a tile's PV and its next S.
@@ -496,7 +532,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         ++it;
         if (!ok) break;
         int sk = 0;
-        if (jn < T) {
+        if (jn < T_end) {
           sk = it % C::kStages;
           ok = mbar_wait(bar_kv_full + 8 * sk, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
           ++it;
@@ -504,7 +540,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         }
         ok = issue_pv(0, sv, jj == 0, jj);
         if (!ok) break;
-        if (jn < T) {
+        if (jn < T_end) {
           issue_s(0, sk);
           umma_commit(bar_s);
         } else {
@@ -512,7 +548,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         }
         ok = issue_pv(1, sv, jj == 0, jj);
         if (!ok) break;
-        if (jn < T) {
+        if (jn < T_end) {
           issue_s(1, sk);
           umma_commit(bar_s + 8);
           umma_commit(bar_kv_empty + 8 * sv);
@@ -552,7 +588,12 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
     const int qcube = (q0 + t * C::kBM + row) >> 6;
     const uint32_t *mrow = kSparse && qcube < p.ncube ? p.mask + (mask_row0 + qcube) * p.nwords
                                                      : nullptr;
-    for (int j = next_tile(-1), jj = 0; j < T; j = next_tile(j), ++jj) {
+    // Sparse: cb is the tile's second cube (ncube when the first one is the
+    // last visited); the next tile starts at the visited cube after cb.
+    int cb = kSparse ? p.ncube : 0;
+    for (int j = next_tile(-1), jj = 0; j < T_end;
+         j = kSparse ? (cb < p.ncube ? next_cube(cb) : p.ncube) : j + 1, ++jj) {
+      if constexpr (kSparse) cb = next_cube(j);
       // Warp-uniform exit: the TMEM accesses below are warp-collective.
       const bool got = mbar_wait(bar_s + 8 * t, jj & 1, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, got)) {
@@ -568,10 +609,24 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       tmem_ld32(tS + 64, &s[64]);
       tmem_ld32(tS + 96, &s[96]);
       tmem_wait_ld();
-      if (j == T - 1 && tail < C::kBN) {
+      if constexpr (!kSparse) {
+        if (j == T - 1 && tail < C::kBN) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= tail) s[c] = 0xFF800000u;  // -inf
+          for (int c = 0; c < 128; ++c)
+            if (c >= tail) s[c] = 0xFF800000u;  // -inf
+        }
+      } else {
+        // keys at or past N (zero rows in shared memory) of a partial last
+        // cube (key cubes are 0 .. ncube-1)
+        const int lim0 = j == p.ncube - 1 ? p.N - 64 * j : 64;
+        const int lim1 = cb == p.ncube - 1 ? p.N - 64 * cb : 64;
+        if (lim0 < 64 || lim1 < 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            if (c >= lim0) s[c] = 0xFF800000u;
+            if (c >= lim1) s[64 + c] = 0xFF800000u;
+          }
+        }
       }
       // Row maximum: eight independent chains of 3-input max over 16
       // scores each, then a short tree.
@@ -585,13 +640,13 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
           m = fmax3(m, __uint_as_float(e[c]), __uint_as_float(e[c + 1]));
         mc[q] = fmaxf(m, __uint_as_float(e[15]));
       }
-      // Sparse: key cube 2j is the tile's first half, 2j + 1 its second; an
-      // unselected half counts for neither the maximum nor the sum.
+      // Sparse: cube j is the tile's first half, cube cb its second; a half
+      // this row's query cube did not select counts for neither the maximum
+      // nor the sum.
       bool sel0 = true, sel1 = true;
       if constexpr (kSparse) {
-        const uint32_t word = mrow != nullptr ? __ldg(mrow + (j >> 4)) >> ((2 * j) & 31) : 0u;
-        sel0 = (word & 1u) != 0u;
-        sel1 = (word & 2u) != 0u;
+        sel0 = mrow != nullptr && ((__ldg(mrow + (j >> 5)) >> (j & 31)) & 1u) != 0u;
+        sel1 = mrow != nullptr && cb < p.ncube && ((__ldg(mrow + (cb >> 5)) >> (cb & 31)) & 1u) != 0u;
       }
       float mx;
       if constexpr (kSparse) {

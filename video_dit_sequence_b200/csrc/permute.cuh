@@ -55,6 +55,9 @@ struct PermuteParams {
   uint32_t H_vec;          // vectors per sequence-sharded token row: H*D/8
   uint32_t Hl_vec;         // vectors per head-sharded token row: Hl*D/8
   uint32_t Nl, Np, B, P;
+  FastDiv hvec;            // H*D/8 (shard modes)
+  FastDiv ntok;            // N (unshard)
+  uint32_t N;
 };
 
 constexpr int kPermThreads = 256;
@@ -124,13 +127,46 @@ __device__ __forceinline__ uint64_t exchange_unpack_src(uint32_t v, const Permut
   return (static_cast<uint64_t>(j) * p.bnl.d + bn) * p.Hl_vec + k;
 }
 
-enum PermuteMode { kModePack = 0, kModeUnpack = 1, kModeExchangePack = 2, kModeExchangeUnpack = 3 };
+// Shard, output vector v: shard row R = v / (H*D/8) = (r*B + b)*Nl + n holds
+// token t = r*Nl + n of batch b of the logical [B][N][H][D] tensor; a token
+// slot at or past N is padding and reads as zero (kNoSource).
+constexpr uint64_t kNoSource = ~0ull;
+__device__ __forceinline__ uint64_t shard_src(uint32_t v, const PermuteParams &p) {
+  uint32_t R = fdiv(v, p.hvec);
+  uint32_t k = v - R * p.hvec.d;
+  uint32_t rb = fdiv(R, p.nl);
+  uint32_t n = R - rb * p.Nl;
+  uint32_t r = fdiv(rb, p.bdiv);
+  uint32_t b = rb - r * p.B;
+  uint32_t t = r * p.Nl + n;
+  if (t >= p.N) return kNoSource;
+  return (static_cast<uint64_t>(b) * p.N + t) * p.hvec.d + k;
+}
+
+// Unshard, output vector v: logical row R = v / (H*D/8) = b*N + t; token t
+// lives in shard t / Nl at local row t % Nl.
+__device__ __forceinline__ uint64_t unshard_src(uint32_t v, const PermuteParams &p) {
+  uint32_t R = fdiv(v, p.hvec);
+  uint32_t k = v - R * p.hvec.d;
+  uint32_t b = fdiv(R, p.ntok);
+  uint32_t t = R - b * p.N;
+  uint32_t r = fdiv(t, p.nl);
+  uint32_t n = t - r * p.Nl;
+  return (static_cast<uint64_t>(r * p.B + b) * p.Nl + n) * p.hvec.d + k;
+}
+
+enum PermuteMode {
+  kModePack = 0, kModeUnpack = 1, kModeExchangePack = 2, kModeExchangeUnpack = 3,
+  kModeShard = 4, kModeUnshard = 5
+};
 
 template <int kMode>
 __device__ __forceinline__ uint64_t permute_src(uint32_t v, const PermuteParams &p) {
   if (kMode == kModePack) return pack_src(v, p);
   if (kMode == kModeUnpack) return unpack_src(v, p);
   if (kMode == kModeExchangePack) return exchange_pack_src(v, p);
+  if (kMode == kModeShard) return shard_src(v, p);
+  if (kMode == kModeUnshard) return unshard_src(v, p);
   return exchange_unpack_src(v, p);
 }
 
@@ -142,7 +178,11 @@ permute_kernel(const PermuteParams p) {
 #pragma unroll
   for (int u = 0; u < kPermUnroll; ++u) {
     uint32_t o = base + u * kPermThreads;
-    if (o < p.total_vec) v[u] = ld_stream(p.src + permute_src<kMode>(o, p));
+    if (o < p.total_vec) {
+      const uint64_t s = permute_src<kMode>(o, p);
+      v[u] = (kMode == kModeShard && s == kNoSource) ? make_uint4(0u, 0u, 0u, 0u)
+                                                     : ld_stream(p.src + s);
+    }
   }
 #pragma unroll
   for (int u = 0; u < kPermUnroll; ++u) {

@@ -100,19 +100,27 @@ int32_t *status_ptr() {
 }
 
 sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, int mode) {
-  sp_status st = check_common(s);
+  // sharding splits tokens only: any P
+  const bool shard = mode == sp::kModeShard || mode == sp::kModeUnshard;
+  sp_status st = check_common(s, !shard);
   if (st != SP_OK) return st;
   if (src == nullptr || dst == nullptr) return SP_ERR_NULL;
   if (!aligned16(src) || !aligned16(dst)) return SP_ERR_ALIGN;
   const uint32_t P = s->P, B = s->B, H = s->H, D = s->D;
-  const uint32_t Hl = H / P;
+  const uint32_t Hl = shard ? H : H / P;  // (unused by the shard modes)
   const uint32_t Nl = (s->N + P - 1) / P;
   sp::PermuteParams p;
+  std::memset(&p, 0, sizeof(p));
   p.src = static_cast<const uint4 *>(src);
   p.dst = static_cast<uint4 *>(dst);
   const bool exchange = mode == sp::kModeExchangePack || mode == sp::kModeExchangeUnpack;
-  // one rank's shard (exchange modes) or all P shards
-  p.total_vec = static_cast<uint32_t>(static_cast<uint64_t>(exchange ? 1 : P) * B * Nl * H * D / 8);
+  // one rank's shard (exchange modes), all P shards, or the logical tensor
+  p.total_vec = static_cast<uint32_t>(
+      mode == sp::kModeUnshard ? static_cast<uint64_t>(B) * s->N * H * D / 8
+                               : static_cast<uint64_t>(exchange ? 1 : P) * B * Nl * H * D / 8);
+  p.hvec = sp::make_fastdiv(H * D / 8);
+  p.ntok = sp::make_fastdiv(static_cast<uint32_t>(s->N));
+  p.N = static_cast<uint32_t>(s->N);
   p.vr = sp::make_fastdiv(Hl * D / 8);
   p.nl = sp::make_fastdiv(Nl);
   p.p = sp::make_fastdiv(P);
@@ -134,6 +142,10 @@ sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, i
     case sp::kModeExchangePack:
       sp::permute_kernel<sp::kModeExchangePack><<<blocks, sp::kPermThreads, 0, cs>>>(p);
       break;
+    case sp::kModeShard: sp::permute_kernel<sp::kModeShard><<<blocks, sp::kPermThreads, 0, cs>>>(p); break;
+    case sp::kModeUnshard:
+      sp::permute_kernel<sp::kModeUnshard><<<blocks, sp::kPermThreads, 0, cs>>>(p);
+      break;
     default:
       sp::permute_kernel<sp::kModeExchangeUnpack><<<blocks, sp::kPermThreads, 0, cs>>>(p);
       break;
@@ -146,14 +158,14 @@ sp_status permute(const void *src, void *dst, const sp_shape *s, void *stream, i
 // es: element size in bytes (2: bf16, 1: E4M3 moved as bytes).  The box is
 // 128 bytes wide: 64 bf16 or 128 E4M3 elements.
 bool make_map(CUtensorMap *m, const void *base, int D, int Hx, int N, int Bx, int64_t row_el,
-              int64_t batch_el, int es = 2) {
+              int64_t batch_el, int es = 2, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hx),
                         static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(Bx)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * es, static_cast<cuuint64_t>(row_el) * es,
                            static_cast<cuuint64_t>(batch_el) * es};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, 128, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / es), 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 4,
                    const_cast<void *>(base), dims, strides,
@@ -164,10 +176,10 @@ bool make_map(CUtensorMap *m, const void *base, int D, int Hx, int N, int Bx, in
 
 // Tensor map over rank-major sequence shards [P][B][Nl][H][D] (B > 1 and
 // P > 1), dims inner to outer (D, H, Nl, B, P).  Used only for token tiles
-// that lie inside one shard; the box is 128 rows (or Nl when smaller, in
-// which case no tile uses the map).
+// that lie inside one shard; the box is box_rows rows (or Nl when smaller,
+// in which case no tile uses the map).
 bool make_map5(CUtensorMap *m, const void *base, int D, int H, int Nl, int B, int P,
-               int es = 2) {
+               int es = 2, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t row = static_cast<cuuint64_t>(H) * D * es;
@@ -177,7 +189,7 @@ bool make_map5(CUtensorMap *m, const void *base, int D, int H, int Nl, int B, in
   cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * es, row, row * Nl,
                            row * Nl * static_cast<cuuint64_t>(B)};
   cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / es), 1,
-                       static_cast<cuuint32_t>(Nl < 128 ? Nl : 128), 1, 1};
+                       static_cast<cuuint32_t>(Nl < box_rows ? Nl : box_rows), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 5,
                    const_cast<void *>(base), dims, strides,
@@ -267,7 +279,7 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   if ((f8 || mask != nullptr) && s->D != 128) return SP_ERR_UNSUPPORTED_D;
   if (mask != nullptr) {
     if ((reinterpret_cast<uintptr_t>(mask) & 3u) != 0) return SP_ERR_ALIGN;
-    if ((s->N + 127) / 128 > 32 * sp::AttnCfg<128>::kMaxSelWords) return SP_ERR_SHAPE;
+    if ((s->N + 63) / 64 > 32 * sp::AttnCfg<128>::kMaxSelWords) return SP_ERR_SHAPE;
   }
   const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
   const int Hl = H / P;
@@ -292,13 +304,16 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   int32_t *status = status_ptr();
   if (status == nullptr) return SP_ERR_CUDA;
   CUtensorMap mq, mk, mv;
+  // the block-sparse kernel loads K and V one 64-token cube at a time
+  const int kv_rows = mask != nullptr ? 64 : 128;
   if (rank_major) {
-    if (!make_map5(&mq, q, D, H, Nl, B, P, es) || !make_map5(&mk, k, D, H, Nl, B, P, es) ||
-        !make_map5(&mv, v, D, H, Nl, B, P, es))
+    if (!make_map5(&mq, q, D, H, Nl, B, P, es) ||
+        !make_map5(&mk, k, D, H, Nl, B, P, es, kv_rows) ||
+        !make_map5(&mv, v, D, H, Nl, B, P, es, kv_rows))
       return SP_ERR_CUDA;
   } else if (!make_map(&mq, q, D, Hx, N, Bx, row_el, batch_el, es) ||
-             !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el, es) ||
-             !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el, es)) {
+             !make_map(&mk, k, D, Hx, N, Bx, row_el, batch_el, es, kv_rows) ||
+             !make_map(&mv, v, D, Hx, N, Bx, row_el, batch_el, es, kv_rows)) {
     return SP_ERR_CUDA;
   }
   sp::AttnParams p;
@@ -747,6 +762,16 @@ sp_status sp_pack(const void *xs, void *xh, const sp_shape *shape, void *stream)
 sp_status sp_unpack(const void *oh, void *os, const sp_shape *shape, void *stream) {
   NvtxRange range("sp_unpack");
   return permute(oh, os, shape, stream, sp::kModeUnpack);
+}
+
+sp_status sp_shard(const void *x, void *xs, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_shard");
+  return permute(x, xs, shape, stream, sp::kModeShard);
+}
+
+sp_status sp_unshard(const void *xs, void *x, const sp_shape *shape, void *stream) {
+  NvtxRange range("sp_unshard");
+  return permute(xs, x, shape, stream, sp::kModeUnshard);
 }
 
 sp_status sp_exchange_pack(const void *xs_r, void *send, const sp_shape *shape, void *stream) {
