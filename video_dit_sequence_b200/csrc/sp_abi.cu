@@ -500,7 +500,7 @@ bool make_map_matrix(CUtensorMap *m, const void *base, int cols, int rows, int b
   return r == CUDA_SUCCESS;
 }
 
-sp_status launch_projection(const CUtensorMap &mx, const CUtensorMap &mw, const sp::ProjParams &p,
+sp_status launch_projection(const CUtensorMap &ma, const void *w, int slots, sp::ProjParams p,
                             void *stream);
 
 sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q, void *k,
@@ -524,10 +524,8 @@ sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q
     return SP_ERR_SHAPE;
   int32_t *status = status_ptr();
   if (status == nullptr) return SP_ERR_CUDA;
-  CUtensorMap mx, mw;
-  if (!make_map_matrix(&mx, x, hidden, static_cast<int>(M64), sp::kProjBM) ||
-      !make_map_matrix(&mw, w, hidden, static_cast<int>(nout64), sp::kProjBN))
-    return SP_ERR_CUDA;
+  CUtensorMap mx;
+  if (!make_map_matrix(&mx, x, hidden, static_cast<int>(M64), 128)) return SP_ERR_CUDA;
   sp::ProjParams p;
   std::memset(&p, 0, sizeof(p));
   p.M = static_cast<int32_t>(M64);
@@ -541,8 +539,6 @@ sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q
   p.Nl = Nl;
   p.Np = Nl * P;
   p.layout = layout;
-  p.tiles_m = static_cast<int32_t>((M64 + sp::kProjBM - 1) / sp::kProjBM);
-  p.tiles_n = static_cast<int32_t>((nout64 + sp::kProjBN - 1) / sp::kProjBN);
   p.out[0] = static_cast<__nv_bfloat16 *>(q);
   p.out[1] = static_cast<__nv_bfloat16 *>(k);
   p.out[2] = static_cast<__nv_bfloat16 *>(v);
@@ -550,8 +546,7 @@ sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q
   p.status = status;
   p.a_load = sp::kALoadMatrix;
   p.rows_per_slot = p.M;
-  p.tiles_per_slot = p.tiles_m;
-  return launch_projection(mx, mw, p, stream);
+  return launch_projection(mx, w, 1, p, stream);
 }
 
 // Tensor map over a bf16 operand viewed as 4-D [d3][d2][d1 rows][d0 cols]
@@ -596,36 +591,30 @@ sp_status out_projection(const void *o, const void *w, const void *bias, void *y
     return SP_ERR_SHAPE;
   int32_t *status = status_ptr();
   if (status == nullptr) return SP_ERR_CUDA;
-  CUtensorMap ma, mw;
+  CUtensorMap ma;
   sp::ProjParams p;
   std::memset(&p, 0, sizeof(p));
   const int64_t gcols = static_cast<int64_t>(Hl) * D;
   bool ok_a;
+  int slots = 1;
   if (layout == SP_O_SEQ_SHARDED) {
     // [P][B][Nl][H][D] = rows x (H*D), row-major
-    ok_a = make_map_rows4(&ma, o, K, rows, 1, 1, K, K * rows, K * rows, sp::kProjBM);
+    ok_a = make_map_rows4(&ma, o, K, rows, 1, 1, K, K * rows, K * rows, 128);
     p.a_load = sp::kALoadMatrix;
     p.rows_per_slot = static_cast<int32_t>(rows);
-    p.tiles_per_slot = static_cast<int32_t>((rows + sp::kProjBM - 1) / sp::kProjBM);
-    p.tiles_m = p.tiles_per_slot;
   } else if (layout == SP_O_HEAD_SHARDED) {
     // [P (group)][B][Np][Hl*D]: one slot per batch, rows = tokens of the slot
-    ok_a = make_map_rows4(&ma, o, gcols, Np, B, P, gcols, gcols * Np, gcols * Np * B, sp::kProjBM);
+    ok_a = make_map_rows4(&ma, o, gcols, Np, B, P, gcols, gcols * Np, gcols * Np * B, 128);
     p.a_load = sp::kALoadHeads;
     p.rows_per_slot = Np;
-    p.tiles_per_slot = (Np + sp::kProjBM - 1) / sp::kProjBM;
-    p.tiles_m = p.tiles_per_slot * B;
+    slots = B;
   } else {
     // one rank's [P (chunk)][B*Nl][Hl*D]
-    ok_a = make_map_rows4(&ma, o, gcols, rows, P, 1, gcols, gcols * rows, gcols * rows * P,
-                          sp::kProjBM);
+    ok_a = make_map_rows4(&ma, o, gcols, rows, P, 1, gcols, gcols * rows, gcols * rows * P, 128);
     p.a_load = sp::kALoadChunks;
     p.rows_per_slot = static_cast<int32_t>(rows);
-    p.tiles_per_slot = static_cast<int32_t>((rows + sp::kProjBM - 1) / sp::kProjBM);
-    p.tiles_m = p.tiles_per_slot;
   }
-  if (!ok_a || !make_map_matrix(&mw, w, static_cast<int>(K), hidden, sp::kProjBN))
-    return SP_ERR_CUDA;
+  if (!ok_a) return SP_ERR_CUDA;
   p.M = static_cast<int32_t>(rows);
   p.K = static_cast<int32_t>(K);
   p.nout = hidden;
@@ -637,30 +626,69 @@ sp_status out_projection(const void *o, const void *w, const void *bias, void *y
   p.Nl = Nl;
   p.Np = Np;
   p.a_cols = static_cast<int32_t>(gcols);
-  p.tiles_n = (hidden + sp::kProjBN - 1) / sp::kProjBN;
   p.out_proj = 1;
   p.y = static_cast<__nv_bfloat16 *>(y);
   p.bias = static_cast<const __nv_bfloat16 *>(bias);
   p.status = status;
-  return launch_projection(ma, mw, p, stream);
+  return launch_projection(ma, w, slots, p, stream);
 }
 
-sp_status launch_projection(const CUtensorMap &mx, const CUtensorMap &mw, const sp::ProjParams &p,
+// Both projections: the tile counts for 256-row blocks, the map over w (a
+// box of 128 rows: each CTA of a pair holds half of a tile's features), and
+// the persistent launch on CTA pairs.  p holds every other field,
+// rows_per_slot included.
+sp_status launch_projection(const CUtensorMap &ma, const void *w, int slots, sp::ProjParams p,
                             void *stream) {
-  static bool attr_set[kMaxDevices] = {};
-  cudaError_t e = set_smem_once(sp::projection_kernel, sp::kProjSmemBytes, attr_set);
-  if (e != cudaSuccess) return SP_ERR_CUDA;
-  const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+  p.tiles_per_slot = (p.rows_per_slot + sp::kPairBM - 1) / sp::kPairBM;
+  const int64_t tiles_m = static_cast<int64_t>(p.tiles_per_slot) * slots;
+  p.tiles_n = (p.nout + sp::kProjBN - 1) / sp::kProjBN;
+  const int64_t tiles = tiles_m * p.tiles_n;
   if (tiles >= (int64_t(1) << 31)) return SP_ERR_SHAPE;
-  // persistent: one CTA per SM (or per tile when there are fewer tiles)
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return SP_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-  sp::projection_kernel<<<grid, sp::kProjThreads, sp::kProjSmemBytes,
-                              static_cast<cudaStream_t>(stream)>>>(mx, mw, p);
-  return launch_status(cudaGetLastError());
+  p.tiles_m = static_cast<int32_t>(tiles_m);
+  CUtensorMap mw;
+  if (!make_map_matrix(&mw, w, p.K, p.nout, 128)) return SP_ERR_CUDA;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
+  // persistent CTA pairs: as many clusters of two as can be resident at once
+  // (or one per tile when there are fewer tiles)
+  static bool attr_set[kMaxDevices] = {};
+  static int max_pairs[kMaxDevices] = {};
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(sp::kProjThreads);
+  cfg.dynamicSmemBytes = sp::kPairSmemBytes;
+  cfg.stream = cs;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(sp::projection_pair_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sp::kPairSmemBytes) != cudaSuccess)
+        return SP_ERR_CUDA;
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SP_ERR_CUDA;
+      cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, sp::projection_pair_kernel, &cfg) != cudaSuccess ||
+          n < 1)
+        return SP_ERR_CUDA;
+      max_pairs[dev] = n;
+      attr_set[dev] = true;
+    }
+  }
+  const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cudaError_t e = cudaLaunchKernelEx(&cfg, sp::projection_pair_kernel, ma, mw, p);
+  return launch_status(e == cudaSuccess ? cudaGetLastError() : e);
 }
 
 using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
