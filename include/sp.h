@@ -324,9 +324,13 @@ sp_status sp_attention_ulysses_peer(const void *const *q_shards, const void *k_g
  * (sp_attention_ulysses_overlap) walks key tiles in their fixed order and,
  * before loading the tiles of source rank r's chunk (and the Q tiles of rank
  * r's shard), waits with a bounded wait until r's counter shows that the
- * chunk has arrived.  Attention on the first chunks runs while the later
- * ones are in flight; the order of the arithmetic is unchanged, so results
- * equal sp_attention_seqsharded's bit for bit.
+ * chunk has arrived.  No collective gates the attention launch: it waits
+ * only for the chunks its tiles read, so peers' pushes still in flight (or
+ * late) overlap attention on the chunks that have arrived.  The order of the
+ * arithmetic is unchanged, so results equal sp_attention_seqsharded's bit
+ * for bit.  A rank's push and attention run in one stream, push first: an
+ * attention kernel must never wait for a push on its own GPU that could run
+ * concurrently with it.
  * Protocol: every rank owns a counter array uint64 [P] (zeroed once, before
  * any rank's first push) and a received-group buffer for K and for V.  Step
  * e = 1, 2, ... of every rank: write Q into its Q shard, then
