@@ -28,11 +28,12 @@
 //
 // The GEMM runs on CTA pairs (a cluster of two CTAs on neighbouring SMs): a
 // tile of y is 256 x 256, each CTA of the pair holds 128 of its rows of A
-// and 128 of its rows of w (64-wide K slices through a 6-stage ring), and
+// and 128 of its rows of w (128-wide K slices through a 3-stage ring), and
 // one thread of the even CTA issues 256 x 256 x 16 tcgen05 MMAs
 // (cta_group::2) that read both CTAs' shared memory and accumulate each
 // CTA's 128 rows in that CTA's tensor memory.  Against one CTA per 128 x 256
-// tile, every SM moves a third less operand data per MMA.  Each CTA's loads
+// tile, every SM moves a third less operand data per MMA.  A stage holds
+// 128 elements of K (two boxes per operand; 3 stages of 64 KB).  Each CTA's loads
 // complete on its own barrier; the odd CTA forwards that completion to the
 // even one with a remote mbarrier arrive (no multicast; the plain arrive form,
 // whose release is CTA-scoped: a cluster-scoped release per 512-cycle stage
@@ -81,10 +82,14 @@ constexpr uint32_t kProjTmemCols = 512;           // two 256-column accumulators
 constexpr uint64_t kProjWaitNs = 2000000000ull;   // 2 s per wait
 constexpr int32_t kProjStatusTimeout = 7;         // SP_ERR_TIMEOUT
 
-// A CTA pair per 256 x 256 tile (each CTA: 128 rows of A, 128 rows of w).
+// A CTA pair per 256 x 256 tile (each CTA: 128 rows of A, 128 rows of w).  A
+// stage holds 128 elements of K: two 64-wide boxes of each operand, so that
+// every stage's barrier round trip and commit cover eight MMAs.
 constexpr int kPairBM = 256;
-constexpr int kPairStages = 6;
-constexpr int kPairHalfBytes = 128 * 128;         // 128 rows x 64 bf16: 16 KB
+constexpr int kPairStages = 3;
+constexpr int kPairBoxes = 2;                     // 64-wide K boxes per operand per stage
+constexpr int kPairBoxBytes = 128 * 128;          // 128 rows x 64 bf16: 16 KB
+constexpr int kPairHalfBytes = kPairBoxes * kPairBoxBytes;   // one operand of a stage
 constexpr int kPairStageBytes = 2 * kPairHalfBytes;
 constexpr int kPairOffBar = kPairStages * kPairStageBytes;
 constexpr int kPairOffMisc = kPairOffBar + (2 * kPairStages + 5) * 8;  // ..., bar_drain
@@ -238,7 +243,8 @@ projection_pair_kernel(const __grid_constant__ CUtensorMap tmX,
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int ntiles = p.tiles_m * p.tiles_n;
-  const int nk = (p.K + kProjBK - 1) / kProjBK;
+  // stages per tile; K slices past K read as zeros and add nothing
+  const int nk = (p.K + kPairBoxes * kProjBK - 1) / (kPairBoxes * kProjBK);
 
   const uint32_t bar_full = sbase + kPairOffBar;                 // [stages]
   const uint32_t bar_empty = bar_full + 8 * kPairStages;          // [stages]
@@ -294,9 +300,12 @@ projection_pair_kernel(const __grid_constant__ CUtensorMap tmX,
           if (!ok) break;
           const uint32_t dst = sbase + s * kPairStageBytes;
           mbar_arrive_expect_tx(bar_full + 8 * s, kPairStageBytes);
-          const int k0 = kb * kProjBK;
-          proj_load_a(&tmX, dst, bar_full + 8 * s, p, k0, row0, slot, pol);
-          tma_load_4d(dst + kPairHalfBytes, &tmW, bar_full + 8 * s, k0, f0, 0, 0, pol);
+          for (int bx = 0; bx < kPairBoxes; ++bx) {
+            const int k0 = (kb * kPairBoxes + bx) * kProjBK;
+            proj_load_a(&tmX, dst + bx * kPairBoxBytes, bar_full + 8 * s, p, k0, row0, slot, pol);
+            tma_load_4d(dst + kPairHalfBytes + bx * kPairBoxBytes, &tmW, bar_full + 8 * s, k0, f0,
+                        0, 0, pol);
+          }
           issued = it + 1;
         }
       }
@@ -322,9 +331,11 @@ projection_pair_kernel(const __grid_constant__ CUtensorMap tmX,
           tc_fence_after();
           const uint32_t stage = static_cast<uint32_t>((s * kPairStageBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kProjBK / 16; ++kk)  // 32 bytes of K per MMA
-            umma_ss_pair(acc, dA + stage + kk * 2, dB + stage + kk * 2, idesc,
+          for (int kk = 0; kk < kPairBoxes * kProjBK / 16; ++kk) {  // 32 bytes of K per MMA
+            const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kPairBoxBytes) >> 4) + (kk & 3) * 2;
+            umma_ss_pair(acc, dA + stage + off, dB + stage + off, idesc,
                          (kb > 0 || kk > 0) ? 1u : 0u);
+          }
           umma_commit_pair(bar_empty + 8 * s);
           umma_commit_pair(mapa_cluster(bar_empty + 8 * s, 1));
         }
