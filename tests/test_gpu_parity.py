@@ -752,13 +752,14 @@ def _guarded(shape, dtype):
     untouched."""
     n = math.prod(shape)
     full = torch.empty(n + GUARD, dtype=dtype, device="cuda")
-    raw = full.view(torch.int16) if full.element_size() == 2 else full.view(torch.int32)
-    raw[n:] = 0x5A5A if full.element_size() == 2 else 0x5A5A5A5A
-    snap = raw[n:].clone()
+    raw = full.view(torch.uint8)
+    nb = n * full.element_size()
+    raw[nb:] = 0x5A
+    snap = raw[nb:].clone()
 
     def check(where):
         torch.cuda.synchronize()
-        assert torch.equal(raw[n:], snap), f"{where} wrote past its output"
+        assert torch.equal(raw[nb:], snap), f"{where} wrote past its output"
     return full[:n].view(shape), check
 
 
@@ -834,6 +835,28 @@ def test_outputs_stay_inside_their_buffers():
         lp, c = _guarded((B, peer.Hl, peer.Np), torch.float32)
         checks.append(c)
         sp.attention_ulysses_peer(q_list, kg, vg, o_list, peer, j, lse=lp)
+
+    # the overlapped form: every rank's received groups and counters guarded
+    groups_k, groups_v, counts, o2 = [], [], [], []
+    for _ in range(P):
+        for lst, shp, dt in ((groups_k, peer.send_chunks, torch.bfloat16),
+                             (groups_v, peer.send_chunks, torch.bfloat16),
+                             (counts, (P,), torch.int64), (o2, peer.rank_shard, torch.bfloat16)):
+            x, c = _guarded(shp, dt)
+            if dt == torch.int64:
+                x.zero_()
+            lst.append(x)
+            checks.append(c)
+    for r in range(P):
+        sp.exchange_push(ks[r], vs[r], groups_k, groups_v, counts, 1, peer, r)
+    for j in range(P):
+        sp.attention_ulysses_overlap(q_list, groups_k[j], groups_v[j], o2, counts[j], 1, peer, j)
+
+    # the logical sequence into shards and back
+    x, c = _guarded(shape.seq_sharded, torch.bfloat16); checks.append(c)
+    sp.shard(to_dev(q), x, shape)
+    y, c = _guarded((B, N, H, D), torch.bfloat16); checks.append(c)
+    sp.unshard(x, y, shape)
     _status_ok()
     for i, c in enumerate(checks):
         c(f"output {i}")
