@@ -262,11 +262,14 @@ sp_status sp_out_projection(const void *o, const void *w, const void *bias, void
  *   key cube 32*w + c; bits for cubes >= ncube are ignored.  Read only,
  *   4-byte aligned.
  * qs, ks, vs, os, lse as for sp_attention_seqsharded; D must be 128 and
- * ceil(N / 64) <= 16384 (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  The kernel
- * visits, for each pair of 128-row query tiles, only the key cubes that one
- * of their four query cubes selects, two cubes per 128-key tile in
- * increasing order.  With every cube selected the result equals
- * sp_attention_seqsharded's bit for bit; results do not depend on P. */
+ * ceil(N / 64) <= 8192 (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  Each 128-row
+ * query tile (two query cubes) visits only the key cubes that one of its two
+ * query cubes selects, two cubes per 128-key step: first the cubes that the
+ * neighbouring tile of its CTA (the next or previous 128 rows) also visits,
+ * then its own, each group in increasing order.  A row's result depends on
+ * the mask rows of its CTA's four query cubes (through that order), never on
+ * P or the layout.  With every cube selected the result equals
+ * sp_attention_seqsharded's bit for bit. */
 sp_status sp_attention_sparse_seqsharded(const void *qs, const void *ks, const void *vs,
                                          const uint32_t *mask, void *os, float *lse,
                                          const sp_shape *shape, void *stream);

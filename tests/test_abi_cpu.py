@@ -141,7 +141,7 @@ def test_argument_errors_return_before_launch(lib):
     assert sparse(0) == sp.SP_ERR_NULL
     assert sparse(C + 2) == sp.SP_ERR_ALIGN
     assert sparse(C, sp.Shape(1, 1000, 4, 64, 2)) == sp.SP_ERR_UNSUPPORTED_D
-    assert sparse(C, sp.Shape(1, 128 * 16384 + 1, 1, 128, 1)) == sp.SP_ERR_SHAPE
+    assert sparse(C, sp.Shape(1, 64 * 8192 + 1, 1, 128, 1)) == sp.SP_ERR_SHAPE   # 8,193 cubes
     proj = lambda x, w, b, q, k, v, hidden, layout, shp=sp.Shape(1, 1000, 4, 128, 2): \
         lib.sp_qkv_projection(*[ctypes.c_void_p(t) if t else None for t in (x, w, b, q, k, v)],
                               hidden, layout, ctypes.byref(shp.c()), None)

@@ -592,6 +592,84 @@ def test_sparse_cta_with_no_selected_tile():
     assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]), "junk bits")
 
 
+def _walk_schedule_mask(B, H, N, seed):
+    """Per-CTA selection patterns for the two query tiles' walks (a CTA holds
+    query cubes 4c .. 4c+3; tile 0 = cubes 4c, 4c+1, tile 1 = 4c+2, 4c+3)."""
+    nc = -(-N // 64)
+    assert nc >= 32
+    rng = np.random.default_rng(seed)
+    m = rng.random((B, H, nc, nc)) < 0.2                 # CTAs 6.. : independent
+    def sel(*cubes):
+        row = np.zeros(nc, bool)
+        row[list(cubes)] = True
+        return row
+    m[:, :, 0:2] = False                                 # CTA 0: tile 0 selects nothing
+    m[:, :, 6:8] = False                                 # CTA 1: tile 1 selects nothing
+    m[:, :, 8] = sel(*range(0, 20))                      # CTA 2: shared steps, then tile 0 alone
+    m[:, :, 9] = sel(1, 3)
+    m[:, :, 10] = sel(0, 1, 2, 3)
+    m[:, :, 11] = sel(7)                                 #   tile 1 ends on an odd pair
+    m[:, :, 12] = sel(5)                                 # CTA 3: tile 1's walk longer
+    m[:, :, 13] = sel(9, 30)
+    m[:, :, 14:16] = sel(*range(2, 31, 2))
+    m[:, :, 16] = sel(0, 1, 4, 5, 8, 9, 12, 13)          # CTA 4: shared / split alternate
+    m[:, :, 17] = sel(0, 4, 9)
+    m[:, :, 18] = sel(0, 1, 6, 7, 8, 9, 14, 15)
+    m[:, :, 19] = sel(1, 7, 15)
+    m[:, :, 20] = sel(2, 11)                             # CTA 5: equal unions, per-cube rows differ
+    m[:, :, 21] = sel(5, 12, nc - 1)
+    m[:, :, 22] = sel(5, 12, nc - 1)
+    m[:, :, 23] = sel(2, 11)
+    return m
+
+
+@pytest.mark.parametrize("P", [1, 3])
+def test_sparse_walk_schedules(P):
+    """The two query tiles of a CTA walk their own cube pairs, sharing a K/V
+    load where the walks meet: one tile empty, walks of unequal length, odd
+    tails, shared and split steps alternating, equal unions with different
+    rows.  Every row against the masked oracle; bit for bit across degrees."""
+    B, N, H, D = 1, 2000, 2, 128
+    q, k, v = _random_logical(B, N, H, D, seed=53)
+    mask = _walk_schedule_mask(B, H, N, seed=53)
+    got, lse = _run_sparse(q, k, v, mask, P, lse=True)
+    O = synth.from_seq_shards(got.reshape(P, B, -1, H, D), N)
+    rows = _rows_all(B, N, H)
+    ref, lref = oracle.attention_rows_masked(q, k, v, mask, rows)
+    gotr = O[rows[:, 0], rows[:, 2], rows[:, 1]]
+    empty = ~mask[rows[:, 0], rows[:, 1], rows[:, 2] // 64].any(axis=1)
+    assert empty.sum() == 4 * 64 * H
+    assert np.all(synth.bf16_to_f32(gotr[empty]) == 0.0)
+    assert np.all(lse[rows[empty, 0], rows[empty, 1], rows[empty, 2]] == -np.inf)
+    assert_parity(compare(gotr[~empty], ref[~empty], rows[~empty, 1]), f"walk schedules P={P}")
+    gl = lse[rows[~empty, 0], rows[~empty, 1], rows[~empty, 2]]
+    assert np.max(np.abs(gl - lref[~empty])) < 2e-2
+    if P > 1:
+        one, _ = _run_sparse(q, k, v, mask, 1)
+        assert np.array_equal(O, synth.from_seq_shards(one.reshape(1, B, -1, H, D), N))
+
+
+def test_sparse_plan_at_the_cube_limit():
+    """8,192 key cubes (524,288 tokens), the most a CTA's plan holds: one
+    query cube selects every key cube, the others about 2 %.  Rows of the
+    first, a middle and the last CTAs against the masked oracle."""
+    B, N, H, D, P = 1, 64 * 8192, 1, 128, 2
+    nc = N // 64
+    q, k, v = _random_logical(B, N, H, D, seed=59)
+    rng = np.random.default_rng(59)
+    mask = (rng.integers(0, 50, size=(B, H, nc, nc), dtype=np.uint8) == 0)
+    mask[0, 0, nc - 4] = True                        # tile 0 of the last CTA: a full plan
+    got, lse = _run_sparse(q, k, v, mask, P, lse=True)
+    O = synth.from_seq_shards(got.reshape(P, B, -1, H, D), N)
+    idx = np.concatenate([np.arange(0, 300), N // 2 + np.arange(256), np.arange(N - 300, N)])
+    rows = np.stack([np.zeros_like(idx), np.zeros_like(idx), idx], axis=1)
+    ref, lref = oracle.attention_rows_masked(q, k, v, mask, rows)
+    gotr = O[rows[:, 0], rows[:, 2], rows[:, 1]]
+    assert mask[0, 0, idx // 64].any(axis=1).all()
+    assert_parity(compare(gotr, ref, rows[:, 1]), "sparse at the cube limit")
+    assert np.max(np.abs(lse[0, 0, idx] - lref)) < 2e-2
+
+
 # ------------------------------------------------------------------ projection
 
 def _proj_inputs(B, N, H, D, P, hidden, seed, bias=True):

@@ -131,11 +131,17 @@ struct AttnCfg {
   static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
   static constexpr int kNumBar = 1 + 2 * kStages + 9;  // ..., bar_o[2], bar_drain
   static constexpr int kOffMisc = kOffBar + kNumBar * 8;
-  // Block-sparse variant: one bit per 64-token key cube, set when any query
-  // cube of the CTA selects it.
-  static constexpr int kMaxSelWords = 512;                  // 16,384 key cubes
-  static constexpr int kOffSel = kOffMisc + 16;
-  static constexpr int kSmemBytes = kOffSel + 4 * kMaxSelWords + 1024;  // + alignment slack
+  // Misc: TMEM base, abort flag, per ring slot the index of the last load
+  // issued into it (-1: none), then the block-sparse plan's two list lengths.
+  static constexpr int kOffCount = kOffMisc + 16 + 4 * kStages;
+  static constexpr int kOffPlan = kOffCount + 16;
+  static constexpr int kSmemBytes = kOffPlan + 1024;  // + alignment slack
+  // Block-sparse plan: per query tile, the 64-token key cubes it visits as
+  // 16-bit indices (and a closing ncube when their number is odd).
+  static constexpr int kMaxPlanCubes = 8192;
+  static constexpr int kPlanStride = kMaxPlanCubes + 2;
+  static constexpr int kSmemBytesSparse = kOffPlan + 2 * 2 * kPlanStride + 1024;
+  static_assert(kSmemBytesSparse <= 227 * 1024, "shared memory per CTA");
   static constexpr int kThreads = 320;
   static constexpr uint32_t kColS1 = 128;
   static constexpr uint32_t kColO0 = 256;
@@ -150,13 +156,17 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 // `peer` (tmQ unused) and O rows go to the ranks' output shards; K and V are
 // this rank's received head group, addressed as for the fused call.
 // kSparse: a block mask over 64-token cubes restricts which keys each query
-// attends; the CTA walks only the key tiles that some of its query cubes
-// select, and each row masks the unselected halves of those tiles.
+// attends.  Each query tile walks only the key cubes that one of its two
+// query cubes selects, two cubes per 128-key step, from a per-CTA plan
+// listing first the cubes both tiles visit; where both walks are at the same
+// pair, one K/V load serves both.  Each row masks the cubes its own query
+// cube did not select.
 template <int D, bool kF8, bool kPeer, bool kSparse = false>
 __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUtensorMap *tmK,
                                                const CUtensorMap *tmV, const AttnParams &p,
                                                const PeerArgs *peer) {
   using C = AttnCfg<D, kF8>;
+  static_assert(!kSparse || C::kHalves == 2, "the block-sparse loads take two column blocks");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -180,47 +190,66 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   const uint32_t bar_drain = bar_o + 16;                  // the MMA thread's last commit
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sptr + C::kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sptr + C::kOffMisc + 4);
-  uint32_t *sel_bits = reinterpret_cast<uint32_t *>(sptr + C::kOffSel);
+  int *slot_item = reinterpret_cast<int *>(sptr + C::kOffMisc + 16);
+  int *plan_n = reinterpret_cast<int *>(sptr + C::kOffCount);
+  uint16_t *plan = reinterpret_cast<uint16_t *>(sptr + C::kOffPlan);
   const int64_t mask_row0 = (static_cast<int64_t>(b) * p.H + hg) * p.ncube;
   if constexpr (kSparse) {
-    // Key cubes this CTA visits: cube c when any of its four query cubes
-    // selects it (bits past the last cube are ignored).
-    const int qc0 = blockIdx.x * 4;
-    for (int w = threadIdx.x; w < p.nwords; w += blockDim.x) {
-      uint32_t bits = 0u;
-      for (int qc = qc0; qc < qc0 + 4 && qc < p.ncube; ++qc)
-        bits |= __ldg(p.mask + (mask_row0 + qc) * p.nwords + w);
-      if (w == p.nwords - 1 && (p.ncube & 31)) bits &= (1u << (p.ncube & 31)) - 1u;
-      sel_bits[w] = bits;
+    // The plan, built once per CTA by warps 0 and 1.  Query tile t (query
+    // cubes 4x + 2t and 4x + 2t + 1) visits the key cubes either of them
+    // selects: first those the other tile visits too, then its own, each
+    // group in increasing order, two per 128-key step.  Both tiles' walks
+    // then start with the same pairs, which one K/V load serves; the rest of
+    // the steps take a load per tile.  Bits past the last cube are ignored.
+    if (warp < 2) {
+      const int t = warp;
+      const int qa = blockIdx.x * 4;
+      uint16_t *list = plan + t * C::kPlanStride;
+      int n = 0;
+      for (int pass = 0; pass < 2; ++pass) {
+        for (int w0 = 0; w0 < p.nwords; w0 += 32) {
+          const int w = w0 + lane;
+          uint32_t bits = 0u;
+          if (w < p.nwords) {
+            uint32_t u0 = 0u, u1 = 0u;
+            for (int qc = qa; qc < qa + 4 && qc < p.ncube; ++qc) {
+              const uint32_t row = __ldg(p.mask + (mask_row0 + qc) * p.nwords + w);
+              if (qc < qa + 2) u0 |= row;
+              else u1 |= row;
+            }
+            if (w == p.nwords - 1 && (p.ncube & 31)) {
+              u0 &= (1u << (p.ncube & 31)) - 1u;
+              u1 &= (1u << (p.ncube & 31)) - 1u;
+            }
+            bits = pass == 0 ? (u0 & u1) : t == 0 ? (u0 & ~u1) : (u1 & ~u0);
+          }
+          // exclusive prefix of the lanes' counts: where this lane's cubes go
+          const int cnt = __popc(bits);
+          int incl = cnt;
+#pragma unroll
+          for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += v;
+          }
+          int pos = n + incl - cnt;
+          while (bits != 0u) {
+            list[pos++] = static_cast<uint16_t>(32 * w + __ffs(bits) - 1);
+            bits &= bits - 1u;
+          }
+          n += __shfl_sync(0xffffffffu, incl, 31);
+        }
+      }
+      if (lane == 0) {
+        if (n & 1) list[n] = static_cast<uint16_t>(p.ncube);
+        plan_n[t] = n;
+      }
     }
   }
-  // Block-sparse walk: the visited cubes in increasing order, two per
-  // 128-key tile (the first in keys 0..63 of the tile, the second in 64..127;
-  // an odd last cube is paired with zero rows).  A tile is named by its first
-  // cube; next_cube(c) is the visited cube after c (ncube when none).
-  auto next_cube = [&](int c) -> int {
-    const int n = c + 1;
-    int w = n >> 5;
-    if (w >= p.nwords) return p.ncube;
-    uint32_t x = sel_bits[w] & (0xffffffffu << (n & 31));
-    while (x == 0u) {
-      if (++w >= p.nwords) return p.ncube;
-      x = sel_bits[w];
-    }
-    return (w << 5) + __ffs(x) - 1;
-  };
-  // One past the last tile name: the walk of every role ends there.
-  const int T_end = kSparse ? p.ncube : T;
-  // The tile visited after tile j (T_end when none; j = -1: the first one);
-  // all roles walk the same sequence.
-  auto next_tile = [&](int j) -> int {
-    if constexpr (!kSparse) {
-      return j + 1;
-    } else {
-      if (j < 0) return next_cube(-1);
-      const int second = next_cube(j);
-      return second >= p.ncube ? p.ncube : next_cube(second);
-    }
+  // Step i of tile t's walk: cubes (x, y) = list entries 2i and 2i + 1
+  // (y = ncube: zero rows); the walk has ceil(n_t / 2) steps.
+  auto pair_at = [&](int t, int i) -> int2 {
+    const uint32_t v = *reinterpret_cast<const uint32_t *>(plan + t * C::kPlanStride + 2 * i);
+    return make_int2(static_cast<int>(v & 0xffffu), static_cast<int>(v >> 16));
   };
 
   if (threadIdx.x == 0) {
@@ -237,6 +266,7 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
+    for (int s = 0; s < C::kStages; ++s) slot_item[s] = -1;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -249,19 +279,21 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   const uint32_t tmem = *tmem_slot;
 
   bool ok = true;
-  // K/V ring loads this thread issued (the TMA producer's lane 0): on the
-  // abort path the last kStages of them may still be in flight.
-  int issued = 0;
-  bool q_issued = false;
+  bool q_issued = false;  // the Q copies were issued (producer warp 8)
   // Block-sparse kernel: 12 warps, so that its per-row mask state fits.  The
-  // third warpgroup (TMA, MMA and two idle warps) gives registers to the two
-  // softmax warpgroups: 384 x 168 at launch = 2 x 128 x 208 + 128 x 88, and
-  // each sub-partition holds 208 + 208 + 88 registers per lane (<= 512).
+  // third warpgroup (two TMA producers, the MMA warp and an idle warp) gives
+  // registers to the two softmax warpgroups: 384 x 168 at launch =
+  // 2 x 128 x 208 + 128 x 88, and each sub-partition holds 208 + 208 + 88
+  // registers per lane (<= 512).
   constexpr bool kSplitRegs = kSparse;
-  if (warp == 8) {
+  if (warp == 8 || (kSparse && warp == 10)) {
     if constexpr (kSplitRegs) asm volatile("setmaxnreg.dec.sync.aligned.u32 88;");
     // ---------------------------------------------------------------- producer
-    // One elected lane issues the TMA loads.  In the rank-major layout a
+    // Warp 8 loads Q and the K/V ring; in the block-sparse kernel warp 10
+    // loads the ring's V slots and warp 8 its K slots, since each slot there
+    // takes four TMA boxes (two cubes x two 128-byte column blocks), which
+    // four lanes issue together.  Otherwise one elected lane issues the TMA
+    // loads.  In the rank-major layout a
     // 128-token tile that crosses a shard boundary is two strided blocks,
     // which one TMA box cannot describe: the whole warp copies such a tile
     // with 16-byte loads into the same 128-byte-swizzled layout the TMA
@@ -357,9 +389,10 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       fence_proxy_async_smem();
     };
     // Q: both tiles complete one barrier.
-    ok = await_tokens(q0, q0 + 2 * C::kBM - 1);
+    const bool q_loader = warp == 8;
+    ok = !q_loader || await_tokens(q0, q0 + 2 * C::kBM - 1);
     uint32_t q_tx = 0;
-    for (int t = 0; t < 2 && ok; ++t) {
+    for (int t = 0; t < 2 && ok && q_loader; ++t) {
       const uint32_t dst = sbase + C::kOffQ + t * C::kTileBytes;
       if (kPeer) {
         if (peer_q_ok(q0 + t * C::kBM)) q_tx += C::kTileBytes;
@@ -370,8 +403,8 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       }
     }
     __syncwarp();
-    q_issued = ok;
-    if (lane == 0 && ok) {
+    q_issued = ok && q_loader;
+    if (lane == 0 && q_issued) {
       mbar_arrive_expect_tx(bar_q, q_tx);
       for (int t = 0; t < 2; ++t) {
         const int t0 = q0 + t * C::kBM;
@@ -388,18 +421,15 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         }
       }
     }
-    // Block-sparse: 64 rows of cube c into rows r0 .. r0 + 63 of a K or V
-    // tile, one TMA box per 128-byte column block (the maps' boxes are 64
-    // rows); a row coordinate at or past N reads zeros.
-    auto tma_cube = [&](const CUtensorMap *m, uint32_t dst, uint32_t bar, int t0, int r0) {
-      for (int h = 0; h < C::kHalves; ++h) {
-        const uint32_t d = dst + h * C::kBlockBytes + r0 * 128;
-        if (nl == 0) {
-          tma_load_4d(d, m, bar, h * C::kBoxInner, map_head, t0, map_batch, pol_kv);
-        } else {
-          const int r = t0 / nl;
-          tma_load_5d(d, m, bar, h * C::kBoxInner, map_head, t0 - r * nl, b, r, pol_kv);
-        }
+    // Block-sparse: column block h of the 64 rows of the cube starting at
+    // token t0, one TMA box (the maps' boxes are 64 rows); a row coordinate
+    // at or past N reads zeros.
+    auto tma_box = [&](const CUtensorMap *m, uint32_t d, uint32_t bar, int h, int t0) {
+      if (nl == 0) {
+        tma_load_4d(d, m, bar, h * C::kBoxInner, map_head, t0, map_batch, pol_kv);
+      } else {
+        const int r = t0 / nl;
+        tma_load_5d(d, m, bar, h * C::kBoxInner, map_head, t0 - r * nl, b, r, pol_kv);
       }
     };
     auto tma_cube_ok = [&](int t0) {
@@ -408,50 +438,91 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
       return t0 - r * nl + 64 <= nl;
     };
     int it = 0;
-    for (int j = next_tile(-1); j < T_end && ok; j = next_tile(j)) {
-      if (!kSparse && !await_tokens(j * C::kBN, j * C::kBN + C::kBN - 1)) {
-        ok = false;
-        break;
-      }
-      for (int kv = 0; kv < 2; ++kv, ++it) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1;
-        const bool free_slot = mbar_wait(bar_kv_empty + 8 * s, ph ^ 1u, abort_flag, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, free_slot)) {
+    if constexpr (!kSparse) {
+      for (int j = 0; j < T && ok; ++j) {
+        if (!await_tokens(j * C::kBN, j * C::kBN + C::kBN - 1)) {
           ok = false;
           break;
         }
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          const bool free_slot = mbar_wait(bar_kv_empty + 8 * s, ph ^ 1u, abort_flag, kWaitLimitNs);
+          if (!__all_sync(0xffffffffu, free_slot)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sbase + C::kOffKV + s * C::kTileBytes;
+          const uint32_t bar = bar_kv_full + 8 * s;
+          if (lane == 0) slot_item[s] = it;
+          if (tma_ok(j * C::kBN)) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(bar, C::kTileBytes);
+              tma_tile(kv == 0 ? tmK : tmV, dst, bar, j * C::kBN, pol_kv);
+            }
+          } else {
+            copy_tile(kv == 0 ? p.k : p.v, dst, j * C::kBN);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+          }
+          __syncwarp();
+        }
+      }
+    } else {
+      // Ring position it: K (kv = 0) or V (kv = 1) rows of the cube pair pr,
+      // cube pr.x in rows 0..63 and cube pr.y (zeros when ncube) in 64..127.
+      // Each warp loads the positions of its own kind and steps over the rest.
+      const int my_kv = warp == 8 ? 0 : 1;
+      auto load_pair = [&](int kv, int2 pr) -> bool {
+        const int pos = it++;
+        if (kv != my_kv) return true;
+        const int s = pos % C::kStages;
+        const uint32_t ph = (pos / C::kStages) & 1;
+        const bool free_slot = mbar_wait(bar_kv_empty + 8 * s, ph ^ 1u, abort_flag, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, free_slot)) return false;
         const uint32_t dst = sbase + C::kOffKV + s * C::kTileBytes;
         const uint32_t bar = bar_kv_full + 8 * s;
-        if constexpr (kSparse) {
-          // cube j in keys 0..63, the next visited cube (or zero rows) in 64..127
-          const int cb = next_cube(j);
-          const int t1 = cb < p.ncube ? 64 * cb : 64 * p.ncube;
-          const bool tma0 = tma_cube_ok(64 * j);
-          const bool tma1 = cb < p.ncube ? tma_cube_ok(t1) : nl == 0;
-          const uint8_t *src = kv == 0 ? p.k : p.v;
-          // one copy loop for both halves (the producer runs on 88 registers)
-          for (int hf = 0; hf < 2; ++hf)
-            if (!(hf ? tma1 : tma0)) copy_tile(src, dst, hf ? t1 : 64 * j, 64 * hf, 64);
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_expect_tx(bar, (tma0 ? C::kTileBytes / 2 : 0) + (tma1 ? C::kTileBytes / 2 : 0));
-            const CUtensorMap *m = kv == 0 ? tmK : tmV;
-            if (tma0) tma_cube(m, dst, bar, 64 * j, 0);
-            if (tma1) tma_cube(m, dst, bar, t1, 64);
-          }
-        } else if (tma_ok(j * C::kBN)) {
-          if (lane == 0) {
-            mbar_arrive_expect_tx(bar, C::kTileBytes);
-            tma_tile(kv == 0 ? tmK : tmV, dst, bar, j * C::kBN, pol_kv);
-          }
-        } else {
-          copy_tile(kv == 0 ? p.k : p.v, dst, j * C::kBN);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar);
+        const int t0 = 64 * pr.x, t1 = 64 * pr.y;
+        const bool tma0 = tma_cube_ok(t0);
+        const bool tma1 = pr.y < p.ncube ? tma_cube_ok(t1) : nl == 0;
+        const uint8_t *src = kv == 0 ? p.k : p.v;
+        // one copy loop for both halves (the producer runs on 88 registers)
+        for (int hf = 0; hf < 2; ++hf)
+          if (!(hf ? tma1 : tma0)) copy_tile(src, dst, hf ? t1 : t0, 64 * hf, 64);
+        __syncwarp();
+        if (lane == 0) {
+          slot_item[s] = pos;
+          mbar_arrive_expect_tx(bar, (tma0 ? C::kTileBytes / 2 : 0) + (tma1 ? C::kTileBytes / 2 : 0));
         }
         __syncwarp();
-        issued = it + 1;
+        // lane 2 hf + h copies cube half hf, column block h: one TMA box each
+        if (lane < 2 * C::kHalves && ((lane >> 1) ? tma1 : tma0))
+          tma_box(kv == 0 ? tmK : tmV, dst + (lane & 1) * C::kBlockBytes + (lane >> 1) * 64 * 128,
+                  bar, lane & 1, (lane >> 1) ? t1 : t0);
+        __syncwarp();
+        return true;
+      };
+      // The ring order, which the MMA thread follows: K of both walks' first
+      // steps, then per step i the V of step i and K of step i+1 for query
+      // tile 0, then the same for tile 1; a slot is loaded once when both
+      // walks are at the same pair.
+      const int len0 = plan_n[0], len1 = plan_n[1];
+      bool a0 = len0 > 0, a1 = len1 > 0;
+      int2 c0 = a0 ? pair_at(0, 0) : make_int2(0, 0), c1 = a1 ? pair_at(1, 0) : make_int2(0, 0);
+      if (ok && a0) ok = load_pair(0, c0);
+      if (ok && a1 && !(a0 && c0.x == c1.x && c0.y == c1.y)) ok = load_pair(0, c1);
+      for (int i = 1; ok && (a0 || a1); ++i) {
+        const bool na0 = 2 * i < len0, na1 = 2 * i < len1;
+        const int2 n0 = na0 ? pair_at(0, i) : c0, n1 = na1 ? pair_at(1, i) : c1;
+        const bool sh_cur = a0 && a1 && c0.x == c1.x && c0.y == c1.y;
+        const bool sh_nxt = na0 && na1 && n0.x == n1.x && n0.y == n1.y;
+        if (a0) ok = load_pair(1, c0) && (!na0 || load_pair(0, n0));
+        if (ok && a1 && !sh_cur) ok = load_pair(1, c1);
+        if (ok && na1 && !sh_nxt) ok = load_pair(0, n1);
+        c0 = n0;
+        c1 = n1;
+        a0 = na0;
+        a1 = na1;
       }
     }
   } else if (warp == 9) {
@@ -503,61 +574,137 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
         return true;
       };
       int it = 0;
-      const int j0 = next_tile(-1);
       // Q has landed before anything else happens (also when no key tile is
       // selected, so that no copy into shared memory outlives the CTA).
       ok = mbar_wait(bar_q, 0, abort_flag, kWaitLimitNs);
-      if (ok && j0 >= T_end) {
-        // no key tile selected for this CTA: O is never written (the rows
-        // come out as zeros), the epilogue only needs its barrier
-        umma_commit(bar_o);
-        umma_commit(bar_o + 8);
-      }
-      ok = ok && (j0 >= T_end || mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs));
-      if (ok && j0 < T_end) {
-        tc_fence_after();
-        issue_s(0, 0);
-        umma_commit(bar_s);
-        issue_s(1, 0);
-        umma_commit(bar_s + 8);
-        umma_commit(bar_kv_empty);
-        it = 1;
-      }
-      for (int j = j0, jj = 0; j < T_end && ok; ++jj) {
-        const int jn = next_tile(j);
-        // Both K/V waits come first: the loads landed long ago, and no
-        // barrier wait sits between a tile's PV and its next S.
-        const int sv = it % C::kStages;
-        ok = mbar_wait(bar_kv_full + 8 * sv, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
-        ++it;
-        if (!ok) break;
-        int sk = 0;
-        if (jn < T_end) {
-          sk = it % C::kStages;
-          ok = mbar_wait(bar_kv_full + 8 * sk, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
+      if constexpr (!kSparse) {
+        ok = ok && mbar_wait(bar_kv_full, 0, abort_flag, kWaitLimitNs);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          umma_commit(bar_s);
+          issue_s(1, 0);
+          umma_commit(bar_s + 8);
+          umma_commit(bar_kv_empty);
+          it = 1;
+        }
+        for (int j = 0; j < T && ok; ++j) {
+          const bool more = j + 1 < T;
+          // Both K/V waits come first: the loads landed long ago, and no
+          // barrier wait sits between a tile's PV and its next S.
+          const int sv = it % C::kStages;
+          ok = mbar_wait(bar_kv_full + 8 * sv, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
           ++it;
           if (!ok) break;
+          int sk = 0;
+          if (more) {
+            sk = it % C::kStages;
+            ok = mbar_wait(bar_kv_full + 8 * sk, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
+            ++it;
+            if (!ok) break;
+          }
+          ok = issue_pv(0, sv, j == 0, j);
+          if (!ok) break;
+          if (more) {
+            issue_s(0, sk);
+            umma_commit(bar_s);
+          } else {
+            umma_commit(bar_o);
+          }
+          ok = issue_pv(1, sv, j == 0, j);
+          if (!ok) break;
+          if (more) {
+            issue_s(1, sk);
+            umma_commit(bar_s + 8);
+            umma_commit(bar_kv_empty + 8 * sv);
+            umma_commit(bar_kv_empty + 8 * sk);
+          } else {
+            umma_commit(bar_o + 8);
+            umma_commit(bar_kv_empty + 8 * sv);
+          }
         }
-        ok = issue_pv(0, sv, jj == 0, jj);
-        if (!ok) break;
-        if (jn < T_end) {
-          issue_s(0, sk);
-          umma_commit(bar_s);
-        } else {
-          umma_commit(bar_o);
+      } else {
+        // Each query tile walks its own cube pairs, in the producer's ring
+        // order.  Per step i: O_0 += P_0 V_0(i), S_0 = Q_0 K_0(i+1)^T, then
+        // the same for tile 1; a slot shared by both walks is released after
+        // tile 1's MMAs, any other one after its own tile's.  A tile whose
+        // walk is shorter stops early: its O barrier follows its last PV, and
+        // a tile with no selected cube commits it before any MMA (its rows
+        // come out as zeros).
+        auto take = [&](int &slot) -> bool {
+          slot = it % C::kStages;
+          const bool got =
+              mbar_wait(bar_kv_full + 8 * slot, (it / C::kStages) & 1, abort_flag, kWaitLimitNs);
+          ++it;
+          return got;
+        };
+        const int len0 = plan_n[0], len1 = plan_n[1];
+        bool a0 = len0 > 0, a1 = len1 > 0;
+        int2 c0 = a0 ? pair_at(0, 0) : make_int2(0, 0), c1 = a1 ? pair_at(1, 0) : make_int2(0, 0);
+        if (ok && !a0) umma_commit(bar_o);
+        if (ok && !a1) umma_commit(bar_o + 8);
+        const bool sh0 = a0 && a1 && c0.x == c1.x && c0.y == c1.y;
+        int sk0 = 0, sk1 = 0;
+        if (ok && a0) {
+          ok = take(sk0);
+          if (ok) {
+            tc_fence_after();
+            issue_s(0, sk0);
+            umma_commit(bar_s);
+            if (!sh0) umma_commit(bar_kv_empty + 8 * sk0);
+          }
         }
-        ok = issue_pv(1, sv, jj == 0, jj);
-        if (!ok) break;
-        if (jn < T_end) {
-          issue_s(1, sk);
-          umma_commit(bar_s + 8);
-          umma_commit(bar_kv_empty + 8 * sv);
-          umma_commit(bar_kv_empty + 8 * sk);
-        } else {
-          umma_commit(bar_o + 8);
-          umma_commit(bar_kv_empty + 8 * sv);
+        if (ok && a1) {
+          if (sh0) sk1 = sk0;
+          else ok = take(sk1);
+          if (ok) {
+            tc_fence_after();
+            issue_s(1, sk1);
+            umma_commit(bar_s + 8);
+            umma_commit(bar_kv_empty + 8 * sk1);
+          }
         }
-        j = jn;
+        for (int jj = 0; ok && (a0 || a1); ++jj) {
+          const bool na0 = 2 * (jj + 1) < len0, na1 = 2 * (jj + 1) < len1;
+          const int2 n0 = na0 ? pair_at(0, jj + 1) : c0, n1 = na1 ? pair_at(1, jj + 1) : c1;
+          const bool sh_cur = a0 && a1 && c0.x == c1.x && c0.y == c1.y;
+          const bool sh_nxt = na0 && na1 && n0.x == n1.x && n0.y == n1.y;
+          int sv0 = 0;
+          sk0 = 0;
+          if (a0) {
+            ok = take(sv0) && (!na0 || take(sk0));
+            ok = ok && issue_pv(0, sv0, jj == 0, jj);
+            if (!ok) break;
+            if (na0) {
+              issue_s(0, sk0);
+              umma_commit(bar_s);
+            } else {
+              umma_commit(bar_o);
+            }
+            if (!sh_cur) umma_commit(bar_kv_empty + 8 * sv0);
+            if (na0 && !sh_nxt) umma_commit(bar_kv_empty + 8 * sk0);
+          }
+          if (a1) {
+            int sv1 = sv0;
+            sk1 = sk0;
+            if (!sh_cur) ok = take(sv1);
+            if (ok && na1 && !sh_nxt) ok = take(sk1);
+            ok = ok && issue_pv(1, sv1, jj == 0, jj);
+            if (!ok) break;
+            if (na1) {
+              issue_s(1, sk1);
+              umma_commit(bar_s + 8);
+            } else {
+              umma_commit(bar_o + 8);
+            }
+            umma_commit(bar_kv_empty + 8 * sv1);
+            if (na1) umma_commit(bar_kv_empty + 8 * sk1);
+          }
+          c0 = n0;
+          c1 = n1;
+          a0 = na0;
+          a1 = na1;
+        }
       }
     }
     __syncwarp();
@@ -588,12 +735,13 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
     const int qcube = (q0 + t * C::kBM + row) >> 6;
     const uint32_t *mrow = kSparse && qcube < p.ncube ? p.mask + (mask_row0 + qcube) * p.nwords
                                                      : nullptr;
-    // Sparse: cb is the tile's second cube (ncube when the first one is the
-    // last visited); the next tile starts at the visited cube after cb.
-    int cb = kSparse ? p.ncube : 0;
-    for (int j = next_tile(-1), jj = 0; j < T_end;
-         j = kSparse ? (cb < p.ncube ? next_cube(cb) : p.ncube) : j + 1, ++jj) {
-      if constexpr (kSparse) cb = next_cube(j);
+    // Sparse: this tile's walk; step jj covers cubes pr.x (keys 0..63) and
+    // pr.y (keys 64..127, ncube when none).  Dense: step jj is key tile jj.
+    const int steps = kSparse ? (plan_n[t] + 1) / 2 : T;
+    for (int jj = 0; jj < steps; ++jj) {
+      const int2 pr = kSparse ? pair_at(t, jj) : make_int2(jj, 0);
+      const int j = pr.x;
+      [[maybe_unused]] const int cb = pr.y;
       // Warp-uniform exit: the TMEM accesses below are warp-collective.
       const bool got = mbar_wait(bar_s + 8 * t, jj & 1, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, got)) {
@@ -805,14 +953,16 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
   if (*abort_flag) {
     // Before the CTA's shared and tensor memory are released, let the
     // asynchronous work it issued land: the TMA copies of Q and of the last
-    // kStages ring loads (earlier slots were consumed, so they landed), and
-    // every MMA the issuing thread enqueued (one more commit, then its
-    // barrier).  None of these depends on another thread, so each bounded
-    // wait ends; if one does not, the status word already holds the error.
+    // load issued into each ring slot (earlier loads into a slot were
+    // consumed, so they landed), and every MMA the issuing thread enqueued
+    // (one more commit, then its barrier).  None of these depends on another
+    // thread, so each bounded wait ends; if one does not, the status word
+    // already holds the error.
     if (warp == 8 && lane == 0) {
       if (q_issued) mbar_wait_drain(bar_q, 0, kWaitLimitNs);
-      for (int i = issued > C::kStages ? issued - C::kStages : 0; i < issued; ++i)
-        mbar_wait_drain(bar_kv_full + 8 * (i % C::kStages), (i / C::kStages) & 1, kWaitLimitNs);
+      for (int s = 0; s < C::kStages; ++s)
+        if (slot_item[s] >= 0)
+          mbar_wait_drain(bar_kv_full + 8 * s, (slot_item[s] / C::kStages) & 1, kWaitLimitNs);
     }
     if (warp == 9 && lane == 0) {
       umma_commit(bar_drain);

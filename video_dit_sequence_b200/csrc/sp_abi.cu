@@ -279,7 +279,7 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   if ((f8 || mask != nullptr) && s->D != 128) return SP_ERR_UNSUPPORTED_D;
   if (mask != nullptr) {
     if ((reinterpret_cast<uintptr_t>(mask) & 3u) != 0) return SP_ERR_ALIGN;
-    if ((s->N + 63) / 64 > 32 * sp::AttnCfg<128>::kMaxSelWords) return SP_ERR_SHAPE;
+    if ((s->N + 63) / 64 > sp::AttnCfg<128>::kMaxPlanCubes) return SP_ERR_SHAPE;
   }
   const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
   const int Hl = H / P;
@@ -347,11 +347,11 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   if (mask != nullptr) {
     using C = sp::AttnCfg<128>;
     static bool attr_set[kMaxDevices] = {};
-    cudaError_t e = set_smem_once(sp::attention_sparse_kernel, C::kSmemBytes, attr_set);
+    cudaError_t e = set_smem_once(sp::attention_sparse_kernel, C::kSmemBytesSparse, attr_set);
     if (e != cudaSuccess) return SP_ERR_CUDA;
     dim3 grid((Np + 2 * C::kBM - 1) / (2 * C::kBM), H, B);
     // 12 warps: the block-sparse kernel splits registers between warpgroups
-    sp::attention_sparse_kernel<<<grid, 384, C::kSmemBytes, cs>>>(mq, mk, mv, p);
+    sp::attention_sparse_kernel<<<grid, 384, C::kSmemBytesSparse, cs>>>(mq, mk, mv, p);
     return launch_status(cudaGetLastError());
   }
   cudaError_t e = f8        ? launch_attention<128, true>(mq, mk, mv, p, B, cs)
