@@ -246,8 +246,10 @@ typedef enum {
 sp_status sp_out_projection(const void *o, const void *w, const void *bias, void *y,
                             int32_t hidden, int32_t layout, const sp_shape *shape, void *stream);
 
-/* Tokens per cube of the block-sparse call's mask. */
+/* Tokens per cube of the block-sparse call's mask, and the most cubes
+ * (ceil(N / SP_SPARSE_CUBE)) the call takes: 524,288 tokens. */
 #define SP_SPARSE_CUBE 64
+#define SP_SPARSE_MAX_CUBES 8192
 
 /* Block-sparse variant of sp_attention_seqsharded: the sparse stage of video
  * sparse attention, which the FastVideo page ("Pair two NVIDIA DGX Sparks",
@@ -262,7 +264,7 @@ sp_status sp_out_projection(const void *o, const void *w, const void *bias, void
  *   key cube 32*w + c; bits for cubes >= ncube are ignored.  Read only,
  *   4-byte aligned.
  * qs, ks, vs, os, lse as for sp_attention_seqsharded; D must be 128 and
- * ceil(N / 64) <= 8192 (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  Each 128-row
+ * ceil(N / 64) <= SP_SPARSE_MAX_CUBES (SP_ERR_UNSUPPORTED_D / SP_ERR_SHAPE).  Each 128-row
  * query tile (two query cubes) visits only the key cubes that one of its two
  * query cubes selects, two cubes per 128-key step: first the cubes that the
  * neighbouring tile of its CTA (the next or previous 128 rows) also visits,

@@ -141,7 +141,8 @@ def test_argument_errors_return_before_launch(lib):
     assert sparse(0) == sp.SP_ERR_NULL
     assert sparse(C + 2) == sp.SP_ERR_ALIGN
     assert sparse(C, sp.Shape(1, 1000, 4, 64, 2)) == sp.SP_ERR_UNSUPPORTED_D
-    assert sparse(C, sp.Shape(1, 64 * 8192 + 1, 1, 128, 1)) == sp.SP_ERR_SHAPE   # 8,193 cubes
+    big = sp.Shape(1, sp.SPARSE_CUBE * sp.SPARSE_MAX_CUBES + 1, 1, 128, 1)   # one cube too many
+    assert sparse(C, big) == sp.SP_ERR_SHAPE
     proj = lambda x, w, b, q, k, v, hidden, layout, shp=sp.Shape(1, 1000, 4, 128, 2): \
         lib.sp_qkv_projection(*[ctypes.c_void_p(t) if t else None for t in (x, w, b, q, k, v)],
                               hidden, layout, ctypes.byref(shp.c()), None)
@@ -250,6 +251,7 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
 int main(void) {
   sp_shape ok = {1, 75601, 40, 128, 8, 0.0f};
   sp_shape bad = {1, 1000, 40, 128, 3, 0.0f};
+  printf("%d %d ", SP_SPARSE_CUBE, SP_SPARSE_MAX_CUBES);
   printf("%lld %d %d %s\n", (long long)sp_padded_tokens(75601, 8), (int)sp_check_shape(&ok),
          (int)sp_check_shape(&bad), sp_status_str(SP_ERR_HEADS_NOT_DIVISIBLE));
   return 0;
@@ -264,6 +266,7 @@ int main(void) {
     assert r.returncode == 0, r.stderr
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stderr
-    padded, st_ok, st_bad, text = out.stdout.split(" ", 3)
+    cube, max_cubes, padded, st_ok, st_bad, text = out.stdout.split(" ", 5)
+    assert (int(cube), int(max_cubes)) == (sp.SPARSE_CUBE, sp.SPARSE_MAX_CUBES)
     assert int(padded) == 75608 and int(st_ok) == sp.SP_OK
     assert int(st_bad) == sp.SP_ERR_HEADS_NOT_DIVISIBLE and text.strip()

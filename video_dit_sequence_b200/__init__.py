@@ -471,6 +471,7 @@ def out_projection(o, w, bias, y, shape: Shape, layout: str = "seq", stream=None
 
 
 SPARSE_CUBE = 64         # SP_SPARSE_CUBE
+SPARSE_MAX_CUBES = 8192  # SP_SPARSE_MAX_CUBES: ceil(N / SPARSE_CUBE) at most
 
 
 def sparse_mask_words(mask):
@@ -494,7 +495,8 @@ def attention_sparse_seqsharded(qs, ks, vs, mask_words, os_, shape: Shape, lse=N
                                 stream=None):
     """Block-sparse fused attention: sequence-sharded bf16 qs/ks/vs/os_ as for
     attention_seqsharded, mask_words a CUDA int32/uint32 tensor
-    [B][H][ncube][nwords] (sparse_mask_words)."""
+    [B][H][ncube][nwords] (sparse_mask_words); D = 128 and ncube = ceil(N / 64)
+    <= SPARSE_MAX_CUBES."""
     torch = _torch()
     s = shape.c()
     ss = shape.seq_sharded

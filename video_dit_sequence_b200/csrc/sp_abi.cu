@@ -279,7 +279,8 @@ sp_status attention(const void *q, const void *k, const void *v, void *o, float 
   if ((f8 || mask != nullptr) && s->D != 128) return SP_ERR_UNSUPPORTED_D;
   if (mask != nullptr) {
     if ((reinterpret_cast<uintptr_t>(mask) & 3u) != 0) return SP_ERR_ALIGN;
-    if ((s->N + 63) / 64 > sp::AttnCfg<128>::kMaxPlanCubes) return SP_ERR_SHAPE;
+    static_assert(sp::AttnCfg<128>::kMaxPlanCubes == SP_SPARSE_MAX_CUBES, "plan capacity");
+    if ((s->N + SP_SPARSE_CUBE - 1) / SP_SPARSE_CUBE > SP_SPARSE_MAX_CUBES) return SP_ERR_SHAPE;
   }
   const int P = s->P, B = s->B, H = s->H, D = s->D, N = s->N;
   const int Hl = H / P;
