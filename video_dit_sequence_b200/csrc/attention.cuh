@@ -152,6 +152,35 @@ struct AttnCfg {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 
+// Rows r0 .. r0 + nrows - 1 of a K/V or Q tile in shared memory at dst take
+// tokens t0 .. t0 + nrows - 1 of the rank-major layout [P][B][nl][H][row]
+// (zeros past N), in the 128-byte-swizzled layout the TMA writes: 16-byte
+// chunk c of row r at chunk c ^ (r mod 8) of its column block.  The whole
+// warp copies with 16-byte loads, then fences the generic-proxy writes for
+// the async proxy.  Out of line: the path is rare (a tile or cube that
+// crosses a shard boundary) and each inlined copy would grow the hot code.
+// kCoherent: plain loads (data another GPU may still be writing), else
+// non-coherent ones.
+template <int kRowBytes, bool kCoherent>
+__device__ __noinline__ void copy_rows(const uint8_t *base, uint32_t dst, int t0, int r0, int nrows,
+                                       int N, int nl, int B, int b, int H, int head, int lane) {
+  constexpr int kChunks = kRowBytes / 16;  // 16-byte chunks per token row
+  constexpr int kBlockBytes = 128 * 128;
+  for (int idx = lane; idx < nrows * kChunks; idx += 32) {
+    const int r = r0 + idx / kChunks, cc = idx % kChunks;
+    const int tok = t0 + (r - r0);
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (tok < N) {
+      const int rk = tok / nl, n = tok - rk * nl;
+      const int64_t off = ((static_cast<int64_t>(rk) * B + b) * nl + n) * H * kRowBytes +
+                          static_cast<int64_t>(head) * kRowBytes + cc * 16;
+      val = kCoherent ? ld_global_v4(base + off) : ld_global_nc_v4(base + off);
+    }
+    st_shared_v4(dst + (cc >> 3) * kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4), val);
+  }
+  fence_proxy_async_smem();
+}
+
 // The kernel body.  kPeer: Q tiles come from the ranks' shards through
 // `peer` (tmQ unused) and O rows go to the ranks' output shards; K and V are
 // this rank's received head group, addressed as for the fused call.
@@ -324,26 +353,9 @@ __device__ __forceinline__ void attention_body(const CUtensorMap *tmQ, const CUt
                       b, r0, pol);
       }
     };
-    // Rows r0 .. r0 + nrows - 1 of the tile hold tokens t0 .. t0 + nrows - 1
-    // (zeros past N).
     auto copy_tile = [&](const uint8_t *base, uint32_t dst, int t0, int r0 = 0,
                          int nrows = C::kBM) {
-      constexpr int kChunks = C::kRowBytes / 16;  // 16-byte chunks per token row
-      for (int idx = lane; idx < nrows * kChunks; idx += 32) {
-        const int r = r0 + idx / kChunks, cc = idx % kChunks;
-        const int tok = t0 + (r - r0);
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (tok < p.N) {
-          const int rk = tok / nl, n = tok - rk * nl;
-          const int64_t off = ((static_cast<int64_t>(rk) * p.B + b) * nl + n) * p.H * C::kRowBytes +
-                              static_cast<int64_t>(map_head) * C::kRowBytes + cc * 16;
-          // the peer step's K/V may arrive while the kernel runs: no
-          // non-coherent loads there
-          val = kPeer ? ld_global_v4(base + off) : ld_global_nc_v4(base + off);
-        }
-        st_shared_v4(dst + (cc >> 3) * C::kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4), val);
-      }
-      fence_proxy_async_smem();
+      copy_rows<C::kRowBytes, kPeer>(base, dst, t0, r0, nrows, p.N, nl, p.B, b, p.H, map_head, lane);
     };
     // Overlapped peer step: before the first load of tokens t0 .. t1, lane 0
     // waits (bounded) until the chunk of every rank holding one of them has
