@@ -274,12 +274,10 @@ def run_ulysses(args):
     if peer:
         pr = sp.UlyssesPeerRank(shape, device=dev, kv_exchange=args.kv_exchange)
         pr.q_shard.copy_(dq)                 # Q lives in the exported shard buffer
-        q_in = pr.q_shard
 
         def step():
             out[0] = pr.step(dk, dv)
     else:
-        q_in = dq
         ur = sp.UlyssesRank(shape)           # exchange buffers reused across steps
 
         def step():
@@ -313,14 +311,42 @@ def run_ulysses(args):
     clocks = sampler.stop()
     t_max = max_over_ranks(t_ms, world, dev)
 
-    def e2e_step():
-        q_in.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        step()
-        ho.copy_(out[0], non_blocking=True)
+    # end to end: the same steps on host-resident shards through the public
+    # StepPipeline (H2D, the step and D2H on three streams); two rank objects
+    # take turns, since a rank's buffers are reused by its next step (for the
+    # peer form, other ranks write its output shard, so each step's closing
+    # all-reduce also waits for the previous output's copy back)
+    if peer:
+        e2e_ranks = [sp.UlyssesPeerRank(shape, device=dev, kv_exchange=args.kv_exchange)
+                     for _ in range(2)]
+        e2e_bufs = [(r.q_shard, torch.empty_like(dk), torch.empty_like(dv)) for r in e2e_ranks]
 
-    te = max_over_ranks(timed(e2e_step), world, dev)
+        def e2e_fn(i, t, left):
+            return e2e_ranks[i].step(t[1], t[2], release_after=left)
+    else:
+        e2e_ranks = [sp.UlyssesRank(shape) for _ in range(2)]
+        e2e_bufs = [tuple(torch.empty_like(x) for x in (dq, dk, dv)) for _ in range(2)]
+
+        def e2e_fn(i, t, left):
+            return sp.ulysses_attention_distributed(t[0], t[1], t[2], shape, a2a,
+                                                    rank=e2e_ranks[i])
+    pipe = sp.StepPipeline(e2e_bufs, e2e_fn, dev)
+    for _ in range(2):
+        pipe.submit((hq, hk, hv), ho)
+    pipe.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    a.record(pipe.h2d)
+    last = None
+    for _ in range(args.steps):
+        last = pipe.submit((hq, hk, hv), ho)
+    pipe.d2h.wait_event(last)
+    b.record(pipe.d2h)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    te = max_over_ranks(a.elapsed_time(b), world, dev)
+    pipe.synchronize()
     if sp.device_status(stream) != sp.SP_OK:
         raise SystemExit("device status not ok after the timed steps")
     pk, pkq = peaks()
@@ -340,7 +366,10 @@ def run_ulysses(args):
                                            "(CUDA IPC)") if peer else "NCCL all_to_all_single"),
                 "e2e": {"value": args.steps * flops / (te * 1e-3) / 1e12, "unit": UNIT,
                         "h2d_bytes_per_step": int(3 * shard_bytes),
-                        "d2h_bytes_per_step": int(shard_bytes)},
+                        "d2h_bytes_per_step": int(shard_bytes),
+                        "ms_per_step": te / args.steps,
+                        "how": "StepPipeline: H2D, the rank's step and D2H on three streams, "
+                               "two rank objects taking turns; every step moves its own bytes"},
                 "gpu_launches": int(launches), "clocks": clocks,
                 "roofline": {"bound": "tensor", "kernel": "whole step per GPU",
                              "achieved": per_gpu, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -350,6 +379,8 @@ def run_ulysses(args):
         print(json.dumps(line), flush=True)
     if peer:
         pr.close()
+        for r in e2e_ranks:
+            r.close()
     dist.barrier()
     dist.destroy_process_group()
     return 0

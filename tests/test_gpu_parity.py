@@ -442,6 +442,57 @@ def test_rank_classes_in_a_one_member_nccl_group(kv_exchange):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("kind", ["nccl", "peer-push", "peer-nccl"])
+def test_step_pipeline_in_a_one_member_nccl_group(kind):
+    """StepPipeline over the multi-GPU forms (two rank objects taking turns;
+    H2D, the step and D2H on three streams; the peer form's closing
+    all-reduce waits for the previous output's copy back): five steps on two
+    alternating host problems give the fused call's outputs bit for bit."""
+    import torch.distributed as dist
+    B, N, H, D = 1, 1000, 4, 128
+    shape = sp.Shape(B, N, H, D, 1)
+    probs = []
+    for seed in (81, 82):
+        q, k, v = _random_logical(B, N, H, D, seed=seed)
+        want, _ = _run_fused(q, k, v, 1)
+        host = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, 1)[0]).view(np.int16))
+                .view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+        probs.append((host, want))
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        def dev_shard():
+            return torch.empty(shape.rank_shard, dtype=torch.bfloat16, device="cuda")
+        if kind == "nccl":
+            ranks = [sp.UlyssesRank(shape) for _ in range(2)]
+            a2a = sp.nccl_all_to_all()
+            bufs = [(dev_shard(), dev_shard(), dev_shard()) for _ in range(2)]
+
+            def fn(i, t, left):
+                return sp.ulysses_attention_distributed(t[0], t[1], t[2], shape, a2a, rank=ranks[i])
+        else:
+            ranks = [sp.UlyssesPeerRank(shape, kv_exchange=kind.split("-")[1]) for _ in range(2)]
+            bufs = [(r.q_shard, dev_shard(), dev_shard()) for r in ranks]
+
+            def fn(i, t, left):
+                return ranks[i].step(t[1], t[2], release_after=left)
+        pipe = sp.StepPipeline(bufs, fn)
+        outs = [torch.empty(shape.rank_shard, dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+        for j in range(5):
+            pipe.submit(probs[j % 2][0], outs[j])
+        pipe.synchronize()
+        for j in range(5):
+            want = probs[j % 2][1]
+            got = outs[j].view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(got.reshape(want.shape), want), j
+        if kind != "nccl":
+            for r in ranks:
+                r.close()
+        _status_ok()
+    finally:
+        dist.destroy_process_group()
+
+
 def test_peer_step_writes_only_its_head_group():
     B, N, H, D, P = 1, 1000, 8, 128, 4
     q, k, v = _random_logical(B, N, H, D, seed=21)

@@ -726,7 +726,10 @@ class UlyssesPeerRank:
     all-reduce follows every rank's kernel, so when it completes here every
     row of this rank's output shard has been written and no peer still reads
     a buffer the next step overwrites.  The returned output shard stays valid
-    until the next step."""
+    until the next step.  step(..., release_after=event) makes the closing
+    all-reduce also wait (on the current stream) for that CUDA event: peers
+    write this rank's output shard in the next step only after it, so a copy
+    of the previous output that the event marks is safe (StepPipeline)."""
 
     def __init__(self, shape: Shape, group=None, backend=None, device=None,
                  kv_exchange: str = "push"):
@@ -771,7 +774,7 @@ class UlyssesPeerRank:
                 self.v_addrs.append(be.part(kv, 1, shape))
                 self.count_addrs.append(self.counts if own else be.open(*exported[2]))
 
-    def step(self, k, v, q=None):
+    def step(self, k, v, q=None, release_after=None):
         import torch.distributed as dist
         be, s = self.backend, self.shape
         if q is not None:
@@ -787,6 +790,8 @@ class UlyssesPeerRank:
             dist.all_to_all_single(self._k_recv, self._k_send, group=self.group)
             dist.all_to_all_single(self._v_recv, self._v_send, group=self.group)
             be.peer_step(self.q_addrs, self._k_recv, self._v_recv, self.o_addrs, self.rank, s)
+        if release_after is not None:
+            _torch().cuda.current_stream(self._flag.device).wait_event(release_after)
         self._flag.zero_()
         dist.all_reduce(self._flag, group=self.group)
         return self.o_shard
@@ -826,63 +831,100 @@ def ulysses_attention_distributed(q, k, v, shape: Shape, all_to_all=None, rank=N
     return rank.step(q, k, v, all_to_all)
 
 
-class HostPipeline:
-    """Fused attention on host-resident problems, with the transfers hidden
-    behind the compute.
+class StepPipeline:
+    """Steps on host-resident inputs with the transfers hidden behind the
+    compute, for any step function: one GPU's fused attention (HostPipeline)
+    or one rank's step of the multi-GPU forms (UlyssesRank, UlyssesPeerRank).
 
-    submit(hq, hk, hv, ho) takes pinned host tensors in the sequence-sharded
-    layout ([P][B][Nl][H][D] bf16) and enqueues, on three streams: the copy of
-    the inputs into one of `depth` device buffer sets, the fused attention on
-    that set, and the copy of the output back into `ho`.  A buffer set is
-    reused only after the output it held has left the device, so step i+1's
-    inputs travel while step i computes and step i's output travels while
-    step i+1 computes.  Nothing here synchronises the host; synchronize()
-    waits for everything submitted."""
+    inputs: per buffer set, the device tensors a step reads (depth =
+    len(inputs)).  step(i, tensors, previous_out_left) enqueues the step on
+    the current stream (the pipeline's compute stream) for buffer set i and
+    returns its device output, which must stay valid until the next step on
+    the same set; previous_out_left is the CUDA event that marks the previous
+    step's output as copied back (None for the first), which a step whose
+    output buffers other ranks write passes on (UlyssesPeerRank's
+    release_after).  submit(host_inputs, host_output) copies the pinned host
+    tensors into the next set on an H2D stream, runs the step once they have
+    arrived, and copies its output into host_output on a D2H stream.  A set
+    is reused only after its last output has left, so step i+1's inputs
+    travel while step i computes and step i's output travels while step i+1
+    computes.  Nothing here synchronises the host; synchronize() waits for
+    everything submitted.  Collectives inside the step run on the compute
+    stream, in submission order on every rank."""
 
-    def __init__(self, shape: Shape, device=None, depth: int = 2):
+    def __init__(self, inputs, step, device=None):
         torch = _torch()
-        self.shape = shape
-        self.device = torch.device(device or "cuda")
+        self.inputs = [tuple(t) for t in inputs]
+        self.step = step
+        self.device = torch.device(device or self.inputs[0][0].device)
         self.h2d = torch.cuda.Stream(self.device)
         self.compute = torch.cuda.Stream(self.device)
         self.d2h = torch.cuda.Stream(self.device)
-        ss = shape.seq_sharded
-        self.sets = [tuple(torch.empty(ss, dtype=torch.bfloat16, device=self.device)
-                           for _ in range(4)) for _ in range(depth)]
-        self.freed = [None] * depth     # event: the set's last output has left
+        self.freed = [None] * len(self.inputs)   # event: the set's last output has left
+        self.last_out_left = None
         self.count = 0
 
-    def submit(self, hq, hk, hv, ho):
+    def submit(self, host_inputs, host_output):
         torch = _torch()
-        i = self.count % len(self.sets)
+        i = self.count % len(self.inputs)
         self.count += 1
-        dq, dk, dv, do = self.sets[i]
+        dev = self.inputs[i]
+        if len(host_inputs) != len(dev):
+            raise ValueError(f"{len(host_inputs)} host inputs for {len(dev)} device buffers")
         if self.freed[i] is not None:
             self.h2d.wait_event(self.freed[i])
         with torch.cuda.stream(self.h2d):
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
+            for d, h in zip(dev, host_inputs):
+                d.copy_(h, non_blocking=True)
         arrived = torch.cuda.Event()
         arrived.record(self.h2d)
         self.compute.wait_event(arrived)
-        attention_seqsharded(dq, dk, dv, do, self.shape, stream=self.compute)
+        with torch.cuda.stream(self.compute):
+            out = self.step(i, dev, self.last_out_left)
         done = torch.cuda.Event()
         done.record(self.compute)
         self.d2h.wait_event(done)
         with torch.cuda.stream(self.d2h):
-            ho.copy_(do, non_blocking=True)
-        freed = torch.cuda.Event()
-        freed.record(self.d2h)
-        self.freed[i] = freed
-        return freed
+            host_output.copy_(out, non_blocking=True)
+        left = torch.cuda.Event()
+        left.record(self.d2h)
+        self.freed[i] = self.last_out_left = left
+        return left
 
     def synchronize(self):
         """Waits for everything submitted, then checks the device status word
         (raises SpError when a kernel gave up on a bounded wait)."""
         for st in (self.h2d, self.compute, self.d2h):
             st.synchronize()
-        _check(device_status(self.compute), "HostPipeline")
+        _check(device_status(self.compute), "StepPipeline")
+
+
+class HostPipeline(StepPipeline):
+    """Fused attention on host-resident problems, with the transfers hidden
+    behind the compute (a StepPipeline over sp_attention_seqsharded).
+
+    submit(hq, hk, hv, ho) takes pinned host tensors in the sequence-sharded
+    layout ([P][B][Nl][H][D] bf16) and enqueues, on three streams: the copy of
+    the inputs into one of `depth` device buffer sets, the fused attention on
+    that set, and the copy of the output back into `ho`."""
+
+    def __init__(self, shape: Shape, device=None, depth: int = 2):
+        torch = _torch()
+        self.shape = shape
+        dev = torch.device(device or "cuda")
+        ss = shape.seq_sharded
+        sets = [tuple(torch.empty(ss, dtype=torch.bfloat16, device=dev) for _ in range(4))
+                for _ in range(depth)]
+        self._outs = [st[3] for st in sets]
+
+        def fused(i, t, _left):
+            attention_seqsharded(t[0], t[1], t[2], self._outs[i], shape,
+                                 stream=torch.cuda.current_stream(dev))
+            return self._outs[i]
+        super().__init__([st[:3] for st in sets], fused, dev)
+
+    def submit(self, hq, hk, hv, ho):
+        return super().submit((hq, hk, hv), ho)
 
 
 def device_status(stream=None, device=None) -> int:
