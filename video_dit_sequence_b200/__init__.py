@@ -839,8 +839,9 @@ class StepPipeline:
     inputs: per buffer set, the device tensors a step reads (depth =
     len(inputs)).  step(i, tensors, previous_out_left) enqueues the step on
     the current stream (the pipeline's compute stream) for buffer set i and
-    returns its device output, which must stay valid until the next step on
-    the same set; previous_out_left is the CUDA event that marks the previous
+    returns its device output: a buffer of its own that stays valid until the
+    next step on the same set, or a fresh tensor; previous_out_left is the
+    CUDA event that marks the previous
     step's output as copied back (None for the first), which a step whose
     output buffers other ranks write passes on (UlyssesPeerRank's
     release_after).  submit(host_inputs, host_output) copies the pinned host
@@ -886,6 +887,7 @@ class StepPipeline:
         self.d2h.wait_event(done)
         with torch.cuda.stream(self.d2h):
             host_output.copy_(out, non_blocking=True)
+        out.record_stream(self.d2h)   # a fresh output stays allocated until it has left
         left = torch.cuda.Event()
         left.record(self.d2h)
         self.freed[i] = self.last_out_left = left
