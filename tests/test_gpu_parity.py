@@ -651,6 +651,30 @@ def test_sparse_against_oracle(B, N, H, P, density, group):
     print(f"sparse B={B} N={N} P={P} density={density}: {m}, nc={nc}")
 
 
+@pytest.mark.parametrize("N,P", [(1, 1), (50, 1), (65, 2), (129, 3)])
+def test_sparse_tiny_sequences(N, P):
+    """One to three cubes (the only CTA's second query tile has nothing to
+    walk when N <= 128; partial last cubes): a full mask equals the dense
+    call bit for bit, a random mask matches the masked oracle on every row."""
+    B, H, D = 1, 2, 128
+    q, k, v = _random_logical(B, N, H, D, seed=97 + N)
+    nc = -(-N // 64)
+    full = np.ones((B, H, nc, nc), bool)
+    got, lg = _run_sparse(q, k, v, full, P, lse=True)
+    want, lw = _run_fused(q, k, v, P, lse=True)
+    assert np.array_equal(got, want)
+    assert np.array_equal(lg, lw)
+    mask = np.random.default_rng(N).random((B, H, nc, nc)) < 0.6
+    mask[..., 0] = True                                  # every query cube selects something
+    got, lse = _run_sparse(q, k, v, mask, P, lse=True)
+    rows = _rows_all(B, N, H)
+    O = synth.from_seq_shards(got.reshape(P, B, -1, H, D), N)
+    ref, lref = oracle.attention_rows_masked(q, k, v, mask, rows)
+    assert_parity(compare(O[rows[:, 0], rows[:, 2], rows[:, 1]], ref, rows[:, 1]),
+                  f"sparse tiny N={N}")
+    assert np.max(np.abs(lse[rows[:, 0], rows[:, 1], rows[:, 2]] - lref)) < 2e-2
+
+
 def test_sparse_cta_with_no_selected_tile():
     """Query cubes 4..7 (one CTA's 256 rows) select nothing: that CTA visits
     no key tile and writes zero rows; bits past the last cube are ignored."""
