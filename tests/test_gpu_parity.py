@@ -816,7 +816,8 @@ def _check_proj(seq, x, w, b, rows, where):
 
 @pytest.mark.parametrize("B,N,H,D,P,hidden,bias", [
     (1, 1000, 4, 128, 2, 512, True), (2, 333, 6, 64, 3, 200, False),
-    (1, 4096, 12, 128, 4, 1536, True), (3, 130, 2, 64, 1, 72, True)])
+    (1, 4096, 12, 128, 4, 1536, True), (3, 130, 2, 64, 1, 72, True),
+    (1, 1, 2, 64, 1, 64, True)])
 def test_qkv_projection_layouts(B, N, H, D, P, hidden, bias):
     """The projection against the fp64 oracle on every row, and its three
     layouts bit for bit against the pinned pack and exchange pack of the
@@ -888,7 +889,7 @@ def _check_oproj(y, o_seq, w, b, rows, where):
 @pytest.mark.parametrize("B,N,H,D,P,hidden,bias", [
     (1, 1000, 4, 128, 2, 512, True), (2, 333, 6, 64, 3, 200, False),
     (1, 4096, 12, 128, 4, 1536, True), (3, 130, 2, 64, 1, 72, True),
-    (2, 517, 8, 128, 8, 264, True)])
+    (2, 517, 8, 128, 8, 264, True), (1, 1, 2, 64, 1, 8, False)])
 def test_out_projection_layouts(B, N, H, D, P, hidden, bias):
     """The output projection against the fp64 oracle on every row, reading O
     as sequence shards; reading O as head groups (the pinned pack of it) and,
@@ -1278,7 +1279,7 @@ def _check_fp8(out, q8, k8, v8, f, rows, P, where):
 
 
 @pytest.mark.parametrize("B,N,H,P", [(1, 1024, 4, 2), (1, 3000, 8, 4), (2, 1000, 8, 4),
-                                     (1, 257, 2, 1)])
+                                     (1, 257, 2, 1), (1, 1, 2, 1), (1, 100, 2, 2)])
 def test_fp8_attention_against_oracle(B, N, H, P):
     q8, k8, v8, d = _fp8_inputs(B, N, H, 128, seed=40 + N)
     out, lse = _run_fp8(q8, k8, v8, d, P, lse=True)
