@@ -628,8 +628,10 @@ def run_ours(args):
         e2e = {"value": weak_scaling_value(world, args.steps, flops, te), "unit": UNIT,
                "h2d_bytes_per_step": int(3 * tensor_bytes), "d2h_bytes_per_step": int(tensor_bytes),
                "ms_per_step": te / args.steps,
-               "how": "HostPipeline: H2D, fused attention and D2H on three streams, "
-                      "two device buffer sets; every step moves its own bytes"}
+               "how": f"HostPipeline: H2D, fused attention and D2H on three streams, "
+                      f"two device buffer sets, each step as {pipe.head_groups} groups of "
+                      f"{pipe.group_shape.H} heads (copied in, attended and copied out one "
+                      f"group at a time); every step moves its own bytes"}
         if sp.device_status(stream) != sp.SP_OK:
             raise SystemExit("device status not ok after e2e")
 

@@ -395,6 +395,23 @@ sp_status sp_ipc_open(const void *handle, void **base_out);
 /* Unmaps an allocation mapped by sp_ipc_open. */
 sp_status sp_ipc_close(void *base);
 
+/* Head-slice copy, for pipelines that move a problem between host and device
+ * one group of heads at a time (heads are independent, so a group of Hg
+ * heads with P | Hg is a problem of its own): for every row r < rows and
+ * head h < nh,
+ *   dst[r][dst_h0 + h][0 .. D-1] = src[r][src_h0 + h][0 .. D-1]
+ * where a dst row holds dst_heads and a src row src_heads heads of D bf16
+ * elements (rows = P*B*Nl for the sequence-sharded layout).  dst and src are
+ * each device memory or page-locked host memory; the direction follows from
+ * the pointers (unified addressing).  Enqueues one strided copy on `stream`
+ * and no kernel; rows == 0 enqueues nothing.  Bit-exact.  Errors: SP_ERR_NULL;
+ * SP_ERR_SHAPE when rows < 0, nh < 1, D < 1, a slice reaches past its row
+ * (h0 < 0 or h0 + nh > heads) or a row is 2^31 bytes or more; SP_ERR_CUDA
+ * when the copy cannot be enqueued. */
+sp_status sp_copy_heads(void *dst, int32_t dst_heads, int32_t dst_h0, const void *src,
+                        int32_t src_heads, int32_t src_h0, int64_t rows, int32_t nh,
+                        int32_t D, void *stream);
+
 /* Takes the device status word of the current device and clears it in one
  * atomic exchange enqueued on `stream`, then synchronises `stream` and
  * returns what it took: SP_ERR_TIMEOUT if a kernel gave up on a bounded wait

@@ -215,7 +215,36 @@ def test_argument_errors_return_before_launch(lib):
         assert _call(fn, 0, B_, shape=shape) == sp.SP_ERR_NULL
         assert _call(fn, A + 8, B_, shape=shape) == sp.SP_ERR_ALIGN
         assert _call(fn, A, B_, shape=bad) == sp.SP_ERR_HEADS_NOT_DIVISIBLE
+    vp = ctypes.c_void_p
+    cp = lambda d, dh, d0, s, sh, s0, rows, nh, D: lib.sp_copy_heads(
+        vp(d) if d else None, dh, d0, vp(s) if s else None, sh, s0, rows, nh, D, None)
+    assert cp(0, 8, 0, A, 40, 0, 10, 8, 128) == sp.SP_ERR_NULL
+    assert cp(A, 8, 0, 0, 40, 0, 10, 8, 128) == sp.SP_ERR_NULL
+    assert cp(A, 8, 1, B_, 40, 0, 10, 8, 128) == sp.SP_ERR_SHAPE     # past the dst row
+    assert cp(A, 8, 0, B_, 40, 33, 10, 8, 128) == sp.SP_ERR_SHAPE    # past the src row
+    assert cp(A, 8, -1, B_, 40, 0, 10, 8, 128) == sp.SP_ERR_SHAPE
+    assert cp(A, 8, 0, B_, 40, 0, -1, 8, 128) == sp.SP_ERR_SHAPE
+    assert cp(A, 8, 0, B_, 40, 0, 10, 0, 128) == sp.SP_ERR_SHAPE
+    assert cp(A, 8, 0, B_, 40, 0, 10, 8, 0) == sp.SP_ERR_SHAPE
+    assert cp(A, 1 << 23, 0, B_, 40, 0, 10, 8, 128) == sp.SP_ERR_SHAPE  # a 2 GiB row
+    assert cp(A, 8, 0, B_, 40, 32, 0, 8, 128) == sp.SP_OK           # no rows: nothing enqueued
     assert lib.sp_launch_count() == 0
+
+
+def test_pipeline_head_groups():
+    """HostPipeline's head groups: P divides every group, and the groups'
+    calls launch no more waves of 148 CTAs than one call over all heads."""
+    g = sp.pipeline_head_groups
+    assert g(sp.Shape(1, 75600, 40, 128, 4)) == 5      # 8 heads a group, 16 waves each
+    assert g(sp.Shape(1, 32760, 12, 128, 2)) == 1      # 11 waves: any split adds one
+    assert g(sp.Shape(1, 124992, 48, 128, 8)) == 3
+    assert g(sp.Shape(1, 1000, 7, 64, 7)) == 1
+    for H, P, N, B in ((40, 4, 75600, 1), (24, 2, 4096, 2), (16, 1, 65536, 1), (64, 8, 99999, 1)):
+        shp = sp.Shape(B, N, H, 128, P)
+        G = g(shp)
+        assert 1 <= G <= 8 and H % G == 0 and (H // G) % P == 0
+        per_head = -(-shp.Np // 256) * B
+        assert G * -(-(H // G) * per_head // 148) <= -(-H * per_head // 148)
 
 
 def test_binding_refuses_cpu_tensors(lib):

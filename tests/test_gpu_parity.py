@@ -1146,6 +1146,56 @@ def test_host_pipeline_matches_direct_calls():
         assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
 
 
+@pytest.mark.parametrize("groups", [1, 2, 4])
+def test_host_pipeline_in_head_groups(groups):
+    """HostPipeline moving and attending one group of heads at a time
+    (sp_copy_heads in and out, one fused call of H/G heads per group): five
+    problems through two buffer sets, each bit-identical to the direct call
+    over all H heads."""
+    B, N, H, D, P = 1, 1100, 8, 128, 2
+    shape = sp.Shape(B, N, H, D, P)
+    pipe = sp.HostPipeline(shape, depth=2, head_groups=groups)
+    assert pipe.head_groups == groups
+    outs, wants = [], []
+    for i in range(5):
+        q, k, v = _random_logical(B, N, H, D, seed=520 + i)
+        host = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, P)).view(np.int16))
+                .view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+        ho = torch.full(shape.seq_sharded, float("nan"), dtype=torch.bfloat16).pin_memory()
+        pipe.submit(*host, ho)
+        outs.append(ho)
+        wants.append(_run_fused(q, k, v, P)[0])
+    pipe.synchronize()
+    _status_ok()
+    for got, want in zip(outs, wants):
+        assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
+
+
+def test_copy_heads_between_host_and_device():
+    """sp_copy_heads: a head slice of pinned host rows into a device array of
+    fewer heads, a device slice into another device array, and back into the
+    host rows; copied elements bit-exact, all others untouched."""
+    rows, H, D = 777, 12, 64
+    g = torch.Generator().manual_seed(7)
+    host = torch.randn(rows, H, D, generator=g).to(torch.bfloat16).pin_memory()
+    dev = torch.full((rows, 5, D), 3.0, dtype=torch.bfloat16, device="cuda")
+    sp.copy_heads(dev, 5, 1, host, H, 6, rows, 4, D)           # heads 6..9 -> 1..4
+    dev2 = torch.zeros((rows, 4, D), dtype=torch.bfloat16, device="cuda")
+    sp.copy_heads(dev2, 4, 0, dev, 5, 1, rows, 4, D)           # device to device
+    back = torch.full((rows, H, D), -1.0, dtype=torch.bfloat16).pin_memory()
+    sp.copy_heads(back, H, 2, dev2, 4, 0, rows, 4, D)          # -> heads 2..5
+    torch.cuda.synchronize()
+    got = dev.cpu()
+    assert torch.equal(got[:, 1:5].view(torch.int16), host[:, 6:10].view(torch.int16))
+    assert bool((got[:, 0] == 3.0).all())
+    assert torch.equal(back[:, 2:6].view(torch.int16), host[:, 6:10].view(torch.int16))
+    assert bool((back[:, :2] == -1.0).all()) and bool((back[:, 6:] == -1.0).all())
+    with pytest.raises(ValueError):
+        sp.copy_heads(dev, 5, 0, torch.zeros(rows, H, D, dtype=torch.bfloat16), H, 0, rows, 4, D)
+    with pytest.raises(sp.SpError):
+        sp.copy_heads(dev, 5, 2, host, H, 0, rows, 4, D)       # past the device row
+
+
 C_PROGRAM = r"""
 /* The fused call from a C program: device memory from the CUDA runtime, the
  * computation through sp.h, no Python or torch on the path. */

@@ -44,7 +44,8 @@ EXPORTED = ("sp_padded_tokens", "sp_check_shape", "sp_pack", "sp_unpack",
             "sp_exchange_pack", "sp_exchange_unpack", "sp_attention_fp8_seqsharded",
             "sp_attention_ulysses_peer", "sp_ipc_export", "sp_ipc_open", "sp_ipc_close",
             "sp_attention_sparse_seqsharded", "sp_qkv_projection", "sp_out_projection",
-            "sp_exchange_push", "sp_attention_ulysses_overlap", "sp_shard", "sp_unshard")
+            "sp_exchange_push", "sp_attention_ulysses_overlap", "sp_shard", "sp_unshard",
+            "sp_copy_heads")
 
 
 class sp_shape(ctypes.Structure):
@@ -109,6 +110,10 @@ def load(path: str = LIB_PATH):
     lib.sp_ipc_open.restype = ctypes.c_int
     lib.sp_ipc_close.argtypes = [vp]
     lib.sp_ipc_close.restype = ctypes.c_int
+    lib.sp_copy_heads.argtypes = [vp, ctypes.c_int32, ctypes.c_int32, vp, ctypes.c_int32,
+                                  ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                  vp]
+    lib.sp_copy_heads.restype = ctypes.c_int
     lib.sp_device_status.argtypes = [vp]
     lib.sp_device_status.restype = ctypes.c_int
     lib.sp_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
@@ -275,6 +280,32 @@ def unshard(xs, x, shape: Shape, stream=None):
         _check(load().sp_unshard(_ptr(xs, shape.seq_sharded, "xs"),
                                  _ptr(x, (shape.B, shape.N, shape.H, shape.D), "x"),
                                  ctypes.byref(s), _stream(stream, xs.device)), "sp_unshard")
+
+
+def copy_heads(dst, dst_heads: int, dst_h0: int, src, src_heads: int, src_h0: int, rows: int,
+               nh: int, D: int, stream=None):
+    """dst[r][dst_h0 + h] = src[r][src_h0 + h] for rows r and heads h < nh
+    (D bf16 elements per head): one strided copy between pinned host memory
+    and the device, or within the device, enqueued on `stream`."""
+    torch = _torch()
+    ptrs, devs = [], set()
+    for t, heads, name in ((dst, dst_heads, "dst"), (src, src_heads, "src")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bf16 tensor")
+        if not t.is_contiguous() or t.numel() != rows * heads * D:
+            raise ValueError(f"{name} must be contiguous with {rows} x {heads} x {D} elements")
+        if t.is_cuda:
+            devs.add(t.device)
+        elif not t.is_pinned():
+            raise ValueError(f"{name} is host memory that is not page-locked")
+        ptrs.append(ctypes.c_void_p(t.data_ptr()))
+    if len(devs) != 1:
+        raise ValueError("copy_heads needs exactly one CUDA device among its tensors")
+    dev = devs.pop()
+    with torch.cuda.device(dev):
+        _check(load().sp_copy_heads(ptrs[0], int(dst_heads), int(dst_h0), ptrs[1],
+                                    int(src_heads), int(src_h0), int(rows), int(nh), int(D),
+                                    _stream(stream, dev)), "sp_copy_heads")
 
 
 def pack(xs, xh, shape: Shape, stream=None):
@@ -901,6 +932,21 @@ class StepPipeline:
         _check(device_status(self.compute), "StepPipeline")
 
 
+def pipeline_head_groups(shape: Shape, sms: int = 148, max_groups: int = 8) -> int:
+    """Head groups per step for HostPipeline: the largest G <= max_groups
+    with P | H/G whose G fused calls of H/G heads run no more waves than one
+    call over all H heads (the fused kernel keeps one CTA on each of `sms`
+    SMs and launches ceil(Np/256) * B CTAs per head)."""
+    per_head = -(-shape.Np // 256) * shape.B
+    one = -(-shape.H * per_head // sms)
+    best = 1
+    for g in range(2, max_groups + 1):
+        if shape.H % g == 0 and (shape.H // g) % shape.P == 0 and \
+                g * -(-(shape.H // g) * per_head // sms) <= one:
+            best = g
+    return best
+
+
 class HostPipeline(StepPipeline):
     """Fused attention on host-resident problems, with the transfers hidden
     behind the compute (a StepPipeline over sp_attention_seqsharded).
@@ -908,25 +954,72 @@ class HostPipeline(StepPipeline):
     submit(hq, hk, hv, ho) takes pinned host tensors in the sequence-sharded
     layout ([P][B][Nl][H][D] bf16) and enqueues, on three streams: the copy of
     the inputs into one of `depth` device buffer sets, the fused attention on
-    that set, and the copy of the output back into `ho`."""
+    that set, and the copy of the output back into `ho`.
 
-    def __init__(self, shape: Shape, device=None, depth: int = 2):
+    Heads are independent, so a step runs as `head_groups` problems of H/G
+    heads each (P | H/G; default pipeline_head_groups): group g's inputs are
+    copied in (sp_copy_heads), attended and copied out while the other groups'
+    copies run, so that only one group's input and output transfers lie
+    outside the compute of a run of steps instead of the whole step's.  Each
+    group's output is bit-identical to the same heads of one call over all H."""
+
+    def __init__(self, shape: Shape, device=None, depth: int = 2, head_groups: int = 0):
         torch = _torch()
         self.shape = shape
         dev = torch.device(device or "cuda")
-        ss = shape.seq_sharded
-        sets = [tuple(torch.empty(ss, dtype=torch.bfloat16, device=dev) for _ in range(4))
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        g = int(head_groups) or pipeline_head_groups(
+            shape, torch.cuda.get_device_properties(dev).multi_processor_count)
+        if g < 1 or shape.H % g or (shape.H // g) % shape.P:
+            raise ValueError(f"{g} head groups: need G | H and P | H/G "
+                             f"(H = {shape.H}, P = {shape.P})")
+        self.head_groups = g
+        self.group_shape = Shape(shape.B, shape.N, shape.H // g, shape.D, shape.P, shape.scale)
+        gs = (g,) + self.group_shape.seq_sharded
+        sets = [tuple(torch.empty(gs, dtype=torch.bfloat16, device=dev) for _ in range(4))
                 for _ in range(depth)]
         self._outs = [st[3] for st in sets]
+        # per buffer set and group: the event that marks its output as copied back
+        self._group_freed = [[None] * g for _ in range(depth)]
 
         def fused(i, t, _left):
-            attention_seqsharded(t[0], t[1], t[2], self._outs[i], shape,
+            attention_seqsharded(t[0], t[1], t[2], self._outs[i][0], shape,
                                  stream=torch.cuda.current_stream(dev))
-            return self._outs[i]
-        super().__init__([st[:3] for st in sets], fused, dev)
+            return self._outs[i][0]
+        # the whole-step path (one group) sees each set as its [P][B][Nl][H][D] views
+        super().__init__([tuple(x[0] if g == 1 else x for x in st[:3]) for st in sets],
+                         fused, dev)
 
     def submit(self, hq, hk, hv, ho):
-        return super().submit((hq, hk, hv), ho)
+        if self.head_groups == 1:
+            return super().submit((hq, hk, hv), ho)
+        torch = _torch()
+        i = self.count % len(self.inputs)
+        self.count += 1
+        q, k, v = self.inputs[i]
+        o = self._outs[i]
+        sh, gs = self.shape, self.group_shape
+        rows, hg = sh.P * sh.B * sh.Nl, gs.H
+        left = None
+        for g in range(self.head_groups):
+            if self._group_freed[i][g] is not None:
+                self.h2d.wait_event(self._group_freed[i][g])
+            for d, h in ((q, hq), (k, hk), (v, hv)):
+                copy_heads(d[g], hg, 0, h, sh.H, g * hg, rows, hg, sh.D, stream=self.h2d)
+            arrived = torch.cuda.Event()
+            arrived.record(self.h2d)
+            self.compute.wait_event(arrived)
+            attention_seqsharded(q[g], k[g], v[g], o[g], gs, stream=self.compute)
+            done = torch.cuda.Event()
+            done.record(self.compute)
+            self.d2h.wait_event(done)
+            copy_heads(ho, sh.H, g * hg, o[g], hg, 0, rows, hg, sh.D, stream=self.d2h)
+            left = torch.cuda.Event()
+            left.record(self.d2h)
+            self._group_freed[i][g] = left
+        self.freed[i] = self.last_out_left = left
+        return left
 
 
 def device_status(stream=None, device=None) -> int:

@@ -911,6 +911,29 @@ sp_status sp_ipc_close(void *base) {
   return cudaIpcCloseMemHandle(base) == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
 
+sp_status sp_copy_heads(void *dst, int32_t dst_heads, int32_t dst_h0, const void *src,
+                        int32_t src_heads, int32_t src_h0, int64_t rows, int32_t nh,
+                        int32_t D, void *stream) {
+  if (dst == nullptr || src == nullptr) return SP_ERR_NULL;
+  if (rows < 0 || nh < 1 || D < 1 || dst_h0 < 0 || src_h0 < 0 ||
+      static_cast<int64_t>(dst_h0) + nh > dst_heads || static_cast<int64_t>(src_h0) + nh > src_heads)
+    return SP_ERR_SHAPE;
+  const int64_t elt = sizeof(__nv_bfloat16);
+  const int64_t dpitch = static_cast<int64_t>(dst_heads) * D * elt;
+  const int64_t spitch = static_cast<int64_t>(src_heads) * D * elt;
+  if (dpitch >= (int64_t{1} << 31) || spitch >= (int64_t{1} << 31)) return SP_ERR_SHAPE;
+  if (rows == 0) return SP_OK;
+  NvtxRange range("sp_copy_heads");
+  char *d = static_cast<char *>(dst) + static_cast<int64_t>(dst_h0) * D * elt;
+  const char *s = static_cast<const char *>(src) + static_cast<int64_t>(src_h0) * D * elt;
+  const cudaError_t e = cudaMemcpy2DAsync(d, static_cast<size_t>(dpitch), s,
+                                          static_cast<size_t>(spitch),
+                                          static_cast<size_t>(nh) * D * elt,
+                                          static_cast<size_t>(rows), cudaMemcpyDefault,
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
 sp_status sp_device_status(void *stream) {
   NvtxRange range("sp_device_status");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
