@@ -504,6 +504,24 @@ bool make_map_matrix(CUtensorMap *m, const void *base, int cols, int rows, int b
 sp_status launch_projection(const CUtensorMap &ma, const void *w, int slots, sp::ProjParams p,
                             void *stream);
 
+// Destination map of the projection epilogue's TMA stores: [Z][rows][W] bf16
+// (W features a row), boxes of 32 rows x 32 features whose 64-byte rows the
+// 64-byte swizzle spreads over the shared-memory banks.
+bool make_map_out(CUtensorMap *m, void *base, int64_t W, int64_t rows, int64_t Z) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t row = static_cast<cuuint64_t>(W) * 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(W), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(Z)};
+  cuuint64_t strides[2] = {row, row * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q, void *k,
                          void *v, int32_t hidden, int32_t layout, const sp_shape *s,
                          void *stream) {
@@ -547,6 +565,9 @@ sp_status qkv_projection(const void *x, const void *w, const void *bias, void *q
   p.status = status;
   p.a_load = sp::kALoadMatrix;
   p.rows_per_slot = p.M;
+  // a tile's rows are consecutive destination rows except in the head-sharded
+  // layout, whose rows jump between token shards and batch entries
+  p.tma_store = layout != SP_QKV_HEAD_SHARDED;
   return launch_projection(mx, w, 1, p, stream);
 }
 
@@ -629,25 +650,39 @@ sp_status out_projection(const void *o, const void *w, const void *bias, void *y
   p.a_cols = static_cast<int32_t>(gcols);
   p.out_proj = 1;
   p.y = static_cast<__nv_bfloat16 *>(y);
+  // with head groups and B > 1 a slot's rows are every B-th run of Nl rows
+  p.tma_store = layout != SP_O_HEAD_SHARDED || B == 1;
   p.bias = static_cast<const __nv_bfloat16 *>(bias);
   p.status = status;
   return launch_projection(ma, w, slots, p, stream);
 }
 
-// Both projections: the tile counts for 256-row blocks, the map over w (a
-// box of 128 rows: each CTA of a pair holds half of a tile's features), and
+// Both projections: the tile counts for 256-row, 512-feature tiles, the map
+// over w (a box of 128 rows: each CTA of a pair holds half of each 256-feature
+// half of a tile), and
 // the persistent launch on CTA pairs.  p holds every other field,
 // rows_per_slot included.
 sp_status launch_projection(const CUtensorMap &ma, const void *w, int slots, sp::ProjParams p,
                             void *stream) {
   p.tiles_per_slot = (p.rows_per_slot + sp::kPairBM - 1) / sp::kPairBM;
   const int64_t tiles_m = static_cast<int64_t>(p.tiles_per_slot) * slots;
-  p.tiles_n = (p.nout + sp::kProjBN - 1) / sp::kProjBN;
+  p.tiles_n = (p.nout + sp::kPairTileN - 1) / sp::kPairTileN;
   const int64_t tiles = tiles_m * p.tiles_n;
   if (tiles >= (int64_t(1) << 31)) return SP_ERR_SHAPE;
   p.tiles_m = static_cast<int32_t>(tiles_m);
   CUtensorMap mw;
   if (!make_map_matrix(&mw, w, p.K, p.nout, 128)) return SP_ERR_CUDA;
+  CUtensorMap my[3] = {mw, mw, mw};   // unused unless the epilogue stores through TMA
+  if (p.tma_store) {
+    if (p.out_proj) {
+      if (!make_map_out(&my[0], p.y, p.nout, p.M, 1)) return SP_ERR_CUDA;
+    } else {
+      const bool send = p.layout == sp::kProjSendChunks;
+      const int64_t W = static_cast<int64_t>(send ? p.Hl : p.H) * p.D;
+      for (int t = 0; t < 3; ++t)
+        if (!make_map_out(&my[t], p.out[t], W, p.M, send ? p.P : 1)) return SP_ERR_CUDA;
+    }
+  }
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
@@ -688,7 +723,7 @@ sp_status launch_projection(const CUtensorMap &ma, const void *w, int slots, sp:
   }
   const int64_t pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cudaError_t e = cudaLaunchKernelEx(&cfg, sp::projection_pair_kernel, ma, mw, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, sp::projection_pair_kernel, ma, mw, my[0], my[1], my[2], p);
   return launch_status(e == cudaSuccess ? cudaGetLastError() : e);
 }
 
