@@ -989,6 +989,21 @@ def test_outputs_stay_inside_their_buffers():
         y, c = _guarded(tuple(rows) + (hidden,), torch.bfloat16); checks.append(c)
         sp.out_projection(src, wo, bo, y, shape, layout=layout)
 
+    # the q, k, v projection into each layout (TMA-stored sequence shards and
+    # send chunks, 16-byte stores for head groups; hidden 200)
+    hin = 200
+    xs = to_dev(synth.normal_bf16(44, 0, 0, P * B * shape.Nl * hin).reshape(P, B, shape.Nl, hin))
+    wq = to_dev(synth.normal_bf16(44, 1, 0, 3 * H * D * hin, mul=0.07).reshape(3 * H * D, hin))
+    bq = to_dev(synth.normal_bf16(44, 2, 0, 3 * H * D, mul=0.1))
+    for layout, src, oshape in (("seq", xs, shape.seq_sharded), ("head", xs, shape.head_sharded),
+                                ("send", xs[1].contiguous(), shape.send_chunks)):
+        outs = []
+        for _ in range(3):
+            o, c = _guarded(oshape, torch.bfloat16)
+            checks.append(c)
+            outs.append(o)
+        sp.qkv_projection(src, wq, bq, *outs, shape, layout=layout)
+
     q8, k8, v8, f = _fp8_inputs(B, N, H, D, seed=41)
     dev8 = [torch.from_numpy(np.ascontiguousarray(synth.to_seq_shards(x, P))).cuda()
             for x in (q8, k8, v8)]
