@@ -36,17 +36,17 @@
 // (x is read once per 512 features instead of per 256); against one CTA per
 // 128 x 256 tile, half as much.  Each CTA's loads complete on its own
 // barrier; the odd CTA forwards that completion to the even one with a
-// remote mbarrier arrive (no multicast; the plain arrive form, whose release
-// is CTA-scoped: a cluster-scoped release per 512-cycle stage cost half the
-// throughput).  Eight epilogue warps per CTA (two per TMEM lane quarter) add
-// the bias, round to bf16 and write 32 x 32 chunks through shared memory and
-// TMA stores (where a tile's rows are consecutive destination rows; else
-// 16-byte stores per row).  The two halves of a tile fill the tensor memory;
-// the MMA thread staggers them at the ends of each tile so that one half
-// drains while the other's MMAs run (see the kernel).  The kernel is
-// persistent, one pair per two SMs; tiles run in groups of kProjGroupN
-// column blocks so that the pairs working at one time share their w slice in
-// L2.
+// remote mbarrier arrive (each CTA loads only its own operands; the plain
+// arrive form, whose release is CTA-scoped: a cluster-scoped release per
+// 512-cycle stage cost half the throughput).  Eight epilogue warps per CTA
+// (two per TMEM lane quarter) add the bias, round to bf16 and write 32 x 32
+// chunks through shared memory and TMA stores (where a tile's rows are
+// consecutive destination rows; else 16-byte stores per row).  The two
+// halves of a tile fill the tensor memory; the MMA thread staggers them at
+// the ends of each tile so that one half drains while the other's MMAs run
+// (see the kernel).  The kernel is persistent, one pair per two SMs; tiles
+// run in groups of kProjGroupN column blocks so that the pairs working at
+// one time share their w slice in L2.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
