@@ -323,14 +323,22 @@ def run_ulysses(args):
 
         def e2e_fn(i, t, left):
             return e2e_ranks[i].step(t[1], t[2], release_after=left)
+        groups = 1
     else:
-        e2e_ranks = [sp.UlyssesRank(shape) for _ in range(2)]
-        e2e_bufs = [tuple(torch.empty_like(x) for x in (dq, dk, dv)) for _ in range(2)]
+        # the all-to-all form in head groups: each group of H/G heads is a
+        # Ulysses step of its own, with a rank object per buffer set and group
+        groups = sp.pipeline_head_groups(
+            shape, torch.cuda.get_device_properties(dev).multi_processor_count, gpus=world)
+        gshape = sp.Shape(shape.B, shape.N, shape.H // groups, shape.D, shape.P, shape.scale)
+        e2e_ranks = [sp.UlyssesRank(gshape) for _ in range(2 * groups)]
+        part = ((groups,) if groups > 1 else ()) + gshape.rank_shard
+        e2e_bufs = [tuple(torch.empty(part, dtype=torch.bfloat16, device=dev) for _ in range(3))
+                    for _ in range(2)]
 
-        def e2e_fn(i, t, left):
-            return sp.ulysses_attention_distributed(t[0], t[1], t[2], shape, a2a,
-                                                    rank=e2e_ranks[i])
-    pipe = sp.StepPipeline(e2e_bufs, e2e_fn, dev)
+        def e2e_fn(k, t, left):
+            return sp.ulysses_attention_distributed(t[0], t[1], t[2], gshape, a2a,
+                                                    rank=e2e_ranks[k])
+    pipe = sp.StepPipeline(e2e_bufs, e2e_fn, dev, head_groups=groups)
     for _ in range(2):
         pipe.submit((hq, hk, hv), ho)
     pipe.synchronize()
@@ -369,7 +377,10 @@ def run_ulysses(args):
                         "d2h_bytes_per_step": int(shard_bytes),
                         "ms_per_step": te / args.steps,
                         "how": "StepPipeline: H2D, the rank's step and D2H on three streams, "
-                               "two rank objects taking turns; every step moves its own bytes"},
+                               "two rank objects taking turns"
+                               + (f", each step as {groups} groups of {shape.H // groups} heads"
+                                  if groups > 1 else "")
+                               + "; every step moves its own bytes"},
                 "gpu_launches": int(launches), "clocks": clocks,
                 "roofline": {"bound": "tensor", "kernel": "whole step per GPU",
                              "achieved": per_gpu, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",

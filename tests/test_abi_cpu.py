@@ -239,6 +239,9 @@ def test_pipeline_head_groups():
     assert g(sp.Shape(1, 32760, 12, 128, 2)) == 1      # 11 waves: any split adds one
     assert g(sp.Shape(1, 124992, 48, 128, 8)) == 3
     assert g(sp.Shape(1, 1000, 7, 64, 7)) == 1
+    # one rank's step of the multi-GPU form attends H/P heads on its GPU
+    assert g(sp.Shape(1, 75600, 40, 128, 8), gpus=8) == 5    # 1 head a rank, 2 waves each
+    assert g(sp.Shape(1, 75600, 40, 128, 4), gpus=4) == 5
     for H, P, N, B in ((40, 4, 75600, 1), (24, 2, 4096, 2), (16, 1, 65536, 1), (64, 8, 99999, 1)):
         shp = sp.Shape(B, N, H, 128, P)
         G = g(shp)

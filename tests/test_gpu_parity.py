@@ -442,12 +442,14 @@ def test_rank_classes_in_a_one_member_nccl_group(kv_exchange):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("kind", ["nccl", "peer-push", "peer-nccl"])
+@pytest.mark.parametrize("kind", ["nccl", "nccl-groups", "peer-push", "peer-nccl"])
 def test_step_pipeline_in_a_one_member_nccl_group(kind):
     """StepPipeline over the multi-GPU forms (two rank objects taking turns;
     H2D, the step and D2H on three streams; the peer form's closing
-    all-reduce waits for the previous output's copy back): five steps on two
-    alternating host problems give the fused call's outputs bit for bit."""
+    all-reduce waits for the previous output's copy back; "nccl-groups" runs
+    each step as two groups of two heads, a rank object per set and group):
+    five steps on two alternating host problems give the fused call's outputs
+    bit for bit."""
     import torch.distributed as dist
     B, N, H, D = 1, 1000, 4, 128
     shape = sp.Shape(B, N, H, D, 1)
@@ -463,6 +465,7 @@ def test_step_pipeline_in_a_one_member_nccl_group(kind):
     try:
         def dev_shard():
             return torch.empty(shape.rank_shard, dtype=torch.bfloat16, device="cuda")
+        groups = 1
         if kind == "nccl":
             ranks = [sp.UlyssesRank(shape) for _ in range(2)]
             a2a = sp.nccl_all_to_all()
@@ -470,13 +473,24 @@ def test_step_pipeline_in_a_one_member_nccl_group(kind):
 
             def fn(i, t, left):
                 return sp.ulysses_attention_distributed(t[0], t[1], t[2], shape, a2a, rank=ranks[i])
+        elif kind == "nccl-groups":
+            groups = 2
+            gshape = sp.Shape(B, N, H // groups, D, 1)
+            ranks = [sp.UlyssesRank(gshape) for _ in range(2 * groups)]
+            a2a = sp.nccl_all_to_all()
+            bufs = [tuple(torch.empty((groups,) + gshape.rank_shard, dtype=torch.bfloat16,
+                                      device="cuda") for _ in range(3)) for _ in range(2)]
+
+            def fn(k, t, left):
+                return sp.ulysses_attention_distributed(t[0], t[1], t[2], gshape, a2a,
+                                                        rank=ranks[k])
         else:
             ranks = [sp.UlyssesPeerRank(shape, kv_exchange=kind.split("-")[1]) for _ in range(2)]
             bufs = [(r.q_shard, dev_shard(), dev_shard()) for r in ranks]
 
             def fn(i, t, left):
                 return ranks[i].step(t[1], t[2], release_after=left)
-        pipe = sp.StepPipeline(bufs, fn)
+        pipe = sp.StepPipeline(bufs, fn, head_groups=groups)
         outs = [torch.empty(shape.rank_shard, dtype=torch.bfloat16).pin_memory() for _ in range(5)]
         for j in range(5):
             pipe.submit(probs[j % 2][0], outs[j])
@@ -485,7 +499,7 @@ def test_step_pipeline_in_a_one_member_nccl_group(kind):
             want = probs[j % 2][1]
             got = outs[j].view(torch.int16).numpy().view(np.uint16)
             assert np.array_equal(got.reshape(want.shape), want), j
-        if kind != "nccl":
+        if kind.startswith("peer"):
             for r in ranks:
                 r.close()
         _status_ok()

@@ -868,23 +868,32 @@ class StepPipeline:
     or one rank's step of the multi-GPU forms (UlyssesRank, UlyssesPeerRank).
 
     inputs: per buffer set, the device tensors a step reads (depth =
-    len(inputs)).  step(i, tensors, previous_out_left) enqueues the step on
-    the current stream (the pipeline's compute stream) for buffer set i and
+    len(inputs)).  step(k, tensors, previous_out_left) enqueues the step on
+    the current stream (the pipeline's compute stream) for buffer set k and
     returns its device output: a buffer of its own that stays valid until the
     next step on the same set, or a fresh tensor; previous_out_left is the
-    CUDA event that marks the previous
-    step's output as copied back (None for the first), which a step whose
-    output buffers other ranks write passes on (UlyssesPeerRank's
-    release_after).  submit(host_inputs, host_output) copies the pinned host
-    tensors into the next set on an H2D stream, runs the step once they have
-    arrived, and copies its output into host_output on a D2H stream.  A set
-    is reused only after its last output has left, so step i+1's inputs
-    travel while step i computes and step i's output travels while step i+1
-    computes.  Nothing here synchronises the host; synchronize() waits for
-    everything submitted.  Collectives inside the step run on the compute
-    stream, in submission order on every rank."""
+    CUDA event that marks the previous step's output as copied back (None for
+    the first), which a step whose output buffers other ranks write passes on
+    (UlyssesPeerRank's release_after).  submit(host_inputs, host_output)
+    copies the pinned host tensors into the next set on an H2D stream, runs
+    the step once they have arrived, and copies its output into host_output
+    on a D2H stream.  A set is reused only after its last output has left, so
+    step i+1's inputs travel while step i computes and step i's output
+    travels while step i+1 computes.  Nothing here synchronises the host;
+    synchronize() waits for everything submitted.  Collectives inside the
+    step run on the compute stream, in submission order on every rank.
 
-    def __init__(self, inputs, step, device=None):
+    head_groups G > 1 runs every step as G problems of H/G heads, which
+    attention allows because heads are independent: the host tensors hold
+    rows of H heads of D elements ([..][H][D], bf16), each input of a set is
+    [G][..][H/G][D] (one part per group), and group g's H/G heads are copied
+    in (sp_copy_heads), stepped, and copied out while the next group's copy
+    and step run.  Only one group's transfers then lie outside the compute of
+    a run of steps.  The step is called with k = set * G + g on group g's
+    parts, so it can keep state (a rank object, say) per set and group; its
+    output is [..][H/G][D].  Every rank calls the groups in the same order."""
+
+    def __init__(self, inputs, step, device=None, head_groups: int = 1):
         torch = _torch()
         self.inputs = [tuple(t) for t in inputs]
         self.step = step
@@ -892,7 +901,16 @@ class StepPipeline:
         self.h2d = torch.cuda.Stream(self.device)
         self.compute = torch.cuda.Stream(self.device)
         self.d2h = torch.cuda.Stream(self.device)
-        self.freed = [None] * len(self.inputs)   # event: the set's last output has left
+        self.head_groups = int(head_groups)
+        if self.head_groups < 1:
+            raise ValueError("head_groups must be at least 1")
+        if self.head_groups > 1:
+            for t in (x for st in self.inputs for x in st):
+                if t.dim() < 3 or t.shape[0] != self.head_groups:
+                    raise ValueError(f"grouped inputs are [{self.head_groups}][..][H/G][D], "
+                                     f"got {tuple(t.shape)}")
+        # per set and group: the event that marks its last output as copied back
+        self.freed = [[None] * self.head_groups for _ in self.inputs]
         self.last_out_left = None
         self.count = 0
 
@@ -903,26 +921,39 @@ class StepPipeline:
         dev = self.inputs[i]
         if len(host_inputs) != len(dev):
             raise ValueError(f"{len(host_inputs)} host inputs for {len(dev)} device buffers")
-        if self.freed[i] is not None:
-            self.h2d.wait_event(self.freed[i])
-        with torch.cuda.stream(self.h2d):
-            for d, h in zip(dev, host_inputs):
-                d.copy_(h, non_blocking=True)
-        arrived = torch.cuda.Event()
-        arrived.record(self.h2d)
-        self.compute.wait_event(arrived)
-        with torch.cuda.stream(self.compute):
-            out = self.step(i, dev, self.last_out_left)
-        done = torch.cuda.Event()
-        done.record(self.compute)
-        self.d2h.wait_event(done)
-        with torch.cuda.stream(self.d2h):
-            host_output.copy_(out, non_blocking=True)
-        out.record_stream(self.d2h)   # a fresh output stays allocated until it has left
-        left = torch.cuda.Event()
-        left.record(self.d2h)
-        self.freed[i] = self.last_out_left = left
-        return left
+        G = self.head_groups
+        for g in range(G):
+            if self.freed[i][g] is not None:
+                self.h2d.wait_event(self.freed[i][g])
+            parts = tuple(d[g] for d in dev) if G > 1 else dev
+            with torch.cuda.stream(self.h2d):
+                for d, h in zip(parts, host_inputs):
+                    if G > 1:
+                        hg, D = d.shape[-2], d.shape[-1]
+                        copy_heads(d, hg, 0, h, G * hg, g * hg, d.numel() // (hg * D), hg, D,
+                                   stream=self.h2d)
+                    else:
+                        d.copy_(h, non_blocking=True)
+            arrived = torch.cuda.Event()
+            arrived.record(self.h2d)
+            self.compute.wait_event(arrived)
+            with torch.cuda.stream(self.compute):
+                out = self.step(i * G + g, parts, self.last_out_left)
+            done = torch.cuda.Event()
+            done.record(self.compute)
+            self.d2h.wait_event(done)
+            with torch.cuda.stream(self.d2h):
+                if G > 1:
+                    hg, D = out.shape[-2], out.shape[-1]
+                    copy_heads(host_output, G * hg, g * hg, out, hg, 0, out.numel() // (hg * D),
+                               hg, D, stream=self.d2h)
+                else:
+                    host_output.copy_(out, non_blocking=True)
+            out.record_stream(self.d2h)   # a fresh output stays allocated until it has left
+            left = torch.cuda.Event()
+            left.record(self.d2h)
+            self.freed[i][g] = self.last_out_left = left
+        return self.last_out_left
 
     def synchronize(self):
         """Waits for everything submitted, then checks the device status word
@@ -932,17 +963,19 @@ class StepPipeline:
         _check(device_status(self.compute), "StepPipeline")
 
 
-def pipeline_head_groups(shape: Shape, sms: int = 148, max_groups: int = 8) -> int:
-    """Head groups per step for HostPipeline: the largest G <= max_groups
-    with P | H/G whose G fused calls of H/G heads run no more waves than one
-    call over all H heads (the fused kernel keeps one CTA on each of `sms`
-    SMs and launches ceil(Np/256) * B CTAs per head)."""
+def pipeline_head_groups(shape: Shape, sms: int = 148, max_groups: int = 8, gpus: int = 1) -> int:
+    """Head groups per step for a StepPipeline: the largest G <= max_groups
+    with P | H/G whose G calls of H/G heads run no more waves than one call
+    over all H heads.  The attention kernel keeps one CTA on each of `sms` SMs
+    and launches ceil(Np/256) * B CTAs per head; each of `gpus` GPUs attends
+    1/gpus of a call's heads (1 for the one-GPU fused call, P for one rank's
+    step of the multi-GPU form)."""
     per_head = -(-shape.Np // 256) * shape.B
-    one = -(-shape.H * per_head // sms)
+    one = -(-(shape.H // gpus) * per_head // sms)
     best = 1
     for g in range(2, max_groups + 1):
         if shape.H % g == 0 and (shape.H // g) % shape.P == 0 and \
-                g * -(-(shape.H // g) * per_head // sms) <= one:
+                g * -(-(shape.H // g // gpus) * per_head // sms) <= one:
             best = g
     return best
 
@@ -954,14 +987,10 @@ class HostPipeline(StepPipeline):
     submit(hq, hk, hv, ho) takes pinned host tensors in the sequence-sharded
     layout ([P][B][Nl][H][D] bf16) and enqueues, on three streams: the copy of
     the inputs into one of `depth` device buffer sets, the fused attention on
-    that set, and the copy of the output back into `ho`.
-
-    Heads are independent, so a step runs as `head_groups` problems of H/G
-    heads each (P | H/G; default pipeline_head_groups): group g's inputs are
-    copied in (sp_copy_heads), attended and copied out while the other groups'
-    copies run, so that only one group's input and output transfers lie
-    outside the compute of a run of steps instead of the whole step's.  Each
-    group's output is bit-identical to the same heads of one call over all H."""
+    that set, and the copy of the output back into `ho`.  A step runs as
+    `head_groups` problems of H/G heads (P | H/G; default
+    pipeline_head_groups), each group's output bit-identical to the same
+    heads of one call over all H."""
 
     def __init__(self, shape: Shape, device=None, depth: int = 2, head_groups: int = 0):
         torch = _torch()
@@ -974,52 +1003,23 @@ class HostPipeline(StepPipeline):
         if g < 1 or shape.H % g or (shape.H // g) % shape.P:
             raise ValueError(f"{g} head groups: need G | H and P | H/G "
                              f"(H = {shape.H}, P = {shape.P})")
-        self.head_groups = g
-        self.group_shape = Shape(shape.B, shape.N, shape.H // g, shape.D, shape.P, shape.scale)
-        gs = (g,) + self.group_shape.seq_sharded
-        sets = [tuple(torch.empty(gs, dtype=torch.bfloat16, device=dev) for _ in range(4))
+        gshape = Shape(shape.B, shape.N, shape.H // g, shape.D, shape.P, shape.scale)
+        self.group_shape = gshape
+        part = ((g,) if g > 1 else ()) + gshape.seq_sharded
+        sets = [tuple(torch.empty(part, dtype=torch.bfloat16, device=dev) for _ in range(4))
                 for _ in range(depth)]
         self._outs = [st[3] for st in sets]
-        # per buffer set and group: the event that marks its output as copied back
-        self._group_freed = [[None] * g for _ in range(depth)]
 
-        def fused(i, t, _left):
-            attention_seqsharded(t[0], t[1], t[2], self._outs[i][0], shape,
+        def fused(k, t, _left):
+            o = self._outs[k // g]
+            o = o[k % g] if g > 1 else o
+            attention_seqsharded(t[0], t[1], t[2], o, gshape,
                                  stream=torch.cuda.current_stream(dev))
-            return self._outs[i][0]
-        # the whole-step path (one group) sees each set as its [P][B][Nl][H][D] views
-        super().__init__([tuple(x[0] if g == 1 else x for x in st[:3]) for st in sets],
-                         fused, dev)
+            return o
+        super().__init__([st[:3] for st in sets], fused, dev, head_groups=g)
 
     def submit(self, hq, hk, hv, ho):
-        if self.head_groups == 1:
-            return super().submit((hq, hk, hv), ho)
-        torch = _torch()
-        i = self.count % len(self.inputs)
-        self.count += 1
-        q, k, v = self.inputs[i]
-        o = self._outs[i]
-        sh, gs = self.shape, self.group_shape
-        rows, hg = sh.P * sh.B * sh.Nl, gs.H
-        left = None
-        for g in range(self.head_groups):
-            if self._group_freed[i][g] is not None:
-                self.h2d.wait_event(self._group_freed[i][g])
-            for d, h in ((q, hq), (k, hk), (v, hv)):
-                copy_heads(d[g], hg, 0, h, sh.H, g * hg, rows, hg, sh.D, stream=self.h2d)
-            arrived = torch.cuda.Event()
-            arrived.record(self.h2d)
-            self.compute.wait_event(arrived)
-            attention_seqsharded(q[g], k[g], v[g], o[g], gs, stream=self.compute)
-            done = torch.cuda.Event()
-            done.record(self.compute)
-            self.d2h.wait_event(done)
-            copy_heads(ho, sh.H, g * hg, o[g], hg, 0, rows, hg, sh.D, stream=self.d2h)
-            left = torch.cuda.Event()
-            left.record(self.d2h)
-            self._group_freed[i][g] = left
-        self.freed[i] = self.last_out_left = left
-        return left
+        return super().submit((hq, hk, hv), ho)
 
 
 def device_status(stream=None, device=None) -> int:
