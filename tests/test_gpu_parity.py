@@ -1175,13 +1175,14 @@ def test_host_pipeline_matches_direct_calls():
         assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), want)
 
 
-@pytest.mark.parametrize("groups", [1, 2, 4])
-def test_host_pipeline_in_head_groups(groups):
+@pytest.mark.parametrize("B,N,H,D,P,groups", [
+    (1, 1100, 8, 128, 2, 1), (1, 1100, 8, 128, 2, 2), (1, 1100, 8, 128, 2, 4),
+    (2, 777, 6, 64, 3, 2)])
+def test_host_pipeline_in_head_groups(B, N, H, D, P, groups):
     """HostPipeline moving and attending one group of heads at a time
     (sp_copy_heads in and out, one fused call of H/G heads per group): five
     problems through two buffer sets, each bit-identical to the direct call
-    over all H heads."""
-    B, N, H, D, P = 1, 1100, 8, 128, 2
+    over all H heads (B > 1, ragged N and D = 64 included)."""
     shape = sp.Shape(B, N, H, D, P)
     pipe = sp.HostPipeline(shape, depth=2, head_groups=groups)
     assert pipe.head_groups == groups
